@@ -1,0 +1,551 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 MSDeformAttn core: queries/s and achieved HBM GB/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
+
+One step = one pass of the whole hot path over one batch: the forward
+(msda_forward) and the training backward (msda_backward) of the encoder
+training workload -- B=4, M=8, D=32, K=4, L=4, levels (100,150),(50,75),
+(25,38),(13,19), S = Lq = 19947, float32 -- on seeded synthetic inputs.  The
+unit is a query (one (b, q) pair), so a step processes B*Lq = 79,788 queries.
+
+Timing: inputs are resident in HBM; L2 (126 MB) is flushed by a 256 MiB write
+before every step, outside the timed events; each step is bracketed by CUDA
+events on the launching stream; W untimed warm-up steps come first.  With
+N > 1 (torchrun, one process per GPU) every rank runs the same workload on its
+own GPU -- the operator has no exchange step, so ranks are replicas ("weak"
+scaling) -- and the step time is the max over ranks.
+
+Printed (rank 0, one JSON line): the contract keys, plus
+  roofline       the dominant launch: algorithmic bytes / its mean event time,
+                 against the measured HBM copy bandwidth of this machine's B200s;
+  forward_encoder the encoder self-attention forward (B=2, S=Lq=19947), timed
+                 alone the same way, with its own roofline;
+  e2e            the same metric through the public API with host buffers: the
+                 H2D copy of every input and the D2H copy of every result are
+                 inside the timed region;
+  cpu_baseline   the float64 CPU oracle on a bounded sample (rank 0, N=1);
+  clocks         SM clocks and throttle reasons sampled during the timed region.
+
+``--impl reference`` times the float64 oracle instead (the deliberately slow
+reference arm; rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from scale_deformable_attention_backward_b200 import workloads as W  # noqa: E402
+
+STEP_WORKLOAD = "encoder_train_fp32"
+FORWARD_WORKLOAD = "encoder_fp32"
+METRIC = "MSDeformAttn fwd/bwd queries/sec and achieved HBM GB/s vs B200 peak (1 GPU)"
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20
+KERNEL_SOURCES = os.path.join(ROOT, "scale_deformable_attention_backward_b200", "csrc")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+# ---------------------------------------------------------------------------
+# algorithmic bytes (compulsory HBM traffic) per launch
+# ---------------------------------------------------------------------------
+
+def algorithmic_bytes(cfg: W.Config, inp: W.Inputs) -> dict:
+    """Compulsory bytes: every input read once and every output written once."""
+    B, S, M, D = inp.value.shape
+    _, Lq, _, L, K, _ = inp.sampling_locations.shape
+    vbytes = 2 if cfg.dtype == "bf16" else 4
+    value = B * S * M * D * vbytes
+    loc = B * Lq * M * L * K * 2 * 4
+    attn = B * Lq * M * L * K * 4
+    out = B * Lq * M * D * vbytes
+    fwd = value + loc + attn + out
+    # backward reads value, loc, attn, grad_output; writes grad_value, grad_loc, grad_attn
+    bwd = value + loc + attn + B * Lq * M * D * 4 + B * S * M * D * 4 + loc + attn
+    return {"forward": fwd, "backward": bwd}
+
+
+def source_digest() -> str:
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(KERNEL_SOURCES)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(KERNEL_SOURCES, name), "rb") as f:
+                h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(key: str):
+    """ncu DRAM bytes per launch recorded for the current kernel sources, or None."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f).get(key)
+    except (OSError, ValueError):
+        return None
+    if not rec or rec.get("source_digest") != source_digest():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, ValueError, KeyError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+        return False
+
+    def summary(self):
+        rows = []
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, flags in rows for i, v in enumerate(flags)
+                          if v.lower() == "active"})
+        top = max(r[0] for r in rows)
+        loaded = [r[0] for r in rows if r[0] >= 0.5 * top] or [r[0] for r in rows]
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": rows[0][1],
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle on a bounded sample (cpu_baseline and the reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_sample(cfg: W.Config, target_s: float = 12.0, per_step_target_s=None):
+    """Time the float64 oracle (single thread, as it stands) on the first n
+    queries of every image of ``cfg``, forward + backward, with n grown until the
+    timed call takes about ``target_s``.  Returns (queries/s, description)."""
+    import oracle  # test infrastructure: used here only for the CPU baseline
+    inp = W.make_inputs(cfg, seed=0, with_grad=True)
+    orc = oracle.default()
+    n = 64
+    while True:
+        sub = W.select_queries(inp, np.arange(n))
+        t0 = time.perf_counter()
+        orc.forward(sub.value, sub.spatial_shapes, sub.level_start_index,
+                    sub.sampling_locations, sub.attention_weights)
+        orc.backward(sub.value, sub.spatial_shapes, sub.level_start_index,
+                     sub.sampling_locations, sub.attention_weights, sub.grad_output)
+        dt = time.perf_counter() - t0
+        target = per_step_target_s if per_step_target_s is not None else target_s
+        if dt >= 0.5 * target or n >= cfg.queries:
+            break
+        n = min(cfg.queries, max(2 * n, int(n * 0.8 * target / max(dt, 1e-3))))
+    queries = cfg.B * n
+    desc = (f"{cfg.name}: forward + backward of the first {n} of {cfg.queries} queries of "
+            f"each of the B={cfg.B} images (value over all {cfg.S} tokens), float64 oracle, "
+            f"single thread, {dt:.2f} s")
+    return queries / dt, desc, dt
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# the B200 arm
+# ---------------------------------------------------------------------------
+
+def _device_inputs(inp, device):
+    import torch
+    d = {
+        "value": torch.from_numpy(inp.value).to(device),
+        "spatial_shapes": torch.from_numpy(inp.spatial_shapes).to(device),
+        "level_start_index": torch.from_numpy(inp.level_start_index).to(device),
+        "sampling_locations": torch.from_numpy(inp.sampling_locations).to(device),
+        "attention_weights": torch.from_numpy(inp.attention_weights).to(device),
+    }
+    if inp.grad_output is not None:
+        d["grad_output"] = torch.from_numpy(inp.grad_output).to(device)
+    return d
+
+
+def run_b200(args, world, rank, local):
+    import torch
+    from scale_deformable_attention_backward_b200 import binding
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    stream = torch.cuda.current_stream(device)
+    cfg = W.CONFIGS[STEP_WORKLOAD]
+    inp = W.make_inputs(cfg, seed=0)
+    d = _device_inputs(inp, device)
+    B, S, M, D = inp.value.shape
+    _, Lq, _, L, K, _ = inp.sampling_locations.shape
+    out = torch.empty((B, Lq, M * D), dtype=torch.float32, device=device)
+    gv = torch.empty_like(d["value"])
+    gl = torch.empty_like(d["sampling_locations"])
+    ga = torch.empty_like(d["attention_weights"])
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+
+    def step():
+        binding.forward(d["value"], d["spatial_shapes"], d["level_start_index"],
+                        d["sampling_locations"], d["attention_weights"], output=out)
+
+    def step_bwd():
+        binding.backward(d["value"], d["spatial_shapes"], d["level_start_index"],
+                         d["sampling_locations"], d["attention_weights"], d["grad_output"],
+                         grad_value=gv, grad_sampling_locations=gl, grad_attention_weights=ga)
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        step()
+        step_bwd()
+    torch.cuda.synchronize()
+
+    e0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e2 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    with ClockSampler(local) as clocks:
+        for i in range(args.steps):
+            flush.fill_(float(i))
+            e0[i].record(stream)
+            step()
+            e1[i].record(stream)
+            step_bwd()
+            e2[i].record(stream)
+        torch.cuda.synchronize()
+    wall = time.perf_counter() - wall0
+    barrier(world)
+    fwd_ms = [a.elapsed_time(b) for a, b in zip(e0, e1)]
+    bwd_ms = [a.elapsed_time(b) for a, b in zip(e1, e2)]
+    total_ms = sum(f + b for f, b in zip(fwd_ms, bwd_ms))
+    total_ms_max = max_over_ranks(total_ms, world, device)
+    ms_per_step = total_ms_max / args.steps
+    queries = B * Lq
+    value = world * queries * args.steps / (total_ms_max / 1e3)
+
+    peak, peak_kind = measured_peak()
+    algo = algorithmic_bytes(cfg, inp)
+    f_ms, b_ms = statistics.mean(fwd_ms), statistics.mean(bwd_ms)
+    dom, dom_ms = ("backward", b_ms) if b_ms >= f_ms else ("forward", f_ms)
+    achieved = algo[dom] / (dom_ms * 1e-3) / 1e9
+    roofline = {
+        "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+        "frac": round(achieved / peak, 4), "traffic": recorded_traffic(f"{STEP_WORKLOAD}.{dom}"),
+        "kernel": ("msda_backward: zero_kernel + backward_kernel" if dom == "backward"
+                   else "msda_forward: forward_kernel"),
+        "algorithmic_bytes": algo[dom], "mean_ms": round(dom_ms, 4),
+        "peak_source": f"{peak_kind} HBM copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
+                       if peak_kind == "measured" else "fallback 6.65 TB/s",
+        "other": {
+            "forward": {"mean_ms": round(f_ms, 4), "algorithmic_bytes": algo["forward"],
+                        "achieved_gbs": round(algo["forward"] / (f_ms * 1e-3) / 1e9, 1),
+                        "frac": round(algo["forward"] / (f_ms * 1e-3) / 1e9 / peak, 4),
+                        "traffic": recorded_traffic(f"{STEP_WORKLOAD}.forward")},
+            "backward": {"mean_ms": round(b_ms, 4), "algorithmic_bytes": algo["backward"],
+                         "achieved_gbs": round(algo["backward"] / (b_ms * 1e-3) / 1e9, 1),
+                         "frac": round(algo["backward"] / (b_ms * 1e-3) / 1e9 / peak, 4),
+                         "traffic": recorded_traffic(f"{STEP_WORKLOAD}.backward")},
+        },
+    }
+
+    # The encoder self-attention forward alone (B=2), the spec workload.
+    fcfg = W.CONFIGS[FORWARD_WORKLOAD]
+    finp = W.make_inputs(fcfg, seed=0)
+    fd = _device_inputs(finp, device)
+    fout = torch.empty((fcfg.B, fcfg.queries, fcfg.M * fcfg.D), dtype=torch.float32,
+                       device=device)
+
+    def fstep():
+        binding.forward(fd["value"], fd["spatial_shapes"], fd["level_start_index"],
+                        fd["sampling_locations"], fd["attention_weights"], output=fout)
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        fstep()
+    fe0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    fe1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        fe0[i].record(stream)
+        fstep()
+        fe1[i].record(stream)
+    torch.cuda.synchronize()
+    fms = statistics.mean(a.elapsed_time(b) for a, b in zip(fe0, fe1))
+    fms = max_over_ranks(fms, world, device)
+    fbytes = algorithmic_bytes(fcfg, finp)["forward"]
+    fach = fbytes / (fms * 1e-3) / 1e9
+    forward_encoder = {
+        "workload": fcfg.description, "queries": fcfg.B * fcfg.queries,
+        "ms": round(fms, 4), "queries_per_s": round(fcfg.B * fcfg.queries / (fms * 1e-3), 1),
+        "roofline": {"bound": "hbm", "achieved": round(fach, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(fach / peak, 4),
+                     "traffic": recorded_traffic(f"{FORWARD_WORKLOAD}.forward"),
+                     "algorithmic_bytes": fbytes},
+    }
+
+    # End to end through the public API with host buffers.
+    pin = {k: torch.from_numpy(getattr(inp, k)).pin_memory() for k in
+           ("value", "sampling_locations", "attention_weights", "grad_output")}
+    host_out = {k: torch.empty(t.shape, dtype=t.dtype).pin_memory() for k, t in
+                (("out", out), ("gv", gv), ("gl", gl), ("ga", ga))}
+    h2d = sum(t.numel() * t.element_size() for t in pin.values()) + \
+        inp.spatial_shapes.nbytes + inp.level_start_index.nbytes
+    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+    ss_host = torch.from_numpy(inp.spatial_shapes)
+    st_host = torch.from_numpy(inp.level_start_index)
+    e2e_steps = max(3, min(args.steps, 20))
+
+    def e2e_step():
+        dv = pin["value"].to(device, non_blocking=True)
+        dl = pin["sampling_locations"].to(device, non_blocking=True)
+        da = pin["attention_weights"].to(device, non_blocking=True)
+        dg = pin["grad_output"].to(device, non_blocking=True)
+        dss = ss_host.to(device, non_blocking=True)
+        dst = st_host.to(device, non_blocking=True)
+        o = binding.forward(dv, dss, dst, dl, da)
+        g = binding.backward(dv, dss, dst, dl, da, dg)
+        for (k, src) in zip(("out", "gv", "gl", "ga"), (o,) + tuple(g)):
+            host_out[k].copy_(src, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    ee0 = torch.cuda.Event(enable_timing=True)
+    ee1 = torch.cuda.Event(enable_timing=True)
+    ee0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    ee1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(ee0.elapsed_time(ee1), world, device) / e2e_steps
+    barrier(world)
+
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": "queries/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded numpy; no dataset)",
+        "config": {"workload": cfg.description, "step": "msda_forward + msda_backward",
+                   "queries_per_step_per_gpu": queries, "parallelism": f"replicas x{world}",
+                   "l2": "flushed before every step by a 256 MiB write (outside the timed events)",
+                   "timing": "CUDA events per step on the launching stream, max over ranks"},
+        "roofline": roofline,
+        "forward_encoder": forward_encoder,
+        "e2e": {"value": round(world * queries / (e2e_ms * 1e-3), 1), "unit": "queries/s",
+                "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(d2h)},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks.summary(),
+        "wall_s_timed_region": round(wall, 3),
+        "cpu_baseline": None,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        qps, desc, _ = oracle_sample(cfg)
+        result["cpu_baseline"] = {"value": round(qps, 2), "unit": "queries/s", "cores": 1,
+                                  "kind": "oracle", "sample": desc}
+    return result
+
+
+def run_case(args, local):
+    """One launch type alone (for profiler captures): W + K launches with an L2
+    flush before each, and a one-line JSON with the mean event time."""
+    import torch
+    from scale_deformable_attention_backward_b200 import binding
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    name = FORWARD_WORKLOAD if args.case == "forward_encoder" else STEP_WORKLOAD
+    cfg = W.CONFIGS[name]
+    inp = W.make_inputs(cfg, seed=0, with_grad=args.case == "backward")
+    d = _device_inputs(inp, device)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+
+    def launch():
+        if args.case == "backward":
+            binding.backward(d["value"], d["spatial_shapes"], d["level_start_index"],
+                             d["sampling_locations"], d["attention_weights"], d["grad_output"])
+        else:
+            binding.forward(d["value"], d["spatial_shapes"], d["level_start_index"],
+                            d["sampling_locations"], d["attention_weights"])
+
+    times = []
+    for i in range(args.warmup + args.steps):
+        flush.fill_(float(i))
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        launch()
+        b.record()
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            times.append(a.elapsed_time(b))
+    return {"case": args.case, "workload": cfg.description,
+            "ms": round(statistics.mean(times), 4), "launches": args.warmup + args.steps}
+
+
+def run_reference(args):
+    """The reference arm: the float64 oracle as it stands, on the host cores."""
+    cfg = W.CONFIGS[STEP_WORKLOAD]
+    budget = 150.0
+    per_step = max(0.5, min(10.0, budget / max(1, args.steps + args.warmup)))
+    qps, desc, dt = oracle_sample(cfg, per_step_target_s=per_step)
+    # Warm-up and timed steps on the calibrated sample size.
+    import oracle
+    n = int(round(qps * dt / cfg.B))
+    inp = W.select_queries(W.make_inputs(cfg, seed=0, with_grad=True), np.arange(n))
+    orc = oracle.default()
+
+    def step():
+        orc.forward(inp.value, inp.spatial_shapes, inp.level_start_index,
+                    inp.sampling_locations, inp.attention_weights)
+        orc.backward(inp.value, inp.spatial_shapes, inp.level_start_index,
+                     inp.sampling_locations, inp.attention_weights, inp.grad_output)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    total = time.perf_counter() - t0
+    ms = total / args.steps * 1e3
+    value = cfg.B * n / (ms * 1e-3)
+    sample = (f"{cfg.name}: forward + backward of the first {n} of {cfg.queries} queries of "
+              f"each of the B={cfg.B} images per step, float64 oracle, single thread")
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "queries/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded numpy; no dataset)",
+        "config": {"workload": cfg.description, "step": "oracle forward + backward",
+                   "queries_per_step": cfg.B * n},
+        "cpu_baseline": {"value": round(value, 3), "unit": "queries/s", "cores": 1,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 3), "unit": "queries/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["b200", "reference"], default="b200")
+    p.add_argument("--no-cpu-baseline", action="store_true",
+                   help="skip the CPU oracle timing (it takes ~10-20 s)")
+    p.add_argument("--case", choices=["step", "forward", "forward_encoder", "backward"],
+                   default="step",
+                   help="time one launch type alone (for profiler captures) instead of "
+                        "the full benchmark")
+    args = p.parse_args(argv)
+    if args.warmup < 3:
+        p.error("--warmup must be at least 3")
+    if args.steps < 1:
+        p.error("--steps must be at least 1")
+    return args
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return 0
+    if args.case != "step":
+        print(json.dumps(run_case(args, local)), flush=True)
+        return 0
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    try:
+        result = run_b200(args, world, rank, local)
+        if rank == 0:
+            print(json.dumps(result), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,150 @@
+/*
+ * msda.h -- C ABI of the B200 (sm_100a) multi-scale deformable attention core
+ * (MSDeformAttn): forward and training backward.
+ *
+ * The operator, per batch b, query q, head m and channel d:
+ *
+ *   out[b, q, m*D + d] = sum_{l < L} sum_{k < K} A[b,q,m,l,k] *
+ *                        bilinear_l(value[b, :, m, d]; loc[b,q,m,l,k])
+ *
+ * "Deformable DETR Deformable Transformers for End-to-End Object Detection"
+ * (paper notes), 核心洞察 2, multi-scale deformable attention equation -- the part
+ * inside the per-head output projection W_m, with the value projection W'_m
+ * already applied to `value`.  The sampling rule is the one of
+ * "Deformable DETR模型解读（附源码+论文）", ms_deform_attn_core_pytorch: level l is
+ * the row-major H_l x W_l block of `value` starting at token
+ * level_start_index[l]; location component 0 is x (scaled by W_l), component 1
+ * is y (scaled by H_l); the pixel coordinate is x = loc_x * W_l - 0.5 (grid_sample,
+ * align_corners=False, grid = 2*loc - 1); the four corners floor(x) + {0,1} x
+ * floor(y) + {0,1} are weighted bilinearly and a corner outside the map reads
+ * zero (padding_mode='zeros').  The call interface mirrors
+ * MSDeformAttnFunction.apply(value, spatial_shapes, level_start_index,
+ * sampling_locations, attention_weights, im2col_step) of
+ * "Deformable DETR模型解读", MultiScaleDeformableAttention.forward (im2col_step,
+ * a batching knob of that implementation, does not change the result and has
+ * no counterpart here).
+ *
+ * Conventions for every entry point
+ *  - All tensor arguments are DEVICE pointers to contiguous row-major arrays
+ *    owned by the caller.  The library allocates nothing and keeps no state
+ *    between calls.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Work is enqueued asynchronously on it; results are ready once the stream
+ *    has been synchronised.
+ *  - Argument errors are detected on the host, before anything is enqueued, and
+ *    returned synchronously; nothing is written in that case.  A failed launch
+ *    returns MSDA_ERR_CUDA.  A fault during kernel execution surfaces at the
+ *    caller's next synchronisation, as with any CUDA call.
+ *  - spatial_shapes / level_start_index are read on the device only (no host
+ *    synchronisation).  The kernels check each level (H, W >= 1, start >= 0,
+ *    start + H*W <= S) before use and treat a level that fails the check as
+ *    empty, so inconsistent metadata gives wrong numbers but never an
+ *    out-of-bounds access.  msda_check_metadata() validates host copies.
+ *  - Supported: value dtype float32 with D % 4 == 0, or bfloat16 with D % 8 == 0
+ *    (each lane moves 16 bytes); 1 <= L <= 16; 1 <= K <= 64; every size >= 0,
+ *    B*S*M*D and B*Lq*M*L*K*2 below 2^62, H_l and W_l below 2^22.  `value`,
+ *    `output`, `grad_output` and `grad_value` must be 16-byte aligned,
+ *    `sampling_locations` 8-byte aligned, the other arrays 4-byte aligned
+ *    (8-byte for the int64 metadata).
+ *  - B*Lq == 0 (or M == 0, or D == 0) is valid and launches nothing, except that
+ *    msda_backward still zeroes grad_value.
+ */
+#ifndef MSDA_H
+#define MSDA_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MSDA_OK = 0,
+    MSDA_ERR_NULL_POINTER = 1,  /* a required pointer is NULL                        */
+    MSDA_ERR_BAD_SHAPE = 2,     /* a size is negative or the metadata is inconsistent */
+    MSDA_ERR_UNSUPPORTED = 3,   /* dtype, D, L or K outside the supported set         */
+    MSDA_ERR_MISALIGNED = 4,    /* a pointer breaks the alignment rule above          */
+    MSDA_ERR_CUDA = 5           /* a CUDA launch or runtime call failed               */
+} msda_status;
+
+typedef enum {
+    MSDA_F32 = 0,   /* IEEE float32                                    */
+    MSDA_BF16 = 1   /* bfloat16 (raw 16-bit, round-to-nearest-even out) */
+} msda_dtype;
+
+/*
+ * Forward.  "Deformable DETR Deformable Transformers for End-to-End Object
+ * Detection", multi-scale deformable attention equation; sampling as in
+ * "Deformable DETR模型解读", ms_deform_attn_core_pytorch.
+ *
+ *   value               [B, S, M, D]        value_dtype   S = sum_l H_l * W_l
+ *   spatial_shapes      [L, 2]  int64       row l = (H_l, W_l)
+ *   level_start_index   [L]     int64       exclusive prefix sum of H_l * W_l
+ *   sampling_locations  [B, Lq, M, L, K, 2] float32       (x, y) normalised
+ *   attention_weights   [B, Lq, M, L, K]    float32       (softmax over L*K is
+ *                                                          the caller's business)
+ *   output              [B, Lq, M * D]      value_dtype   written; channel m*D + d
+ *
+ * Accumulation is float32 for both dtypes; a bfloat16 output is rounded to
+ * nearest-even from the float32 sum.
+ */
+msda_status msda_forward(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq,
+                         int64_t L, int64_t K, msda_dtype value_dtype,
+                         const void *value, const int64_t *spatial_shapes,
+                         const int64_t *level_start_index,
+                         const float *sampling_locations,
+                         const float *attention_weights, void *output,
+                         void *stream);
+
+/*
+ * Training backward: the gradients of <grad_output, forward(...)> with respect
+ * to value, sampling_locations and attention_weights.  The pages print no
+ * backward; this is the exact derivative of the forward above, taken inside the
+ * cell floor(x), floor(y) (one-sided at integer pixel coordinates), as the
+ * autograd of the grid_sample formulation in "Deformable DETR模型解读",
+ * ms_deform_attn_core_pytorch, gives it.  attention_weights are treated as
+ * inputs (the softmax before them is not differentiated).
+ *
+ *   value, spatial_shapes, level_start_index, sampling_locations,
+ *   attention_weights   as for msda_forward (value_dtype must be MSDA_F32)
+ *   grad_output              [B, Lq, M * D]        float32
+ *   grad_value               [B, S, M, D]          float32  overwritten: zeroed on
+ *                                                  `stream`, then accumulated with
+ *                                                  atomics (summation order, and so
+ *                                                  the last bits, vary run to run)
+ *   grad_sampling_locations  [B, Lq, M, L, K, 2]   float32  overwritten
+ *   grad_attention_weights   [B, Lq, M, L, K]      float32  overwritten
+ */
+msda_status msda_backward(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq,
+                          int64_t L, int64_t K, msda_dtype value_dtype,
+                          const void *value, const int64_t *spatial_shapes,
+                          const int64_t *level_start_index,
+                          const float *sampling_locations,
+                          const float *attention_weights,
+                          const float *grad_output, float *grad_value,
+                          float *grad_sampling_locations,
+                          float *grad_attention_weights, void *stream);
+
+/*
+ * Host-side metadata check, for callers that hold host copies of the metadata
+ * (the pages' layer asserts sum_l H_l * W_l == S before calling the op;
+ * "Deformable DETR模型解读", MultiScaleDeformableAttention.forward).
+ * Returns MSDA_OK if every H_l, W_l >= 1, level_start_index is the exclusive
+ * prefix sum of H_l * W_l and the total is S; MSDA_ERR_BAD_SHAPE otherwise;
+ * MSDA_ERR_NULL_POINTER for NULL arrays with L > 0.  Reads host memory only.
+ */
+msda_status msda_check_metadata(int64_t S, int64_t L,
+                                const int64_t *spatial_shapes_host,
+                                const int64_t *level_start_index_host);
+
+/* Static, NUL-terminated description of a status code. */
+const char *msda_status_string(int status);
+
+/* ABI version: major * 10000 + minor * 100 + patch. */
+int msda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MSDA_H */

@@ -28,7 +28,10 @@
  *    loc * W - 0.5.  Pixel centres sit at integer coordinates.
  *  - Each of the four bilinear corners is used only if it lies inside the map;
  *    a corner outside contributes zero (zeros padding).  A location whose
- *    coordinate is not finite has no corner inside the map.
+ *    coordinate is not finite has no corner inside the map, but its bilinear
+ *    weights are NaN: its sample -- and with it the output, grad_attn and
+ *    grad_loc of that point -- is NaN, and grad_value receives nothing from it
+ *    (this is also what grid_sample does).
  *  - The pages print no backward.  The backward is the exact derivative of the
  *    forward above, taken inside the cell [x0, x0 + 1) x [y0, y0 + 1) with
  *    x0 = floor(x), y0 = floor(y) (the one-sided derivative at integer

@@ -1,0 +1,227 @@
+"""Thin PyTorch binding of the C ABI in ``include/msda.h`` (``libmsda.so``).
+
+Argument marshalling only: tensors are checked for device, dtype, shape and
+contiguity, their device pointers and the current CUDA stream are passed to
+``msda_forward`` / ``msda_backward``, and the status code is turned into an
+exception.  Every step of the operator runs in the library's CUDA kernels;
+there is no CPU or PyTorch fallback, and a missing library is an error.
+
+Interface as in "Deformable DETR模型解读（附源码+论文）",
+MultiScaleDeformableAttention.forward: ``MSDeformAttnFunction.apply(value,
+spatial_shapes, level_start_index, sampling_locations, attention_weights,
+im2col_step)``; ``im2col_step`` is accepted and ignored (it only batches the
+work in that implementation and does not change the result).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIBRARY_PATH = os.path.join(_HERE, "libmsda.so")
+
+MSDA_F32, MSDA_BF16 = 0, 1
+_STATUS = {0: "MSDA_OK", 1: "MSDA_ERR_NULL_POINTER", 2: "MSDA_ERR_BAD_SHAPE",
+           3: "MSDA_ERR_UNSUPPORTED", 4: "MSDA_ERR_MISALIGNED", 5: "MSDA_ERR_CUDA"}
+
+# Every symbol include/msda.h declares, with its ctypes signature.
+_I64, _VP, _I32 = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int
+SIGNATURES = {
+    "msda_forward": (_I32, [_I64] * 7 + [_I32] + [_VP] * 7),
+    "msda_backward": (_I32, [_I64] * 7 + [_I32] + [_VP] * 10),
+    "msda_check_metadata": (_I32, [_I64, _I64, _VP, _VP]),
+    "msda_status_string": (ctypes.c_char_p, [_I32]),
+    "msda_version": (_I32, []),
+}
+
+
+class MSDAError(RuntimeError):
+    """A non-OK status from the C ABI, or a missing library."""
+
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        name = _STATUS.get(status, str(status))
+        msg = f"{name}"
+        if _LIB is not None:
+            msg += f" ({_LIB.msda_status_string(status).decode()})"
+        super().__init__(f"{what}: {msg}" if what else msg)
+
+
+_LIB = None
+
+
+def library() -> ctypes.CDLL:
+    """Load ``libmsda.so`` (once).  Raises if it has not been built."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIBRARY_PATH):
+            raise RuntimeError(
+                f"{LIBRARY_PATH} is missing: build it with "
+                "`python scale_deformable_attention_backward_b200/csrc/build.py` "
+                "(there is no fallback implementation)")
+        lib = ctypes.CDLL(LIBRARY_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _LIB = lib
+    return _LIB
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        raise MSDAError(status, what)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _metadata(spatial_shapes, level_start_index, S, device):
+    """Metadata as contiguous int64 device tensors.  Host tensors are checked on
+    the host (sum of H*W == S, exclusive prefix sum) before the copy."""
+    ss = torch.as_tensor(spatial_shapes)
+    st = torch.as_tensor(level_start_index)
+    if ss.dtype != torch.int64 or st.dtype != torch.int64:
+        ss, st = ss.to(torch.int64), st.to(torch.int64)
+    if ss.device.type == "cpu" and st.device.type == "cpu":
+        ss, st = ss.contiguous(), st.contiguous()
+        _check(library().msda_check_metadata(S, st.numel(), _ptr(ss), _ptr(st)),
+               "spatial_shapes / level_start_index")
+    return ss.to(device).contiguous(), st.to(device).contiguous()
+
+
+def _dims(value, sampling_locations, attention_weights):
+    if value.dim() != 4:
+        raise ValueError("value must be [B, S, M, D]")
+    B, S, M, D = value.shape
+    if sampling_locations.dim() != 6 or sampling_locations.shape[-1] != 2:
+        raise ValueError("sampling_locations must be [B, Lq, M, L, K, 2]")
+    Bq, Lq, Mq, L, K, _ = sampling_locations.shape
+    if (Bq, Mq) != (B, M):
+        raise ValueError("sampling_locations batch / head dims do not match value")
+    if tuple(attention_weights.shape) != (B, Lq, M, L, K):
+        raise ValueError("attention_weights must be [B, Lq, M, L, K]")
+    return B, S, M, D, Lq, L, K
+
+
+def _require(t: torch.Tensor, name: str, dtype, device):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (there is no CPU path)")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, value on {device}")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _value_code(value: torch.Tensor) -> int:
+    if value.dtype == torch.float32:
+        return MSDA_F32
+    if value.dtype == torch.bfloat16:
+        return MSDA_BF16
+    raise ValueError(f"value dtype {value.dtype} is not supported (float32 or bfloat16)")
+
+
+def forward(value: torch.Tensor, spatial_shapes, level_start_index,
+            sampling_locations: torch.Tensor, attention_weights: torch.Tensor,
+            im2col_step: Optional[int] = None,
+            output: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """MSDeformAttn forward: returns ``[B, Lq, M*D]`` in value's dtype."""
+    del im2col_step
+    dev = value.device
+    B, S, M, D, Lq, L, K = _dims(value, sampling_locations, attention_weights)
+    _require(value, "value", None, dev)
+    code = _value_code(value)
+    _require(sampling_locations, "sampling_locations", torch.float32, dev)
+    _require(attention_weights, "attention_weights", torch.float32, dev)
+    ss, st = _metadata(spatial_shapes, level_start_index, S, dev)
+    if ss.shape != (L, 2) or st.shape != (L,):
+        raise ValueError("spatial_shapes must be [L, 2] and level_start_index [L]")
+    if output is None:
+        output = torch.empty((B, Lq, M * D), dtype=value.dtype, device=dev)
+    else:
+        _require(output, "output", value.dtype, dev)
+        if tuple(output.shape) != (B, Lq, M * D):
+            raise ValueError("output must be [B, Lq, M*D]")
+    with torch.cuda.device(dev):
+        stream = torch.cuda.current_stream(dev).cuda_stream
+        _check(library().msda_forward(B, S, M, D, Lq, L, K, code, _ptr(value), _ptr(ss),
+                                      _ptr(st), _ptr(sampling_locations),
+                                      _ptr(attention_weights), _ptr(output),
+                                      ctypes.c_void_p(stream)), "msda_forward")
+    return output
+
+
+def backward(value: torch.Tensor, spatial_shapes, level_start_index,
+             sampling_locations: torch.Tensor, attention_weights: torch.Tensor,
+             grad_output: torch.Tensor,
+             grad_value: Optional[torch.Tensor] = None,
+             grad_sampling_locations: Optional[torch.Tensor] = None,
+             grad_attention_weights: Optional[torch.Tensor] = None,
+             ) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """MSDeformAttn backward: (grad_value, grad_sampling_locations,
+    grad_attention_weights), all float32."""
+    dev = value.device
+    B, S, M, D, Lq, L, K = _dims(value, sampling_locations, attention_weights)
+    _require(value, "value", torch.float32, dev)
+    _require(sampling_locations, "sampling_locations", torch.float32, dev)
+    _require(attention_weights, "attention_weights", torch.float32, dev)
+    _require(grad_output, "grad_output", torch.float32, dev)
+    if tuple(grad_output.shape) != (B, Lq, M * D):
+        raise ValueError("grad_output must be [B, Lq, M*D]")
+    ss, st = _metadata(spatial_shapes, level_start_index, S, dev)
+    if ss.shape != (L, 2) or st.shape != (L,):
+        raise ValueError("spatial_shapes must be [L, 2] and level_start_index [L]")
+    out = []
+    for t, shape, name in ((grad_value, (B, S, M, D), "grad_value"),
+                           (grad_sampling_locations, (B, Lq, M, L, K, 2),
+                            "grad_sampling_locations"),
+                           (grad_attention_weights, (B, Lq, M, L, K), "grad_attention_weights")):
+        if t is None:
+            t = torch.empty(shape, dtype=torch.float32, device=dev)
+        else:
+            _require(t, name, torch.float32, dev)
+            if tuple(t.shape) != shape:
+                raise ValueError(f"{name} must be {list(shape)}")
+        out.append(t)
+    gv, gl, ga = out
+    with torch.cuda.device(dev):
+        stream = torch.cuda.current_stream(dev).cuda_stream
+        _check(library().msda_backward(B, S, M, D, Lq, L, K, MSDA_F32, _ptr(value), _ptr(ss),
+                                       _ptr(st), _ptr(sampling_locations),
+                                       _ptr(attention_weights), _ptr(grad_output), _ptr(gv),
+                                       _ptr(gl), _ptr(ga), ctypes.c_void_p(stream)),
+               "msda_backward")
+    return gv, gl, ga
+
+
+class MSDeformAttnFunction(torch.autograd.Function):
+    """Autograd wrapper: forward and backward both run in libmsda.so."""
+
+    @staticmethod
+    def forward(ctx, value, spatial_shapes, level_start_index, sampling_locations,
+                attention_weights, im2col_step=None):
+        out = forward(value, spatial_shapes, level_start_index, sampling_locations,
+                      attention_weights)
+        ctx.save_for_backward(value, sampling_locations, attention_weights)
+        ctx.meta = (spatial_shapes, level_start_index)
+        return out
+
+    @staticmethod
+    def backward(ctx, grad_output):
+        value, loc, attn = ctx.saved_tensors
+        ss, st = ctx.meta
+        gv, gl, ga = backward(value, ss, st, loc, attn, grad_output.contiguous())
+        return gv, None, None, gl, ga, None
+
+
+def ms_deform_attn(value, spatial_shapes, level_start_index, sampling_locations,
+                   attention_weights, im2col_step=None):
+    """Differentiable MSDeformAttn core (value float32 for the backward)."""
+    return MSDeformAttnFunction.apply(value, spatial_shapes, level_start_index,
+                                      sampling_locations, attention_weights, im2col_step)

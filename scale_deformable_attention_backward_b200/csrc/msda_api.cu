@@ -1,0 +1,210 @@
+// msda_api.cu -- the C ABI declared in include/msda.h: argument validation on
+// the host, then one launch sequence on the caller's stream.  No allocation,
+// no state, no host synchronisation (except the opt-in MSDA_VALIDATE=1 check,
+// which copies the two small metadata arrays to the host).
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <cuda_runtime.h>
+
+#include "msda.h"
+#include "msda_launch.h"
+
+namespace {
+
+constexpr int64_t kLimit = int64_t(1) << 62;
+
+// a * b * ... without overflow; false if the product reaches kLimit.
+bool product_ok(std::initializer_list<int64_t> xs, int64_t* out) {
+  int64_t p = 1;
+  for (int64_t x : xs) {
+    if (x == 0) {
+      *out = 0;
+      return true;
+    }
+  }
+  for (int64_t x : xs) {
+    if (p > kLimit / x) return false;
+    p *= x;
+  }
+  *out = p;
+  return true;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+int pow2_at_least(int64_t n) {
+  int p = 1;
+  while (p < n && p < 32) p <<= 1;
+  return p;
+}
+
+bool validate_env() {
+  static const bool on = [] {
+    const char* v = std::getenv("MSDA_VALIDATE");
+    return v != nullptr && v[0] != '\0' && std::strcmp(v, "0") != 0;
+  }();
+  return on;
+}
+
+// Host check of device metadata, only when MSDA_VALIDATE is set.
+msda_status check_device_metadata(int64_t S, int64_t L, const int64_t* shapes,
+                                  const int64_t* starts) {
+  int64_t hs[2 * msda::kMaxLevels], hl[msda::kMaxLevels];
+  if (cudaMemcpy(hs, shapes, sizeof(int64_t) * 2 * L, cudaMemcpyDeviceToHost) != cudaSuccess ||
+      cudaMemcpy(hl, starts, sizeof(int64_t) * L, cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MSDA_ERR_CUDA;
+  return msda_check_metadata(S, L, hs, hl);
+}
+
+struct Common {
+  int64_t value_elems = 0, point_elems = 0, out_elems = 0;
+};
+
+msda_status check_common(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq, int64_t L,
+                         int64_t K, Common* c) {
+  if (B < 0 || S < 0 || M < 0 || D < 0 || Lq < 0 || L < 0 || K < 0) return MSDA_ERR_BAD_SHAPE;
+  if (L < 1 || L > msda::kMaxLevels || K < 1 || K > msda::kMaxPoints) return MSDA_ERR_UNSUPPORTED;
+  if (!product_ok({B, S, M, D}, &c->value_elems) ||
+      !product_ok({B, Lq, M, L, K, 2}, &c->point_elems) ||
+      !product_ok({B, Lq, M, D}, &c->out_elems))
+    return MSDA_ERR_BAD_SHAPE;
+  return MSDA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+msda_status msda_forward(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq, int64_t L,
+                         int64_t K, msda_dtype value_dtype, const void* value,
+                         const int64_t* spatial_shapes, const int64_t* level_start_index,
+                         const float* sampling_locations, const float* attention_weights,
+                         void* output, void* stream) {
+  Common c;
+  msda_status st = check_common(B, S, M, D, Lq, L, K, &c);
+  if (st != MSDA_OK) return st;
+  if (value_dtype != MSDA_F32 && value_dtype != MSDA_BF16) return MSDA_ERR_UNSUPPORTED;
+  const int E = value_dtype == MSDA_F32 ? 4 : 8;
+  if (D % E != 0 || M > INT32_MAX || D > INT32_MAX) return MSDA_ERR_UNSUPPORTED;
+  if (c.out_elems == 0) return MSDA_OK;
+  if ((c.value_elems > 0 && value == nullptr) || spatial_shapes == nullptr ||
+      level_start_index == nullptr || sampling_locations == nullptr ||
+      attention_weights == nullptr || output == nullptr)
+    return MSDA_ERR_NULL_POINTER;
+  if (!aligned(value, 16) || !aligned(output, 16) || !aligned(sampling_locations, 8) ||
+      !aligned(attention_weights, 4) || !aligned(spatial_shapes, 8) ||
+      !aligned(level_start_index, 8))
+    return MSDA_ERR_MISALIGNED;
+  if (validate_env()) {
+    st = check_device_metadata(S, L, spatial_shapes, level_start_index);
+    if (st != MSDA_OK) return st;
+  }
+  msda::ForwardArgs a;
+  a.value = value;
+  a.spatial_shapes = spatial_shapes;
+  a.level_start_index = level_start_index;
+  a.sampling_locations = sampling_locations;
+  a.attention_weights = attention_weights;
+  a.output = output;
+  a.S = S;
+  a.Lq = Lq;
+  a.M = static_cast<int>(M);
+  a.D = static_cast<int>(D);
+  a.L = static_cast<int>(L);
+  a.K = static_cast<int>(K);
+  a.bf16 = value_dtype == MSDA_BF16;
+  const int64_t nvec = D / E;
+  a.lanes = pow2_at_least(nvec);
+  a.chunks = static_cast<int>((nvec + a.lanes - 1) / a.lanes);
+  a.groups = B * Lq * M * a.chunks;
+  return msda::launch_forward(a, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? MSDA_OK
+             : MSDA_ERR_CUDA;
+}
+
+msda_status msda_backward(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq, int64_t L,
+                          int64_t K, msda_dtype value_dtype, const void* value,
+                          const int64_t* spatial_shapes, const int64_t* level_start_index,
+                          const float* sampling_locations, const float* attention_weights,
+                          const float* grad_output, float* grad_value,
+                          float* grad_sampling_locations, float* grad_attention_weights,
+                          void* stream) {
+  Common c;
+  msda_status st = check_common(B, S, M, D, Lq, L, K, &c);
+  if (st != MSDA_OK) return st;
+  if (value_dtype != MSDA_F32) return MSDA_ERR_UNSUPPORTED;
+  if (D % 4 != 0 || D > 128 || M > INT32_MAX) return MSDA_ERR_UNSUPPORTED;
+  if (c.value_elems == 0 && c.out_elems == 0) return MSDA_OK;
+  if (c.value_elems > 0 && grad_value == nullptr) return MSDA_ERR_NULL_POINTER;
+  if (!aligned(grad_value, 16)) return MSDA_ERR_MISALIGNED;
+  const bool work = c.out_elems > 0;
+  if (work && (value == nullptr || spatial_shapes == nullptr || level_start_index == nullptr ||
+               sampling_locations == nullptr || attention_weights == nullptr ||
+               grad_output == nullptr || grad_sampling_locations == nullptr ||
+               grad_attention_weights == nullptr))
+    return MSDA_ERR_NULL_POINTER;
+  if (work && (!aligned(value, 16) || !aligned(grad_output, 16) ||
+               !aligned(sampling_locations, 8) || !aligned(grad_sampling_locations, 8) ||
+               !aligned(attention_weights, 4) || !aligned(grad_attention_weights, 4) ||
+               !aligned(spatial_shapes, 8) || !aligned(level_start_index, 8)))
+    return MSDA_ERR_MISALIGNED;
+  if (work && validate_env()) {
+    st = check_device_metadata(S, L, spatial_shapes, level_start_index);
+    if (st != MSDA_OK) return st;
+  }
+  msda::BackwardArgs a;
+  a.value = static_cast<const float*>(value);
+  a.spatial_shapes = spatial_shapes;
+  a.level_start_index = level_start_index;
+  a.sampling_locations = sampling_locations;
+  a.attention_weights = attention_weights;
+  a.grad_output = grad_output;
+  a.grad_value = grad_value;
+  a.grad_sampling_locations = grad_sampling_locations;
+  a.grad_attention_weights = grad_attention_weights;
+  a.S = S;
+  a.Lq = Lq;
+  a.M = static_cast<int>(M);
+  a.D = static_cast<int>(D);
+  a.L = static_cast<int>(L);
+  a.K = static_cast<int>(K);
+  a.lanes = pow2_at_least(D / 4);
+  a.groups = work ? B * Lq * M : 0;
+  a.value_elements = c.value_elems;
+  return msda::launch_backward(a, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? MSDA_OK
+             : MSDA_ERR_CUDA;
+}
+
+msda_status msda_check_metadata(int64_t S, int64_t L, const int64_t* shapes,
+                                const int64_t* starts) {
+  if (L < 0 || S < 0) return MSDA_ERR_BAD_SHAPE;
+  if (L > 0 && (shapes == nullptr || starts == nullptr)) return MSDA_ERR_NULL_POINTER;
+  int64_t total = 0;
+  for (int64_t l = 0; l < L; ++l) {
+    const int64_t h = shapes[2 * l], w = shapes[2 * l + 1];
+    if (h < 1 || w < 1 || h >= msda::kMaxLevelExtent || w >= msda::kMaxLevelExtent)
+      return MSDA_ERR_BAD_SHAPE;
+    if (starts[l] != total) return MSDA_ERR_BAD_SHAPE;
+    total += h * w;
+    if (total > S) return MSDA_ERR_BAD_SHAPE;
+  }
+  return total == S ? MSDA_OK : MSDA_ERR_BAD_SHAPE;
+}
+
+const char* msda_status_string(int status) {
+  switch (status) {
+    case MSDA_OK: return "ok";
+    case MSDA_ERR_NULL_POINTER: return "a required pointer is NULL";
+    case MSDA_ERR_BAD_SHAPE: return "negative size, size overflow or inconsistent level metadata";
+    case MSDA_ERR_UNSUPPORTED: return "unsupported dtype, head dim, level count or point count";
+    case MSDA_ERR_MISALIGNED: return "a pointer is not aligned as required";
+    case MSDA_ERR_CUDA: return "a CUDA launch or runtime call failed";
+    default: return "unknown status";
+  }
+}
+
+int msda_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,191 @@
+// msda_backward.cu -- training backward of the MSDeformAttn core (sm_100a).
+//
+// The pages print no backward.  These are the exact derivatives of the forward
+// ("Deformable DETR Deformable Transformers for End-to-End Object Detection",
+// multi-scale deformable attention equation, sampled as in "Deformable DETR模型
+// 解读（附源码+论文）", ms_deform_attn_core_pytorch), taken inside the cell
+// [x0, x0+1) x [y0, y0+1), x0 = floor(x), y0 = floor(y).  With
+// V_ij = V(x0 + i, y0 + j) (zero outside the map), hx = 1 - fx, hy = 1 - fy and
+// gO = grad_output[b, q, m*D : m*D + D]:
+//
+//   grad_attn[p]    = sum_d gO * (hy (hx V00 + fx V10) + fy (hx V01 + fx V11))
+//   grad_loc[p].x   = A * W_l * sum_d gO * (hy (V10 - V00) + fy (V11 - V01))
+//   grad_loc[p].y   = A * H_l * sum_d gO * (hx (V01 - V00) + fx (V11 - V10))
+//   grad_value[corner ij] += A * (i ? fx : hx) * (j ? fy : hy) * gO   (corners in the map)
+//
+// (dx/dloc_x = W_l because x = loc_x * W_l - 0.5.)
+//
+// Decomposition as in the forward: a sub-warp of LANES lanes owns one (b, q, m);
+// each lane owns 4 channels.  Per point the lanes gather the four corners,
+// form their partial channel sums, reduce them with a butterfly of shuffles and
+// scatter the grad_value contributions with 16-byte vector atomics
+// (red.global.add.v4.f32).  Lane j keeps the reduced sums of point j of the
+// current round and writes them coalesced at the end of the round.
+#include "msda_device.cuh"
+#include "msda_launch.h"
+
+namespace msda {
+
+template <int LANES>
+__global__ void __launch_bounds__(256)
+backward_kernel(const float* __restrict__ value, const int64_t* __restrict__ spatial_shapes,
+                const int64_t* __restrict__ level_start_index,
+                const float* __restrict__ sampling_locations,
+                const float* __restrict__ attention_weights,
+                const float* __restrict__ grad_output, float* __restrict__ grad_value,
+                float* __restrict__ grad_sampling_locations,
+                float* __restrict__ grad_attention_weights, long long S, int M, int D,
+                long long Lq, int L, int K, long long groups) {
+  using V = Vec<float>;
+  constexpr int E = V::N;
+  __shared__ Levels lv;
+  stage_levels(lv, spatial_shapes, level_start_index, L, S);
+
+  const int lane = threadIdx.x % LANES;
+  const int groups_per_block = blockDim.x / LANES;
+  const int LK = L * K;
+  const long long MD = static_cast<long long>(M) * D;
+
+  for (long long g0 = static_cast<long long>(blockIdx.x) * groups_per_block; g0 < groups;
+       g0 += static_cast<long long>(gridDim.x) * groups_per_block) {
+    const long long g_raw = g0 + threadIdx.x / LANES;
+    const bool active = g_raw < groups;
+    const Group grp = decompose(active ? g_raw : groups - 1, 1, M, Lq);
+    const int ch = lane * E;
+    const bool lane_on = active && ch < D;  // clamped tail groups touch no memory
+    const long long vofs = (grp.b * S * M + grp.m) * static_cast<long long>(D) + ch;
+    const float* vbase = value + vofs;
+    float* gvbase = grad_value + vofs;
+    const float* gloc = sampling_locations + grp.bqm * LK * 2;
+    const float* gatt = attention_weights + grp.bqm * LK;
+
+    float go[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) go[e] = 0.0f;
+    if (lane_on) V::load(grad_output + grp.bq * MD + static_cast<long long>(grp.m) * D + ch, go);
+
+    int l = 0, k = 0;
+    int H = lv.H[0], W = lv.W[0];
+    long long start = lv.start[0];
+    for (int p0 = 0; p0 < LK; p0 += LANES) {
+      const int pj = p0 + lane;
+      float2 xy = make_float2(0.0f, 0.0f);
+      float aj = 0.0f;
+      if (pj < LK) {
+        xy = __ldg(reinterpret_cast<const float2*>(gloc) + pj);
+        aj = __ldg(gatt + pj);
+      }
+      float keep_attn = 0.0f, keep_x = 0.0f, keep_y = 0.0f;
+      const int n = min(LANES, LK - p0);
+      for (int j = 0; j < n; ++j) {
+        const float lx = __shfl_sync(kFullMask, xy.x, j, LANES);
+        const float ly = __shfl_sync(kFullMask, xy.y, j, LANES);
+        const float a = __shfl_sync(kFullMask, aj, j, LANES);
+        const Cell c = locate(lx, ly, H, W);
+        const float hx = 1.0f - c.fx, hy = 1.0f - c.fy;
+        const long long row = static_cast<long long>(W) * MD;
+        const long long off = (start + static_cast<long long>(c.y0) * W + c.x0) * MD;
+        const bool v00 = c.vx0 && c.vy0, v10 = c.vx1 && c.vy0;
+        const bool v01 = c.vx0 && c.vy1, v11 = c.vx1 && c.vy1;
+        float s_attn = 0.0f, s_x = 0.0f, s_y = 0.0f;
+        if (lane_on) {
+          // Corner naming: q<i><j> = V(x0 + i, y0 + j).
+          float q00[E], q10[E], q01[E], q11[E];
+#pragma unroll
+          for (int e = 0; e < E; ++e) q00[e] = q10[e] = q01[e] = q11[e] = 0.0f;
+          if (v00) V::load(vbase + off, q00);
+          if (v10) V::load(vbase + off + MD, q10);
+          if (v01) V::load(vbase + off + row, q01);
+          if (v11) V::load(vbase + off + row + MD, q11);
+#pragma unroll
+          for (int e = 0; e < E; ++e) {
+            const float top = fmaf(c.fx, q10[e], hx * q00[e]);
+            const float bot = fmaf(c.fx, q11[e], hx * q01[e]);
+            s_attn = fmaf(go[e], fmaf(c.fy, bot, hy * top), s_attn);
+            s_x = fmaf(go[e], fmaf(c.fy, q11[e] - q01[e], hy * (q10[e] - q00[e])), s_x);
+            s_y = fmaf(go[e], fmaf(c.fx, q11[e] - q10[e], hx * (q01[e] - q00[e])), s_y);
+          }
+          const float w00 = a * hx * hy, w10 = a * c.fx * hy;
+          const float w01 = a * hx * c.fy, w11 = a * c.fx * c.fy;
+          if (v00) atomicAdd(reinterpret_cast<float4*>(gvbase + off),
+                             make_float4(w00 * go[0], w00 * go[1], w00 * go[2], w00 * go[3]));
+          if (v10) atomicAdd(reinterpret_cast<float4*>(gvbase + off + MD),
+                             make_float4(w10 * go[0], w10 * go[1], w10 * go[2], w10 * go[3]));
+          if (v01) atomicAdd(reinterpret_cast<float4*>(gvbase + off + row),
+                             make_float4(w01 * go[0], w01 * go[1], w01 * go[2], w01 * go[3]));
+          if (v11) atomicAdd(reinterpret_cast<float4*>(gvbase + off + row + MD),
+                             make_float4(w11 * go[0], w11 * go[1], w11 * go[2], w11 * go[3]));
+        }
+#pragma unroll
+        for (int o = LANES / 2; o > 0; o >>= 1) {
+          s_attn += __shfl_xor_sync(kFullMask, s_attn, o, LANES);
+          s_x += __shfl_xor_sync(kFullMask, s_x, o, LANES);
+          s_y += __shfl_xor_sync(kFullMask, s_y, o, LANES);
+        }
+        if (lane == j) {
+          keep_attn = s_attn;
+          keep_x = a * static_cast<float>(W) * s_x;
+          keep_y = a * static_cast<float>(H) * s_y;
+        }
+        if (++k == K) {
+          k = 0;
+          if (++l < L) {
+            H = lv.H[l];
+            W = lv.W[l];
+            start = lv.start[l];
+          }
+        }
+      }
+      if (active && pj < LK) {
+        grad_attention_weights[grp.bqm * LK + pj] = keep_attn;
+        reinterpret_cast<float2*>(grad_sampling_locations + grp.bqm * LK * 2)[pj] =
+            make_float2(keep_x, keep_y);
+      }
+    }
+  }
+}
+
+__global__ void zero_kernel(float4* __restrict__ p, long long n4) {
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n4;
+       i += static_cast<long long>(gridDim.x) * blockDim.x)
+    p[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+}
+
+cudaError_t launch_zero(float* p, long long n, cudaStream_t stream) {
+  // n is a multiple of 4 (D % 4 == 0) and p is 16-byte aligned.
+  const long long n4 = n / 4;
+  if (n4 == 0) return cudaSuccess;
+  long long blocks = (n4 + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  zero_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(reinterpret_cast<float4*>(p), n4);
+  return cudaGetLastError();
+}
+
+template <int LANES>
+static cudaError_t launch_backward_t(const BackwardArgs& a, cudaStream_t stream) {
+  constexpr int kThreads = 256;
+  const long long per_block = kThreads / LANES;
+  long long blocks = (a.groups + per_block - 1) / per_block;
+  if (blocks > (1ll << 30)) blocks = 1ll << 30;
+  backward_kernel<LANES><<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(
+      a.value, a.spatial_shapes, a.level_start_index, a.sampling_locations,
+      a.attention_weights, a.grad_output, a.grad_value, a.grad_sampling_locations,
+      a.grad_attention_weights, a.S, a.M, a.D, a.Lq, a.L, a.K, a.groups);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t stream) {
+  cudaError_t err = launch_zero(a.grad_value, a.value_elements, stream);
+  if (err != cudaSuccess || a.groups == 0) return err;
+  switch (a.lanes) {
+    case 1: return launch_backward_t<1>(a, stream);
+    case 2: return launch_backward_t<2>(a, stream);
+    case 4: return launch_backward_t<4>(a, stream);
+    case 8: return launch_backward_t<8>(a, stream);
+    case 16: return launch_backward_t<16>(a, stream);
+    case 32: return launch_backward_t<32>(a, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace msda

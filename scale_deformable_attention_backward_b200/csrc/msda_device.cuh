@@ -1,0 +1,157 @@
+// msda_device.cuh -- device-side building blocks shared by the forward and
+// backward kernels of the MSDeformAttn core (sm_100a).
+//
+// Sampling rule ("Deformable DETR模型解读（附源码+论文）", ms_deform_attn_core_pytorch:
+// grid = 2*loc - 1, grid_sample bilinear, zeros padding, align_corners=False):
+// the pixel coordinate of a normalised location is x = loc * W - 0.5, the
+// bilinear cell is [floor(x), floor(x) + 1) and a corner outside [0, W) reads 0.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include "msda_launch.h"
+
+namespace msda {
+
+constexpr unsigned kFullMask = 0xffffffffu;
+
+// Per-level metadata staged in shared memory.  A level whose metadata would
+// reach outside `value` is staged as 0 x 0, so none of its corners is valid and
+// it is never read.
+struct Levels {
+  int H[kMaxLevels];
+  int W[kMaxLevels];
+  long long start[kMaxLevels];
+};
+
+__device__ __forceinline__ void stage_levels(Levels& lv, const int64_t* __restrict__ shapes,
+                                             const int64_t* __restrict__ level_start, int L,
+                                             int64_t S) {
+  for (int l = threadIdx.x; l < L; l += blockDim.x) {
+    const int64_t h = shapes[2 * l + 0];
+    const int64_t w = shapes[2 * l + 1];
+    const int64_t st = level_start[l];
+    const bool ok = h >= 1 && w >= 1 && h < kMaxLevelExtent && w < kMaxLevelExtent &&
+                    st >= 0 && st <= S && h * w <= S - st;
+    lv.H[l] = ok ? static_cast<int>(h) : 0;
+    lv.W[l] = ok ? static_cast<int>(w) : 0;
+    lv.start[l] = ok ? st : 0;
+  }
+  __syncthreads();
+}
+
+// One axis of the pixel mapping, exact in the floor.
+//   x = loc * n - 0.5 (real arithmetic);  c = floor(x);  f = x - c rounded once.
+// fmaf gives x rounded once, which may land on the wrong side of an integer;
+// the sign of fmaf(loc, n, -(c + 0.5)) = RN(x - c) is exact (round-to-nearest
+// keeps signs, and x - c is a nonzero multiple of 2^-149 or exactly zero), so c is
+// corrected by at most one step.  c + 0.5 and c + 1.5 are exact for |c| < 2^22.
+// A coordinate outside (-2, n + 1) has no corner inside the map and is reported
+// as c = -2 (with f = 0; no weight of it multiplies a value).  A non-finite
+// location also gets c = -2 but f = NaN, so the point's weights -- and its
+// sample, as in grid_sample -- are NaN.
+__device__ __forceinline__ void pixel_coordinate(float loc, float n, float& c, float& f) {
+  const float t = fmaf(loc, n, -0.5f);
+  if (!(fabsf(loc) <= 3.402823466e38f)) {
+    c = -2.0f;
+    f = loc - loc;  // NaN for NaN and for +-Inf
+  } else if (t > -2.0f && t < n + 1.0f) {
+    c = floorf(t);
+    f = fmaf(loc, n, -(c + 0.5f));
+    if (f < 0.0f) {
+      c -= 1.0f;
+      f = fmaf(loc, n, -(c + 0.5f));
+    } else if (fmaf(loc, n, -(c + 1.5f)) >= 0.0f) {
+      c += 1.0f;
+      f = fmaf(loc, n, -(c + 0.5f));
+    }
+  } else {
+    c = -2.0f;
+    f = 0.0f;
+  }
+}
+
+// The sampling geometry of one point on its level.
+struct Cell {
+  int x0, y0;                 // top-left corner (may lie outside the map)
+  float fx, fy;               // position inside the cell
+  bool vx0, vx1, vy0, vy1;    // corner columns / rows inside the map
+};
+
+__device__ __forceinline__ Cell locate(float lx, float ly, int H, int W) {
+  Cell c;
+  float cx, cy;
+  pixel_coordinate(lx, static_cast<float>(W), cx, c.fx);
+  pixel_coordinate(ly, static_cast<float>(H), cy, c.fy);
+  c.x0 = static_cast<int>(cx);
+  c.y0 = static_cast<int>(cy);
+  c.vx0 = static_cast<unsigned>(c.x0) < static_cast<unsigned>(W);
+  c.vx1 = static_cast<unsigned>(c.x0 + 1) < static_cast<unsigned>(W);
+  c.vy0 = static_cast<unsigned>(c.y0) < static_cast<unsigned>(H);
+  c.vy1 = static_cast<unsigned>(c.y0 + 1) < static_cast<unsigned>(H);
+  return c;
+}
+
+// ---------------------------------------------------------------------------
+// 16-byte lane vectors: 4 x float32 or 8 x bfloat16, widened to float32.
+// ---------------------------------------------------------------------------
+template <typename T>
+struct Vec;
+
+template <>
+struct Vec<float> {
+  static constexpr int N = 4;
+  __device__ __forceinline__ static void load(const float* p, float (&v)[N]) {
+    const float4 r = __ldg(reinterpret_cast<const float4*>(p));
+    v[0] = r.x; v[1] = r.y; v[2] = r.z; v[3] = r.w;
+  }
+  __device__ __forceinline__ static void store(float* p, const float (&v)[N]) {
+    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  }
+};
+
+template <>
+struct Vec<__nv_bfloat16> {
+  static constexpr int N = 8;
+  __device__ __forceinline__ static void load(const __nv_bfloat16* p, float (&v)[N]) {
+    const uint4 r = __ldg(reinterpret_cast<const uint4*>(p));
+    const unsigned w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i + 0] = __uint_as_float(w[i] << 16);
+      v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+  }
+  __device__ __forceinline__ static void store(__nv_bfloat16* p, const float (&v)[N]) {
+    unsigned w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i + 0], v[2 * i + 1]);
+      w[i] = *reinterpret_cast<const unsigned*>(&h);
+    }
+    *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+};
+
+// Decomposition of a flat work-group index g = ((b * Lq + q) * M + m) * chunks + c.
+struct Group {
+  long long bq;    // b * Lq + q
+  long long bqm;   // (b * Lq + q) * M + m
+  long long b;
+  int m;
+  int chunk;
+};
+
+__device__ __forceinline__ Group decompose(long long g, int chunks, int M, long long Lq) {
+  Group r;
+  r.chunk = static_cast<int>(g % chunks);
+  r.bqm = g / chunks;
+  r.m = static_cast<int>(r.bqm % M);
+  r.bq = r.bqm / M;
+  r.b = r.bq / Lq;
+  return r;
+}
+
+}  // namespace msda

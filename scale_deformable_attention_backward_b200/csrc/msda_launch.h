@@ -1,0 +1,50 @@
+// msda_launch.h -- internal launch interface between the C ABI (msda_api.cu)
+// and the kernels.  Arguments arrive here already validated.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace msda {
+
+constexpr int kMaxLevels = 16;
+constexpr int kMaxPoints = 64;
+constexpr int kMaxLevelExtent = 1 << 22;  // H_l, W_l below 2^22: float coordinates stay exact
+
+struct ForwardArgs {
+  const void* value;
+  const int64_t* spatial_shapes;
+  const int64_t* level_start_index;
+  const float* sampling_locations;
+  const float* attention_weights;
+  void* output;
+  long long S, Lq;
+  int M, D, L, K;
+  bool bf16;
+  int lanes;         // lanes per work group: a power of two <= 32
+  int chunks;        // channel chunks per (b, q, m): ceil(D / (lanes * elements per lane))
+  long long groups;  // B * Lq * M * chunks
+};
+
+struct BackwardArgs {
+  const float* value;
+  const int64_t* spatial_shapes;
+  const int64_t* level_start_index;
+  const float* sampling_locations;
+  const float* attention_weights;
+  const float* grad_output;
+  float* grad_value;
+  float* grad_sampling_locations;
+  float* grad_attention_weights;
+  long long S, Lq;
+  int M, D, L, K;
+  int lanes;         // lanes per (b, q, m) group; D <= 4 * lanes
+  long long groups;  // B * Lq * M
+  long long value_elements;  // B * S * M * D (grad_value is zeroed first)
+};
+
+cudaError_t launch_forward(const ForwardArgs& a, cudaStream_t stream);
+cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t stream);
+cudaError_t launch_zero(float* p, long long n, cudaStream_t stream);
+
+}  // namespace msda

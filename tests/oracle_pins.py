@@ -433,6 +433,22 @@ def pin_grid_sample(orc):
     _close(gl, ref_gl, 1e-11, 1e-11, "grad_loc vs grid_sample autograd")
     _close(ga, ref_ga, 1e-12, 1e-12, "grad_attn vs grid_sample autograd")
 
+    # Non-finite locations: grid_sample turns the sample into NaN and gives
+    # grad_value nothing from it; the oracle must agree on where NaN appears.
+    loc = loc.copy()
+    loc[0, 1, 0, 0, 0, 0] = np.nan
+    loc[1, 2, 2, 1, 1, 1] = np.inf
+    loc[0, 5, 1, 2, 0, 0] = -np.inf
+    ref_out, ref_gv, ref_gl, ref_ga = grid_sample_reference(v, ss, start, loc, attn, grad)
+    out = orc.forward(v, ss, start, loc, attn)
+    gv, gl, ga = orc.backward(v, ss, start, loc, attn, grad)
+    for got, ref, what in ((out, ref_out, "output"), (gv, ref_gv, "grad_value"),
+                           (gl, ref_gl, "grad_loc"), (ga, ref_ga, "grad_attn")):
+        assert np.array_equal(np.isnan(got), np.isnan(ref)), f"NaN pattern of {what}"
+        keep = ~np.isnan(ref)
+        _close(got[keep], ref[keep], 1e-11, 1e-11, f"{what} with non-finite locations")
+    assert np.isnan(out).any() and not np.isnan(gv).any()
+
 
 ALL_PINS = [
     pin_pixel_centre,

@@ -1,0 +1,122 @@
+"""The C-ABI library on the host (no GPU): it loads, exports every symbol that
+include/msda.h declares, and rejects bad arguments before touching a device."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from scale_deformable_attention_backward_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "msda.h")
+
+OK, NULLP, BAD, UNSUP, MISAL = 0, 1, 2, 3, 4
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(msda_[a-z_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return binding.library()
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert {"msda_forward", "msda_backward"} <= set(names)
+    for name in names:
+        assert hasattr(lib, name), f"libmsda.so does not export {name}"
+        assert name in binding.SIGNATURES, f"binding has no signature for {name}"
+
+
+def test_status_strings_and_version(lib):
+    for code in range(6):
+        assert lib.msda_status_string(code)
+    assert lib.msda_status_string(99) == b"unknown status"
+    assert lib.msda_version() >= 100
+
+
+def _i64(a):
+    a = np.ascontiguousarray(np.asarray(a, dtype=np.int64))
+    return a, ctypes.c_void_p(a.ctypes.data)
+
+
+def test_check_metadata(lib):
+    ss, pss = _i64([[100, 150], [50, 75], [25, 38], [13, 19]])
+    st, pst = _i64([0, 15000, 18750, 19700])
+    assert lib.msda_check_metadata(19947, 4, pss, pst) == OK
+    assert lib.msda_check_metadata(19946, 4, pss, pst) == BAD
+    st2, pst2 = _i64([0, 15000, 18751, 19700])
+    assert lib.msda_check_metadata(19947, 4, pss, pst2) == BAD
+    ss3, pss3 = _i64([[0, 150], [50, 75], [25, 38], [13, 19]])
+    assert lib.msda_check_metadata(19947, 4, pss3, pst) == BAD
+    assert lib.msda_check_metadata(19947, 4, None, pst) == NULLP
+    assert lib.msda_check_metadata(0, 0, None, None) == OK
+    assert lib.msda_check_metadata(-1, 0, None, None) == BAD
+
+
+FAKE = 0x10000  # aligned, never dereferenced: every call below fails validation first
+
+
+def _fwd(lib, B=1, S=80, M=2, D=8, Lq=80, L=2, K=2, dtype=0, value=FAKE, shapes=FAKE,
+         starts=FAKE, loc=FAKE, attn=FAKE, out=FAKE):
+    v = lambda p: None if p is None else ctypes.c_void_p(p)
+    return lib.msda_forward(B, S, M, D, Lq, L, K, dtype, v(value), v(shapes), v(starts), v(loc),
+                            v(attn), v(out), None)
+
+
+def _bwd(lib, B=1, S=80, M=2, D=8, Lq=80, L=2, K=2, dtype=0, ptrs=None):
+    p = [FAKE] * 9 if ptrs is None else ptrs
+    v = lambda x: None if x is None else ctypes.c_void_p(x)
+    return lib.msda_backward(B, S, M, D, Lq, L, K, dtype, *[v(x) for x in p], None)
+
+
+def test_forward_argument_errors(lib):
+    assert _fwd(lib, B=-1) == BAD
+    assert _fwd(lib, K=-2) == BAD
+    assert _fwd(lib, L=0) == UNSUP
+    assert _fwd(lib, L=17) == UNSUP
+    assert _fwd(lib, K=65) == UNSUP
+    assert _fwd(lib, D=6) == UNSUP                 # float32 needs D % 4 == 0
+    assert _fwd(lib, D=12, dtype=1) == UNSUP       # bfloat16 needs D % 8 == 0
+    assert _fwd(lib, dtype=7) == UNSUP
+    assert _fwd(lib, value=None) == NULLP
+    assert _fwd(lib, out=None) == NULLP
+    assert _fwd(lib, loc=None) == NULLP
+    assert _fwd(lib, value=FAKE + 8) == MISAL
+    assert _fwd(lib, out=FAKE + 4) == MISAL
+    assert _fwd(lib, loc=FAKE + 4) == MISAL
+    assert _fwd(lib, attn=FAKE + 2) == MISAL
+    assert _fwd(lib, B=1 << 40, S=1 << 40) == BAD  # element count overflow
+
+
+def test_forward_empty_work_is_ok_without_launch(lib):
+    # Nothing to compute: OK, no launch, NULL pointers allowed.
+    assert _fwd(lib, B=0, value=None, loc=None, attn=None, out=None) == OK
+    assert _fwd(lib, Lq=0, loc=None, attn=None, out=None) == OK
+    assert _fwd(lib, M=0, value=None, loc=None, attn=None, out=None) == OK
+
+
+def test_backward_argument_errors(lib):
+    assert _bwd(lib, dtype=1) == UNSUP             # backward is float32 only
+    assert _bwd(lib, D=132) == UNSUP               # at most 128 channels per head
+    assert _bwd(lib, D=6) == UNSUP
+    assert _bwd(lib, S=-3) == BAD
+    p = [FAKE] * 9
+    p[6] = None                                    # grad_value
+    assert _bwd(lib, ptrs=p) == NULLP
+    p = [FAKE] * 9
+    p[6] = FAKE + 4
+    assert _bwd(lib, ptrs=p) == MISAL
+    p = [FAKE] * 9
+    p[5] = FAKE + 8                                # grad_output
+    assert _bwd(lib, ptrs=p) == MISAL
+    p = [FAKE] * 9
+    p[7] = FAKE + 4                                # grad_sampling_locations
+    assert _bwd(lib, ptrs=p) == MISAL
+    assert _bwd(lib, B=0, ptrs=[None] * 9) == OK  # nothing to write at all

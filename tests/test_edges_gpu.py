@@ -1,0 +1,247 @@
+"""GPU parity on shapes and inputs chosen to break things: every lane width and
+channel chunking, ragged query counts, levels of height or width 1, locations
+far outside the maps or within one float32 ulp of a pixel boundary, non-finite
+locations, empty calls, inconsistent metadata, misaligned pointers, and guard
+bands around every output."""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import gpu_support as G
+from scale_deformable_attention_backward_b200 import binding
+from scale_deformable_attention_backward_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+
+def random_inputs(seed, B, M, D, K, shapes, Lq, lo=-0.3, hi=1.3, dtype="f32", grad=True):
+    rng = np.random.default_rng(seed)
+    ss, start = W.level_metadata(shapes)
+    S = int((ss[:, 0] * ss[:, 1]).sum())
+    L = len(shapes)
+    value = rng.standard_normal((B, S, M, D)).astype(np.float32)
+    bits = None
+    if dtype == "bf16":
+        bits = W.bf16_round_bits(value)
+        value = W.bf16_bits_to_f32(bits)
+    loc = rng.uniform(lo, hi, size=(B, Lq, M, L, K, 2)).astype(np.float32)
+    attn = rng.uniform(0, 1, size=(B, Lq, M, L, K))
+    attn = (attn / attn.sum(axis=(3, 4), keepdims=True)).astype(np.float32)
+    go = rng.standard_normal((B, Lq, M * D)).astype(np.float32) if grad else None
+    cfg = W.Config("random", B, M, D, K, tuple(shapes), "uniform", dtype, grad, Lq)
+    return W.Inputs(cfg, np.ascontiguousarray(value), bits, ss, start, loc, attn, go)
+
+
+SHAPES = [[(5, 7)], [(1, 9), (6, 1), (3, 4)], [(16, 3), (8, 2), (4, 1), (2, 1)],
+          [(11, 13), (1, 1)]]
+
+
+@pytest.mark.parametrize("D", [4, 8, 12, 16, 20, 32, 64, 128])
+@pytest.mark.parametrize("shapes_id", range(len(SHAPES)))
+def test_random_shapes_f32(D, shapes_id):
+    shapes = SHAPES[shapes_id]
+    inp = random_inputs(100 + D + shapes_id, B=2, M=3, D=D, K=3, shapes=shapes, Lq=37)
+    d = G.device_inputs(inp)
+    G.assert_forward_f32(G.gpu_forward(d), G.oracle_forward(inp), f"forward D={D}")
+    gv, gl, ga = G.gpu_backward(d)
+    rv, rl, ra = G.oracle_backward(inp)
+    G.assert_backward_f32(gv, rv, "grad_value")
+    G.assert_backward_f32(gl, rl, "grad_sampling_locations")
+    G.assert_backward_f32(ga, ra, "grad_attention_weights")
+
+
+@pytest.mark.parametrize("D", [256, 384])
+def test_forward_channel_chunks_f32(D):
+    """More than 32 lanes' worth of channels: several chunks per head."""
+    inp = random_inputs(7 + D, B=1, M=2, D=D, K=2, shapes=SHAPES[1], Lq=19, grad=False)
+    G.assert_forward_f32(G.gpu_forward(G.device_inputs(inp)), G.oracle_forward(inp))
+
+
+@pytest.mark.parametrize("D", [8, 16, 24, 32, 64, 256, 512])
+def test_random_shapes_bf16(D):
+    inp = random_inputs(200 + D, B=2, M=2, D=D, K=4, shapes=SHAPES[2], Lq=29, dtype="bf16",
+                        grad=False)
+    G.assert_forward_bf16(G.gpu_forward(G.device_inputs(inp)), G.oracle_forward(inp))
+
+
+@pytest.mark.parametrize("L,K", [(1, 1), (3, 5), (16, 1), (1, 64), (16, 4)])
+def test_level_and_point_counts(L, K):
+    rng = np.random.default_rng(L * 100 + K)
+    shapes = [(int(rng.integers(1, 9)), int(rng.integers(1, 9))) for _ in range(L)]
+    inp = random_inputs(300 + L + K, B=1, M=2, D=8, K=K, shapes=shapes, Lq=13)
+    d = G.device_inputs(inp)
+    G.assert_forward_f32(G.gpu_forward(d), G.oracle_forward(inp))
+    gv, gl, ga = G.gpu_backward(d)
+    rv, rl, ra = G.oracle_backward(inp)
+    G.assert_backward_f32(gv, rv, "grad_value")
+    G.assert_backward_f32(gl, rl, "grad_sampling_locations")
+    G.assert_backward_f32(ga, ra, "grad_attention_weights")
+
+
+def test_locations_at_pixel_boundaries():
+    """Pixel coordinates x = loc*W - 0.5 within a few float32 ulps of an integer,
+    on maps whose widths are not powers of two.  The cell (floor) must match the
+    oracle's exact one, or grad_sampling_locations jumps by a whole corner
+    difference."""
+    shapes = [(100, 150), (25, 38), (13, 19)]
+    ss, start = W.level_metadata(shapes)
+    rng = np.random.default_rng(5)
+    B, M, D, K, Lq = 1, 2, 8, 4, 256
+    L = len(shapes)
+    loc = np.empty((B, Lq, M, L, K, 2), dtype=np.float32)
+    for l, (h, w) in enumerate(shapes):
+        for comp, n in ((0, w), (1, h)):
+            pix = rng.integers(0, n, size=(B, Lq, M, K))
+            base = ((pix + 0.5) / n).astype(np.float32)
+            steps = rng.integers(-3, 4, size=base.shape)
+            out = base.copy()
+            for s in range(1, 4):
+                out = np.where(steps >= s, np.nextafter(out, np.float32(2)), out)
+                out = np.where(steps <= -s, np.nextafter(out, np.float32(-1)), out)
+            loc[:, :, :, l, :, comp] = out
+    inp = random_inputs(6, B, M, D, K, shapes, Lq)
+    inp = dataclasses.replace(inp, sampling_locations=loc)
+    d = G.device_inputs(inp)
+    G.assert_forward_f32(G.gpu_forward(d), G.oracle_forward(inp))
+    gv, gl, ga = G.gpu_backward(d)
+    rv, rl, ra = G.oracle_backward(inp)
+    G.assert_backward_f32(gl, rl, "grad_sampling_locations at pixel boundaries")
+    G.assert_backward_f32(gv, rv, "grad_value")
+    G.assert_backward_f32(ga, ra, "grad_attention_weights")
+
+
+def test_far_and_nonfinite_locations():
+    inp = random_inputs(8, B=2, M=2, D=8, K=3, shapes=SHAPES[1], Lq=11)
+    loc = inp.sampling_locations.copy()
+    loc[0, 0, 0, 0, 0] = (1e30, 0.5)
+    loc[0, 1, 1, 1, 2] = (-1e30, -1e30)
+    loc[1, 2, 0, 2, 1] = (3.0e38, 0.2)
+    loc[1, 3, 1, 0, 0] = (-7.5, 42.0)
+    loc[0, 4, 0, 0, 1] = (np.nan, 0.5)
+    loc[1, 5, 1, 2, 2] = (0.5, np.inf)
+    loc[0, 6, 0, 1, 0] = (-np.inf, -np.inf)
+    inp = dataclasses.replace(inp, sampling_locations=loc)
+    d = G.device_inputs(inp)
+    G.assert_forward_f32(G.gpu_forward(d), G.oracle_forward(inp))
+    gv, gl, ga = G.gpu_backward(d)
+    rv, rl, ra = G.oracle_backward(inp)
+    G.assert_backward_f32(gv, rv, "grad_value")
+    G.assert_backward_f32(gl, rl, "grad_sampling_locations")
+    G.assert_backward_f32(ga, ra, "grad_attention_weights")
+
+
+def test_empty_calls():
+    inp = random_inputs(9, B=2, M=2, D=8, K=2, shapes=SHAPES[0], Lq=0)
+    d = G.device_inputs(inp)
+    out = binding.forward(d["value"], d["spatial_shapes"], d["level_start_index"],
+                          d["sampling_locations"], d["attention_weights"])
+    assert out.shape == (2, 0, 16)
+    gv = torch.full(d["value"].shape, 7.0, device="cuda")
+    binding.backward(d["value"], d["spatial_shapes"], d["level_start_index"],
+                     d["sampling_locations"], d["attention_weights"], d["grad_output"],
+                     grad_value=gv)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(gv).item() == 0, "grad_value must be zeroed even with Lq = 0"
+    inp0 = random_inputs(9, B=0, M=2, D=8, K=2, shapes=SHAPES[0], Lq=5)
+    d0 = G.device_inputs(inp0)
+    out = binding.forward(d0["value"], d0["spatial_shapes"], d0["level_start_index"],
+                          d0["sampling_locations"], d0["attention_weights"])
+    assert out.shape == (0, 5, 16)
+
+
+def _guarded(shape, fill, dtype=torch.float32, pad=64):
+    n = int(np.prod(shape))
+    buf = torch.full((n + 2 * pad,), fill, dtype=dtype, device="cuda")
+    return buf, buf[pad:pad + n].view(shape)
+
+
+def test_guard_bands_untouched():
+    inp = random_inputs(10, B=2, M=3, D=12, K=3, shapes=SHAPES[1], Lq=21)
+    d = G.device_inputs(inp)
+    B, S, M, D = inp.value.shape
+    _, Lq, _, L, K, _ = inp.sampling_locations.shape
+    sentinel = 12345.0
+    ob, out = _guarded((B, Lq, M * D), sentinel)
+    binding.forward(d["value"], d["spatial_shapes"], d["level_start_index"],
+                    d["sampling_locations"], d["attention_weights"], output=out)
+    vb, gv = _guarded((B, S, M, D), sentinel)
+    lb, gl = _guarded((B, Lq, M, L, K, 2), sentinel)
+    ab, ga = _guarded((B, Lq, M, L, K), sentinel)
+    binding.backward(d["value"], d["spatial_shapes"], d["level_start_index"],
+                     d["sampling_locations"], d["attention_weights"], d["grad_output"],
+                     grad_value=gv, grad_sampling_locations=gl, grad_attention_weights=ga)
+    torch.cuda.synchronize()
+    for buf in (ob, vb, lb, ab):
+        assert torch.all(buf[:64] == sentinel) and torch.all(buf[-64:] == sentinel)
+    G.assert_forward_f32(out.double().cpu().numpy(), G.oracle_forward(inp))
+    rv, rl, ra = G.oracle_backward(inp)
+    G.assert_backward_f32(gv.double().cpu().numpy(), rv, "grad_value")
+    G.assert_backward_f32(gl.double().cpu().numpy(), rl, "grad_sampling_locations")
+    G.assert_backward_f32(ga.double().cpu().numpy(), ra, "grad_attention_weights")
+
+
+def test_misaligned_pointer_is_rejected():
+    inp = random_inputs(11, B=1, M=2, D=8, K=2, shapes=SHAPES[0], Lq=4)
+    d = G.device_inputs(inp)
+    flat = torch.zeros(d["value"].numel() + 1, device="cuda")
+    shifted = flat[1:].view(d["value"].shape)           # 4 bytes off a 16-byte boundary
+    with pytest.raises(binding.MSDAError) as e:
+        binding.forward(shifted, d["spatial_shapes"], d["level_start_index"],
+                        d["sampling_locations"], d["attention_weights"])
+    assert e.value.status == 4
+
+
+def test_inconsistent_device_metadata_is_memory_safe():
+    """A level whose start + H*W reaches past S is treated as empty: the result
+    equals the oracle run with that level's weights set to zero, and no memory
+    outside the buffers is touched (guard bands)."""
+    inp = random_inputs(12, B=1, M=2, D=8, K=2, shapes=SHAPES[1], Lq=9)
+    d = G.device_inputs(inp)
+    bad = inp.level_start_index.copy()
+    bad[2] = inp.value.shape[1] - 3                      # level 2 (3x4) overruns S
+    d["level_start_index"] = torch.from_numpy(bad).cuda()
+    got = G.gpu_forward(d)
+    attn = inp.attention_weights.copy()
+    attn[:, :, :, 2, :] = 0.0
+    ref = G.oracle_forward(dataclasses.replace(inp, attention_weights=attn))
+    G.assert_forward_f32(got, ref, "forward with an overrunning level")
+    gv, gl, ga = G.gpu_backward(d)
+    assert np.all(gl[:, :, :, 2] == 0.0) and np.all(ga[:, :, :, 2] == 0.0)
+
+
+def test_host_metadata_is_checked():
+    inp = random_inputs(13, B=1, M=2, D=8, K=2, shapes=SHAPES[1], Lq=3)
+    d = G.device_inputs(inp)
+    bad = torch.from_numpy(inp.level_start_index.copy())
+    bad[1] += 1
+    with pytest.raises(binding.MSDAError) as e:
+        binding.forward(d["value"], torch.from_numpy(inp.spatial_shapes), bad,
+                        d["sampling_locations"], d["attention_weights"])
+    assert e.value.status == 2
+    out = binding.forward(d["value"], torch.from_numpy(inp.spatial_shapes),
+                          torch.from_numpy(inp.level_start_index),
+                          d["sampling_locations"], d["attention_weights"])
+    torch.cuda.synchronize()
+    G.assert_forward_f32(out.double().cpu().numpy(), G.oracle_forward(inp))
+
+
+def test_autograd_function_and_side_stream():
+    from scale_deformable_attention_backward_b200 import ms_deform_attn
+    inp = random_inputs(14, B=2, M=2, D=8, K=2, shapes=SHAPES[1], Lq=17)
+    d = G.device_inputs(inp)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        v = d["value"].clone().requires_grad_()
+        lo = d["sampling_locations"].clone().requires_grad_()
+        at = d["attention_weights"].clone().requires_grad_()
+        out = ms_deform_attn(v, d["spatial_shapes"], d["level_start_index"], lo, at, 64)
+        out.backward(d["grad_output"])
+    s.synchronize()
+    G.assert_forward_f32(out.detach().double().cpu().numpy(), G.oracle_forward(inp))
+    rv, rl, ra = G.oracle_backward(inp)
+    G.assert_backward_f32(v.grad.double().cpu().numpy(), rv, "autograd grad_value")
+    G.assert_backward_f32(lo.grad.double().cpu().numpy(), rl, "autograd grad_loc")
+    G.assert_backward_f32(at.grad.double().cpu().numpy(), ra, "autograd grad_attn")
