@@ -53,6 +53,9 @@ FORWARD_WORKLOAD = "encoder_fp32"
 METRIC = "MSDeformAttn fwd/bwd queries/sec and achieved HBM GB/s vs B200 peak (1 GPU)"
 FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
+# msda_backward with a workspace: zero grad_value, zero cell counts, bin, three
+# scan passes, place, cells.
+BACKWARD_LAUNCHES = 8
 KERNEL_SOURCES = os.path.join(ROOT, "scale_deformable_attention_backward_b200", "csrc")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 
@@ -255,6 +258,8 @@ def run_b200(args, world, rank, local):
     gl = torch.empty_like(d["sampling_locations"])
     ga = torch.empty_like(d["attention_weights"])
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    ws = torch.empty(binding.workspace_size(B, S, M, D, Lq, L, K), dtype=torch.uint8,
+                     device=device)
 
     def step():
         binding.forward(d["value"], d["spatial_shapes"], d["level_start_index"],
@@ -263,7 +268,8 @@ def run_b200(args, world, rank, local):
     def step_bwd():
         binding.backward(d["value"], d["spatial_shapes"], d["level_start_index"],
                          d["sampling_locations"], d["attention_weights"], d["grad_output"],
-                         grad_value=gv, grad_sampling_locations=gl, grad_attention_weights=ga)
+                         grad_value=gv, grad_sampling_locations=gl, grad_attention_weights=ga,
+                         workspace=ws)
 
     for _ in range(args.warmup):
         flush.fill_(1.0)
@@ -304,7 +310,8 @@ def run_b200(args, world, rank, local):
     roofline = {
         "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
         "frac": round(achieved / peak, 4), "traffic": recorded_traffic(f"{STEP_WORKLOAD}.{dom}"),
-        "kernel": ("msda_backward: zero_kernel + backward_kernel" if dom == "backward"
+        "kernel": (f"msda_backward launch sequence ({BACKWARD_LAUNCHES} kernels: zero fills, "
+                   "bin, 3-pass scan, place, cell)" if dom == "backward"
                    else "msda_forward: forward_kernel"),
         "algorithmic_bytes": algo[dom], "mean_ms": round(dom_ms, 4),
         "peak_source": f"{peak_kind} HBM copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
@@ -409,7 +416,7 @@ def run_b200(args, world, rank, local):
         "e2e": {"value": round(world * queries / (e2e_ms * 1e-3), 1), "unit": "queries/s",
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h)},
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": (1 + BACKWARD_LAUNCHES) * args.steps,
         "clocks": clocks.summary(),
         "wall_s_timed_region": round(wall, 3),
         "cpu_baseline": None,

@@ -42,7 +42,8 @@
  *    out-of-bounds access.  msda_check_metadata() validates host copies.
  *  - Supported: value dtype float32 with D % 4 == 0, or bfloat16 with D % 8 == 0
  *    (each lane moves 16 bytes); 1 <= L <= 16; 1 <= K <= 64; every size >= 0,
- *    B*S*M*D and B*Lq*M*L*K*2 below 2^62, H_l and W_l below 2^22.  `value`,
+ *    B*S*M*D and B*Lq*M*L*K*2 below 2^62, S*M*D below 2^31 (one image's value
+ *    block is addressed with 32-bit offsets), H_l and W_l below 2^22.  `value`,
  *    `output`, `grad_output` and `grad_value` must be 16-byte aligned,
  *    `sampling_locations` 8-byte aligned, the other arrays 4-byte aligned
  *    (8-byte for the int64 metadata).
@@ -52,6 +53,7 @@
 #ifndef MSDA_H
 #define MSDA_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -64,7 +66,8 @@ typedef enum {
     MSDA_ERR_BAD_SHAPE = 2,     /* a size is negative or the metadata is inconsistent */
     MSDA_ERR_UNSUPPORTED = 3,   /* dtype, D, L or K outside the supported set         */
     MSDA_ERR_MISALIGNED = 4,    /* a pointer breaks the alignment rule above          */
-    MSDA_ERR_CUDA = 5           /* a CUDA launch or runtime call failed               */
+    MSDA_ERR_CUDA = 5,          /* a CUDA launch or runtime call failed               */
+    MSDA_ERR_WORKSPACE = 6      /* workspace smaller than msda_backward_workspace_size */
 } msda_status;
 
 typedef enum {
@@ -106,7 +109,8 @@ msda_status msda_forward(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq,
  * inputs (the softmax before them is not differentiated).
  *
  *   value, spatial_shapes, level_start_index, sampling_locations,
- *   attention_weights   as for msda_forward (value_dtype must be MSDA_F32)
+ *   attention_weights   as for msda_forward (value_dtype must be MSDA_F32,
+ *                       D <= 128)
  *   grad_output              [B, Lq, M * D]        float32
  *   grad_value               [B, S, M, D]          float32  overwritten: zeroed on
  *                                                  `stream`, then accumulated with
@@ -114,6 +118,16 @@ msda_status msda_forward(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq,
  *                                                  the last bits, vary run to run)
  *   grad_sampling_locations  [B, Lq, M, L, K, 2]   float32  overwritten
  *   grad_attention_weights   [B, Lq, M, L, K]      float32  overwritten
+ *   workspace, workspace_bytes
+ *                 device scratch owned by the caller, 256-byte aligned, at least
+ *                 msda_backward_workspace_size() bytes; its contents on entry do
+ *                 not matter and are garbage on exit.  With a workspace the points
+ *                 are grouped by bilinear cell first, so each cell's corners are
+ *                 read once and each grad_value row gets one atomic per cell
+ *                 instead of one per point.  workspace == NULL selects the
+ *                 scratch-free path (one atomic per point corner; slower).  A
+ *                 workspace that is too small returns MSDA_ERR_WORKSPACE.  Two
+ *                 calls that overlap on the GPU must not share a workspace.
  */
 msda_status msda_backward(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq,
                           int64_t L, int64_t K, msda_dtype value_dtype,
@@ -123,7 +137,21 @@ msda_status msda_backward(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq
                           const float *attention_weights,
                           const float *grad_output, float *grad_value,
                           float *grad_sampling_locations,
-                          float *grad_attention_weights, void *stream);
+                          float *grad_attention_weights, void *workspace,
+                          size_t workspace_bytes, void *stream);
+
+/*
+ * Bytes of workspace msda_backward needs for these sizes (host only; no device
+ * access).  The bound depends on the sizes alone: a level of H x W pixels has
+ * (H + 1)(W + 1) bilinear cells, and sum_l (H_l + 1)(W_l + 1) <= 2 S + 2 L.
+ * For B=4, S=Lq=19947, M=8, L=K=4 it is about 250 MB.  Returns
+ * MSDA_ERR_UNSUPPORTED when the sorted path's 32-bit cell and point ids would
+ * overflow (B*M*(2S+2L) or B*Lq*M*L*K at 2^31 or more); the scratch-free path
+ * still accepts those sizes.
+ */
+msda_status msda_backward_workspace_size(int64_t B, int64_t S, int64_t M, int64_t D,
+                                         int64_t Lq, int64_t L, int64_t K,
+                                         size_t *bytes);
 
 /*
  * Host-side metadata check, for callers that hold host copies of the metadata

@@ -25,13 +25,15 @@ LIBRARY_PATH = os.path.join(_HERE, "libmsda.so")
 
 MSDA_F32, MSDA_BF16 = 0, 1
 _STATUS = {0: "MSDA_OK", 1: "MSDA_ERR_NULL_POINTER", 2: "MSDA_ERR_BAD_SHAPE",
-           3: "MSDA_ERR_UNSUPPORTED", 4: "MSDA_ERR_MISALIGNED", 5: "MSDA_ERR_CUDA"}
+           3: "MSDA_ERR_UNSUPPORTED", 4: "MSDA_ERR_MISALIGNED", 5: "MSDA_ERR_CUDA",
+           6: "MSDA_ERR_WORKSPACE"}
 
 # Every symbol include/msda.h declares, with its ctypes signature.
-_I64, _VP, _I32 = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int
+_I64, _VP, _I32, _SZ = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
 SIGNATURES = {
     "msda_forward": (_I32, [_I64] * 7 + [_I32] + [_VP] * 7),
-    "msda_backward": (_I32, [_I64] * 7 + [_I32] + [_VP] * 10),
+    "msda_backward": (_I32, [_I64] * 7 + [_I32] + [_VP] * 10 + [_SZ, _VP]),
+    "msda_backward_workspace_size": (_I32, [_I64] * 7 + [ctypes.POINTER(_SZ)]),
     "msda_check_metadata": (_I32, [_I64, _I64, _VP, _VP]),
     "msda_status_string": (ctypes.c_char_p, [_I32]),
     "msda_version": (_I32, []),
@@ -163,9 +165,14 @@ def backward(value: torch.Tensor, spatial_shapes, level_start_index,
              grad_value: Optional[torch.Tensor] = None,
              grad_sampling_locations: Optional[torch.Tensor] = None,
              grad_attention_weights: Optional[torch.Tensor] = None,
+             workspace="auto",
              ) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
     """MSDeformAttn backward: (grad_value, grad_sampling_locations,
-    grad_attention_weights), all float32."""
+    grad_attention_weights), all float32.
+
+    ``workspace``: ``"auto"`` (default) takes scratch for the cell-sorted path
+    from torch's caching allocator; a uint8 CUDA tensor supplies it; ``None``
+    selects the scratch-free path (one atomic per point corner)."""
     dev = value.device
     B, S, M, D, Lq, L, K = _dims(value, sampling_locations, attention_weights)
     _require(value, "value", torch.float32, dev)
@@ -190,14 +197,33 @@ def backward(value: torch.Tensor, spatial_shapes, level_start_index,
                 raise ValueError(f"{name} must be {list(shape)}")
         out.append(t)
     gv, gl, ga = out
+    ws, ws_bytes = None, 0
+    if isinstance(workspace, str):
+        if workspace != "auto":
+            raise ValueError("workspace must be 'auto', None or a uint8 CUDA tensor")
+        need = workspace_size(B, S, M, D, Lq, L, K)
+        ws = torch.empty(need, dtype=torch.uint8, device=dev)
+        ws_bytes = need
+    elif workspace is not None:
+        _require(workspace, "workspace", torch.uint8, dev)
+        ws, ws_bytes = workspace, workspace.numel()
     with torch.cuda.device(dev):
         stream = torch.cuda.current_stream(dev).cuda_stream
         _check(library().msda_backward(B, S, M, D, Lq, L, K, MSDA_F32, _ptr(value), _ptr(ss),
                                        _ptr(st), _ptr(sampling_locations),
                                        _ptr(attention_weights), _ptr(grad_output), _ptr(gv),
-                                       _ptr(gl), _ptr(ga), ctypes.c_void_p(stream)),
+                                       _ptr(gl), _ptr(ga), _ptr(ws), ws_bytes,
+                                       ctypes.c_void_p(stream)),
                "msda_backward")
     return gv, gl, ga
+
+
+def workspace_size(B, S, M, D, Lq, L, K) -> int:
+    """Bytes of scratch the cell-sorted backward needs (host computation)."""
+    n = ctypes.c_size_t(0)
+    _check(library().msda_backward_workspace_size(B, S, M, D, Lq, L, K, ctypes.byref(n)),
+           "msda_backward_workspace_size")
+    return int(n.value)
 
 
 class MSDeformAttnFunction(torch.autograd.Function):

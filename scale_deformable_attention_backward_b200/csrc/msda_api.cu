@@ -69,6 +69,10 @@ msda_status check_common(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq,
       !product_ok({B, Lq, M, L, K, 2}, &c->point_elems) ||
       !product_ok({B, Lq, M, D}, &c->out_elems))
     return MSDA_ERR_BAD_SHAPE;
+  // The kernels address one image's value block [S, M, D] with 32-bit offsets.
+  int64_t per_image = 0;
+  if (!product_ok({S, M, D}, &per_image) || per_image >= (int64_t(1) << 31))
+    return MSDA_ERR_UNSUPPORTED;
   return MSDA_OK;
 }
 
@@ -129,12 +133,19 @@ msda_status msda_backward(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq
                           const float* sampling_locations, const float* attention_weights,
                           const float* grad_output, float* grad_value,
                           float* grad_sampling_locations, float* grad_attention_weights,
-                          void* stream) {
+                          void* workspace, size_t workspace_bytes, void* stream) {
   Common c;
   msda_status st = check_common(B, S, M, D, Lq, L, K, &c);
   if (st != MSDA_OK) return st;
   if (value_dtype != MSDA_F32) return MSDA_ERR_UNSUPPORTED;
   if (D % 4 != 0 || D > 128 || M > INT32_MAX) return MSDA_ERR_UNSUPPORTED;
+  if (workspace != nullptr) {
+    size_t need = 0;
+    st = msda_backward_workspace_size(B, S, M, D, Lq, L, K, &need);
+    if (st != MSDA_OK) return st;
+    if (workspace_bytes < need) return MSDA_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return MSDA_ERR_MISALIGNED;
+  }
   if (c.value_elems == 0 && c.out_elems == 0) return MSDA_OK;
   if (c.value_elems > 0 && grad_value == nullptr) return MSDA_ERR_NULL_POINTER;
   if (!aligned(grad_value, 16)) return MSDA_ERR_MISALIGNED;
@@ -163,6 +174,7 @@ msda_status msda_backward(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq
   a.grad_value = grad_value;
   a.grad_sampling_locations = grad_sampling_locations;
   a.grad_attention_weights = grad_attention_weights;
+  a.B = B;
   a.S = S;
   a.Lq = Lq;
   a.M = static_cast<int>(M);
@@ -172,9 +184,28 @@ msda_status msda_backward(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq
   a.lanes = pow2_at_least(D / 4);
   a.groups = work ? B * Lq * M : 0;
   a.value_elements = c.value_elems;
-  return msda::launch_backward(a, static_cast<cudaStream_t>(stream)) == cudaSuccess
-             ? MSDA_OK
-             : MSDA_ERR_CUDA;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const cudaError_t err = workspace != nullptr ? msda::launch_backward_sorted(a, workspace, s)
+                                               : msda::launch_backward(a, s);
+  return err == cudaSuccess ? MSDA_OK : MSDA_ERR_CUDA;
+}
+
+msda_status msda_backward_workspace_size(int64_t B, int64_t S, int64_t M, int64_t D,
+                                         int64_t Lq, int64_t L, int64_t K, size_t* bytes) {
+  if (bytes == nullptr) return MSDA_ERR_NULL_POINTER;
+  *bytes = 0;
+  Common c;
+  const msda_status st = check_common(B, S, M, D, Lq, L, K, &c);
+  if (st != MSDA_OK) return st;
+  // Cell ids, slots and point ids are 32-bit in the sorted pass.
+  const int64_t cells = 2 * S + 2 * L;
+  int64_t bins = 0;
+  if (!product_ok({B, M, cells}, &bins) || bins + 1 >= (int64_t(1) << 31) ||
+      c.point_elems / 2 >= (int64_t(1) << 31))
+    return MSDA_ERR_UNSUPPORTED;
+  *bytes = static_cast<size_t>(
+      msda::sorted_layout(B, S, M, Lq, static_cast<int>(L), static_cast<int>(K)).bytes);
+  return MSDA_OK;
 }
 
 msda_status msda_check_metadata(int64_t S, int64_t L, const int64_t* shapes,
@@ -201,6 +232,7 @@ const char* msda_status_string(int status) {
     case MSDA_ERR_UNSUPPORTED: return "unsupported dtype, head dim, level count or point count";
     case MSDA_ERR_MISALIGNED: return "a pointer is not aligned as required";
     case MSDA_ERR_CUDA: return "a CUDA launch or runtime call failed";
+    case MSDA_ERR_WORKSPACE: return "the workspace is smaller than msda_backward_workspace_size";
     default: return "unknown status";
   }
 }

@@ -6,120 +6,206 @@
 // multi-scale deformable attention equation; sampling rule and output layout of
 // "Deformable DETR模型解读（附源码+论文）", ms_deform_attn_core_pytorch.
 //
-// Work decomposition: a sub-warp of LANES lanes owns one (b, q, m, channel
-// chunk) group; each lane owns 16 contiguous bytes of the head's channels, so one
-// corner of one point is a single fully used 128-byte line for D = 32 float32.
-// The group's 2*L*K locations and L*K weights are read coalesced, LANES points at
-// a time (lane j holds point j of the round), and broadcast with shuffles; every
-// lane then maps the point to its cell and gathers its slice of the four corners
-// with 16-byte read-only loads, accumulating in float32 registers.  Consecutive
-// groups are consecutive heads of consecutive queries, so the blocks resident at
-// any moment cover neighbouring queries, whose samples overlap in L1 and L2.
+// Work decomposition.  A sub-warp of LANES lanes owns one (b, q, m, channel
+// chunk) group; each lane owns 16 contiguous bytes of the head's channels, so
+// one corner of one point is a single fully used 128-byte line for D = 32
+// float32.  A block of 256 threads owns G = 256 / LANES consecutive groups and
+// walks their points in chunks of PC = 2 * LANES points per group (G * PC = 512
+// points per chunk):
+//   phase 1  every thread maps two of the chunk's points to their cell -- exact
+//            floor, corner validity, the four corners' element offsets and the
+//            four weights A * bilinear -- reading locations and weights
+//            coalesced, and writes them to shared memory (swizzled so that both
+//            the writes and the phase-2 broadcasts are free of bank conflicts);
+//   phase 2  every sub-warp reads its points' setups (one broadcast per 16
+//            bytes), gathers its slice of the four corners with 16-byte
+//            read-only loads and accumulates in float32 with packed two-wide
+//            FMAs.
+// The per-point index arithmetic is thus done once per point instead of once
+// per lane.  Consecutive groups are consecutive heads of consecutive queries and
+// a block owns one tile, so the blocks resident at a time work on neighbouring
+// queries, whose samples overlap in L2.  (Head-major tiles and per-block tile
+// ranges, which favour L1 reuse, measured slower on the encoder workload.)
 #include "msda_device.cuh"
 #include "msda_launch.h"
 
 namespace msda {
 
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kChunkPoints = 512;
+
+// The setup of one point: element offsets of its four corners relative to the
+// (b, m, channel) base pointer, -1 for a corner outside the map, in the order
+// V(x0,y0), V(x0+1,y0), V(x0,y0+1), V(x0+1,y0+1); and the four weights
+// A * bilinear in the same order.
+struct PointSetup {
+  int4 off;
+  float4 w;
+};
+
+__device__ __forceinline__ PointSetup setup_point(float lx, float ly, float a, int H, int W,
+                                                  long long start, int MD) {
+  const Cell c = locate(lx, ly, H, W);
+  const float hx = 1.0f - c.fx, hy = 1.0f - c.fy;
+  PointSetup s;
+  s.w = make_float4(a * hx * hy, a * c.fx * hy, a * hx * c.fy, a * c.fx * c.fy);
+  const int base = static_cast<int>(start + static_cast<long long>(c.y0) * W + c.x0);
+  // Offsets are formed only for corners inside the map, where 0 <= pixel < S and
+  // pixel * M * D < 2^31 (checked by the C ABI).
+  s.off.x = (c.vx0 && c.vy0) ? base * MD : -1;
+  s.off.y = (c.vx1 && c.vy0) ? (base + 1) * MD : -1;
+  s.off.z = (c.vx0 && c.vy1) ? (base + W) * MD : -1;
+  s.off.w = (c.vx1 && c.vy1) ? (base + W + 1) * MD : -1;
+  // A point with no corner in the map adds A * 0 to the output, which is NaN when
+  // its weights are not finite (a non-finite location or weight).  Such a point
+  // reads the level's first pixel with a NaN weight, so the NaN reaches the sum.
+  if ((s.off.x & s.off.y & s.off.z & s.off.w) < 0 && W > 0 &&
+      !isfinite(s.w.x + s.w.y + s.w.z + s.w.w)) {
+    s.off.x = static_cast<int>(start) * MD;
+    s.w.x = __int_as_float(0x7fffffff);
+  }
+  return s;
+}
+
+// Packed float32 pair FMA (sm_100): d = a * b + c on both halves.
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;"
+      : "=l"(d)
+      : "l"(*reinterpret_cast<unsigned long long*>(&a)),
+        "l"(*reinterpret_cast<unsigned long long*>(&b)),
+        "l"(*reinterpret_cast<unsigned long long*>(&c)));
+  return *reinterpret_cast<float2*>(&d);
+}
+
+template <typename T>
+struct Corner;
+
+template <>
+struct Corner<float> {
+  static constexpr int N = 4;
+  // acc += w * value[0..3] for one corner inside the map.
+  __device__ __forceinline__ static void accumulate(const float* p, float w, float2 (&acc)[2]) {
+    const float4 v = __ldg(reinterpret_cast<const float4*>(p));
+    const float2 ww = make_float2(w, w);
+    acc[0] = fma2(ww, make_float2(v.x, v.y), acc[0]);
+    acc[1] = fma2(ww, make_float2(v.z, v.w), acc[1]);
+  }
+  __device__ __forceinline__ static void store(float* p, const float2 (&acc)[2]) {
+    *reinterpret_cast<float4*>(p) = make_float4(acc[0].x, acc[0].y, acc[1].x, acc[1].y);
+  }
+};
+
+template <>
+struct Corner<__nv_bfloat16> {
+  static constexpr int N = 8;
+  __device__ __forceinline__ static void accumulate(const __nv_bfloat16* p, float w,
+                                                    float2 (&acc)[4]) {
+    const uint4 r = __ldg(reinterpret_cast<const uint4*>(p));
+    const unsigned u[4] = {r.x, r.y, r.z, r.w};
+    const float2 ww = make_float2(w, w);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      acc[i] = fma2(ww, make_float2(__uint_as_float(u[i] << 16),
+                                    __uint_as_float(u[i] & 0xffff0000u)), acc[i]);
+  }
+  __device__ __forceinline__ static void store(__nv_bfloat16* p, const float2 (&acc)[4]) {
+    unsigned u[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __nv_bfloat162 h = __floats2bfloat162_rn(acc[i].x, acc[i].y);
+      u[i] = *reinterpret_cast<const unsigned*>(&h);
+    }
+    *reinterpret_cast<uint4*>(p) = make_uint4(u[0], u[1], u[2], u[3]);
+  }
+};
+
+}  // namespace
+
 template <typename T, int LANES>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(kThreads)
 forward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial_shapes,
                const int64_t* __restrict__ level_start_index,
                const float* __restrict__ sampling_locations,
                const float* __restrict__ attention_weights, T* __restrict__ output,
                long long S, int M, int D, long long Lq, int L, int K, int chunks,
                long long groups) {
-  using V = Vec<T>;
-  constexpr int E = V::N;
+  using C = Corner<T>;
+  constexpr int E = C::N;
+  constexpr int G = kThreads / LANES;   // groups per block
+  constexpr int PC = kChunkPoints / G;  // points per group per chunk (= 2 * LANES)
+  static_assert(G >= 8, "the shared-memory swizzle needs at least 8 groups per block");
   __shared__ Levels lv;
+  __shared__ int4 s_off[kChunkPoints];
+  __shared__ float4 s_w[kChunkPoints];
   stage_levels(lv, spatial_shapes, level_start_index, L, S);
 
   const int lane = threadIdx.x % LANES;
-  const int groups_per_block = blockDim.x / LANES;
+  const int gi = threadIdx.x / LANES;
   const int LK = L * K;
-  const long long MD = static_cast<long long>(M) * D;
+  const int MD = M * D;
 
-  for (long long g0 = static_cast<long long>(blockIdx.x) * groups_per_block; g0 < groups;
-       g0 += static_cast<long long>(gridDim.x) * groups_per_block) {
-    const long long g_raw = g0 + threadIdx.x / LANES;
+  for (long long g0 = static_cast<long long>(blockIdx.x) * G; g0 < groups;
+       g0 += static_cast<long long>(gridDim.x) * G) {
+    const long long g_raw = g0 + gi;
     const bool active = g_raw < groups;
-    // Inactive groups (the tail of the last block) still take part in the
-    // shuffles, on a clamped group, and store nothing.
     const Group grp = decompose(active ? g_raw : groups - 1, chunks, M, Lq);
     const int ch = (grp.chunk * LANES + lane) * E;
     const bool lane_on = active && ch < D;  // clamped tail groups touch no memory
     const T* vbase = value + (grp.b * S * M + grp.m) * static_cast<long long>(D) + ch;
-    const float* gloc = sampling_locations + grp.bqm * LK * 2;
-    const float* gatt = attention_weights + grp.bqm * LK;
 
-    float acc[E];
+    float2 acc[E / 2];
 #pragma unroll
-    for (int e = 0; e < E; ++e) acc[e] = 0.0f;
+    for (int e = 0; e < E / 2; ++e) acc[e] = make_float2(0.0f, 0.0f);
 
-    int l = 0, k = 0;
-    int H = lv.H[0], W = lv.W[0];
-    long long start = lv.start[0];
-    for (int p0 = 0; p0 < LK; p0 += LANES) {
-      const int pj = p0 + lane;
-      float2 xy = make_float2(0.0f, 0.0f);
-      float aj = 0.0f;
-      if (pj < LK) {
-        xy = __ldg(reinterpret_cast<const float2*>(gloc) + pj);
-        aj = __ldg(gatt + pj);
-      }
-      const int n = min(LANES, LK - p0);
-      for (int j = 0; j < n; ++j) {
-        const float lx = __shfl_sync(kFullMask, xy.x, j, LANES);
-        const float ly = __shfl_sync(kFullMask, xy.y, j, LANES);
-        const float a = __shfl_sync(kFullMask, aj, j, LANES);
-        const Cell c = locate(lx, ly, H, W);
-        if (lane_on) {
-          // Corner weights, w<i><j> for V(x0 + i, y0 + j).
-          const float hx = 1.0f - c.fx, hy = 1.0f - c.fy;
-          const float w00 = a * hx * hy, w10 = a * c.fx * hy;
-          const float w01 = a * hx * c.fy, w11 = a * c.fx * c.fy;
-          const long long row = static_cast<long long>(W) * MD;
-          const long long off = (start + static_cast<long long>(c.y0) * W + c.x0) * MD;
-          float v[E];
+    for (int p0 = 0; p0 < LK; p0 += PC) {
+      const int pc = min(PC, LK - p0);
+      // Phase 1: setups of this chunk's points; thread t takes point tj of group tg.
 #pragma unroll
-          for (int e = 0; e < E; ++e) v[e] = 0.0f;
-          if (c.vx0 && c.vy0) V::load(vbase + off, v);
-#pragma unroll
-          for (int e = 0; e < E; ++e) acc[e] = fmaf(w00, v[e], acc[e]);
-#pragma unroll
-          for (int e = 0; e < E; ++e) v[e] = 0.0f;
-          if (c.vx1 && c.vy0) V::load(vbase + off + MD, v);
-#pragma unroll
-          for (int e = 0; e < E; ++e) acc[e] = fmaf(w10, v[e], acc[e]);
-#pragma unroll
-          for (int e = 0; e < E; ++e) v[e] = 0.0f;
-          if (c.vx0 && c.vy1) V::load(vbase + off + row, v);
-#pragma unroll
-          for (int e = 0; e < E; ++e) acc[e] = fmaf(w01, v[e], acc[e]);
-#pragma unroll
-          for (int e = 0; e < E; ++e) v[e] = 0.0f;
-          if (c.vx1 && c.vy1) V::load(vbase + off + row + MD, v);
-#pragma unroll
-          for (int e = 0; e < E; ++e) acc[e] = fmaf(w11, v[e], acc[e]);
-        }
-        if (++k == K) {
-          k = 0;
-          if (++l < L) {
-            H = lv.H[l];
-            W = lv.W[l];
-            start = lv.start[l];
-          }
+      for (int t = threadIdx.x; t < kChunkPoints; t += kThreads) {
+        const int tg = t / PC, tj = t % PC;
+        const long long g = g0 + tg;
+        if (tj < pc && g < groups) {
+          const long long bqm = g / chunks;
+          const int p = p0 + tj;
+          const int l = p / K;
+          const float2 xy = __ldg(reinterpret_cast<const float2*>(sampling_locations) +
+                                  bqm * LK + p);
+          const float a = __ldg(attention_weights + bqm * LK + p);
+          const PointSetup su = setup_point(xy.x, xy.y, a, lv.H[l], lv.W[l], lv.start[l], MD);
+          const int slot = tj * G + (tg ^ (tj & 7));
+          s_off[slot] = su.off;
+          s_w[slot] = su.w;
         }
       }
+      __syncthreads();
+      // Phase 2: gather and accumulate.
+      if (lane_on) {
+#pragma unroll 4
+        for (int j = 0; j < pc; ++j) {
+          const int slot = j * G + (gi ^ (j & 7));
+          const int4 o = s_off[slot];
+          const float4 w = s_w[slot];
+          if (o.x >= 0) C::accumulate(vbase + o.x, w.x, acc);
+          if (o.y >= 0) C::accumulate(vbase + o.y, w.y, acc);
+          if (o.z >= 0) C::accumulate(vbase + o.z, w.z, acc);
+          if (o.w >= 0) C::accumulate(vbase + o.w, w.w, acc);
+        }
+      }
+      __syncthreads();
     }
-    if (lane_on) V::store(output + grp.bq * MD + static_cast<long long>(grp.m) * D + ch, acc);
+    if (lane_on) C::store(output + grp.bq * MD + static_cast<long long>(grp.m) * D + ch, acc);
   }
 }
 
+// One block per tile: the block scheduler hands tiles out in order as SMs free
+// up, so the resident blocks always cover a window of neighbouring queries.
 template <typename T, int LANES>
 static cudaError_t launch_forward_t(const ForwardArgs& a, cudaStream_t stream) {
-  constexpr int kThreads = 256;
-  const long long per_block = kThreads / LANES;
-  long long blocks = (a.groups + per_block - 1) / per_block;
+  constexpr int G = kThreads / LANES;
+  long long blocks = (a.groups + G - 1) / G;
   if (blocks > (1ll << 30)) blocks = 1ll << 30;
   forward_kernel<T, LANES><<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(
       static_cast<const T*>(a.value), a.spatial_shapes, a.level_start_index,

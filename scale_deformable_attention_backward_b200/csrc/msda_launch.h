@@ -36,15 +36,30 @@ struct BackwardArgs {
   float* grad_value;
   float* grad_sampling_locations;
   float* grad_attention_weights;
-  long long S, Lq;
+  long long B, S, Lq;
   int M, D, L, K;
   int lanes;         // lanes per (b, q, m) group; D <= 4 * lanes
   long long groups;  // B * Lq * M
   long long value_elements;  // B * S * M * D (grad_value is zeroed first)
 };
 
+// Scratch layout of the cell-sorted backward (msda_backward_sorted.cu).
+struct SortedLayout {
+  long long cells_per_bm;  // bound on sum_l (H_l + 1)(W_l + 1) from S and L alone
+  long long bins;          // B * M * cells_per_bm
+  long long points;        // B * Lq * M * L * K
+  long long scan_tiles;
+  long long bytes;         // workspace bytes
+};
+
+SortedLayout sorted_layout(long long B, long long S, long long M, long long Lq, int L, int K);
+
 cudaError_t launch_forward(const ForwardArgs& a, cudaStream_t stream);
+// Backward with one vector atomic per point corner (no scratch).
 cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t stream);
+// Backward with the points grouped by cell; `workspace` holds sorted_layout().bytes.
+cudaError_t launch_backward_sorted(const BackwardArgs& a, void* workspace, cudaStream_t stream);
 cudaError_t launch_zero(float* p, long long n, cudaStream_t stream);
+cudaError_t launch_zero_words(int* p, long long n, cudaStream_t stream);
 
 }  // namespace msda

@@ -44,12 +44,29 @@ def gpu_forward(d):
     return out.float().cpu().numpy().astype(np.float64)
 
 
-def gpu_backward(d):
+BACKWARD_PATHS = ("sorted", "direct")
+
+
+def gpu_backward(d, path="sorted"):
+    """Backward through the C ABI: ``sorted`` passes a workspace (cell-sorted
+    kernels), ``direct`` passes none (one atomic per point corner)."""
     gv, gl, ga = binding.backward(d["value"], d["spatial_shapes"], d["level_start_index"],
                                   d["sampling_locations"], d["attention_weights"],
-                                  d["grad_output"])
+                                  d["grad_output"],
+                                  workspace="auto" if path == "sorted" else None)
     torch.cuda.synchronize()
     return tuple(t.cpu().numpy().astype(np.float64) for t in (gv, gl, ga))
+
+
+def check_backward_paths(d, inp, what=""):
+    """Both backward paths against one oracle backward."""
+    rv, rl, ra = oracle_backward(inp)
+    for path in BACKWARD_PATHS:
+        gv, gl, ga = gpu_backward(d, path)
+        tag = f" {what} ({path})"
+        assert_backward_f32(gv, rv, "grad_value" + tag)
+        assert_backward_f32(gl, rl, "grad_sampling_locations" + tag)
+        assert_backward_f32(ga, ra, "grad_attention_weights" + tag)
 
 
 def oracle_forward(inp):

@@ -12,7 +12,7 @@ from scale_deformable_attention_backward_b200 import binding
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "msda.h")
 
-OK, NULLP, BAD, UNSUP, MISAL = 0, 1, 2, 3, 4
+OK, NULLP, BAD, UNSUP, MISAL, CUDA, WORKSPACE = 0, 1, 2, 3, 4, 5, 6
 
 
 def declared_functions():
@@ -35,7 +35,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_status_strings_and_version(lib):
-    for code in range(6):
+    for code in range(7):
         assert lib.msda_status_string(code)
     assert lib.msda_status_string(99) == b"unknown status"
     assert lib.msda_version() >= 100
@@ -70,10 +70,17 @@ def _fwd(lib, B=1, S=80, M=2, D=8, Lq=80, L=2, K=2, dtype=0, value=FAKE, shapes=
                             v(attn), v(out), None)
 
 
-def _bwd(lib, B=1, S=80, M=2, D=8, Lq=80, L=2, K=2, dtype=0, ptrs=None):
+def _bwd(lib, B=1, S=80, M=2, D=8, Lq=80, L=2, K=2, dtype=0, ptrs=None, ws=None, ws_bytes=0):
     p = [FAKE] * 9 if ptrs is None else ptrs
     v = lambda x: None if x is None else ctypes.c_void_p(x)
-    return lib.msda_backward(B, S, M, D, Lq, L, K, dtype, *[v(x) for x in p], None)
+    return lib.msda_backward(B, S, M, D, Lq, L, K, dtype, *[v(x) for x in p], v(ws), ws_bytes,
+                             None)
+
+
+def _ws_size(lib, B=1, S=80, M=2, D=8, Lq=80, L=2, K=2):
+    n = ctypes.c_size_t(0)
+    st = lib.msda_backward_workspace_size(B, S, M, D, Lq, L, K, ctypes.byref(n))
+    return st, n.value
 
 
 def test_forward_argument_errors(lib):
@@ -120,3 +127,20 @@ def test_backward_argument_errors(lib):
     p[7] = FAKE + 4                                # grad_sampling_locations
     assert _bwd(lib, ptrs=p) == MISAL
     assert _bwd(lib, B=0, ptrs=[None] * 9) == OK  # nothing to write at all
+    # A workspace that is too small, or misaligned, is rejected before any launch.
+    st, need = _ws_size(lib)
+    assert st == OK and need > 0
+    assert _bwd(lib, ws=FAKE, ws_bytes=need - 1) == WORKSPACE
+    assert _bwd(lib, ws=FAKE + 16, ws_bytes=need) == MISAL
+
+
+def test_workspace_size(lib):
+    st, need = _ws_size(lib, B=4, S=19947, M=8, D=32, Lq=19947, L=4, K=4)
+    assert st == OK
+    points = 4 * 19947 * 8 * 16
+    bins = 4 * 8 * (2 * 19947 + 8)
+    assert need >= 24 * points + 4 * (bins + 1)
+    assert need < 24 * points + 4 * (bins + 1) + 64 * 1024
+    assert _ws_size(lib, B=-1)[0] == BAD
+    assert _ws_size(lib, B=1 << 20, S=1 << 12, M=8)[0] == UNSUP  # 32-bit cell ids overflow
+    assert lib.msda_backward_workspace_size(1, 80, 2, 8, 80, 2, 2, None) == NULLP

@@ -45,11 +45,7 @@ def test_random_shapes_f32(D, shapes_id):
     inp = random_inputs(100 + D + shapes_id, B=2, M=3, D=D, K=3, shapes=shapes, Lq=37)
     d = G.device_inputs(inp)
     G.assert_forward_f32(G.gpu_forward(d), G.oracle_forward(inp), f"forward D={D}")
-    gv, gl, ga = G.gpu_backward(d)
-    rv, rl, ra = G.oracle_backward(inp)
-    G.assert_backward_f32(gv, rv, "grad_value")
-    G.assert_backward_f32(gl, rl, "grad_sampling_locations")
-    G.assert_backward_f32(ga, ra, "grad_attention_weights")
+    G.check_backward_paths(d, inp)
 
 
 @pytest.mark.parametrize("D", [256, 384])
@@ -73,11 +69,7 @@ def test_level_and_point_counts(L, K):
     inp = random_inputs(300 + L + K, B=1, M=2, D=8, K=K, shapes=shapes, Lq=13)
     d = G.device_inputs(inp)
     G.assert_forward_f32(G.gpu_forward(d), G.oracle_forward(inp))
-    gv, gl, ga = G.gpu_backward(d)
-    rv, rl, ra = G.oracle_backward(inp)
-    G.assert_backward_f32(gv, rv, "grad_value")
-    G.assert_backward_f32(gl, rl, "grad_sampling_locations")
-    G.assert_backward_f32(ga, ra, "grad_attention_weights")
+    G.check_backward_paths(d, inp)
 
 
 def test_locations_at_pixel_boundaries():
@@ -105,11 +97,7 @@ def test_locations_at_pixel_boundaries():
     inp = dataclasses.replace(inp, sampling_locations=loc)
     d = G.device_inputs(inp)
     G.assert_forward_f32(G.gpu_forward(d), G.oracle_forward(inp))
-    gv, gl, ga = G.gpu_backward(d)
-    rv, rl, ra = G.oracle_backward(inp)
-    G.assert_backward_f32(gl, rl, "grad_sampling_locations at pixel boundaries")
-    G.assert_backward_f32(gv, rv, "grad_value")
-    G.assert_backward_f32(ga, ra, "grad_attention_weights")
+    G.check_backward_paths(d, inp, "at pixel boundaries")
 
 
 def test_far_and_nonfinite_locations():
@@ -125,11 +113,7 @@ def test_far_and_nonfinite_locations():
     inp = dataclasses.replace(inp, sampling_locations=loc)
     d = G.device_inputs(inp)
     G.assert_forward_f32(G.gpu_forward(d), G.oracle_forward(inp))
-    gv, gl, ga = G.gpu_backward(d)
-    rv, rl, ra = G.oracle_backward(inp)
-    G.assert_backward_f32(gv, rv, "grad_value")
-    G.assert_backward_f32(gl, rl, "grad_sampling_locations")
-    G.assert_backward_f32(ga, ra, "grad_attention_weights")
+    G.check_backward_paths(d, inp)
 
 
 def test_empty_calls():
@@ -166,20 +150,42 @@ def test_guard_bands_untouched():
     ob, out = _guarded((B, Lq, M * D), sentinel)
     binding.forward(d["value"], d["spatial_shapes"], d["level_start_index"],
                     d["sampling_locations"], d["attention_weights"], output=out)
-    vb, gv = _guarded((B, S, M, D), sentinel)
-    lb, gl = _guarded((B, Lq, M, L, K, 2), sentinel)
-    ab, ga = _guarded((B, Lq, M, L, K), sentinel)
-    binding.backward(d["value"], d["spatial_shapes"], d["level_start_index"],
-                     d["sampling_locations"], d["attention_weights"], d["grad_output"],
-                     grad_value=gv, grad_sampling_locations=gl, grad_attention_weights=ga)
     torch.cuda.synchronize()
-    for buf in (ob, vb, lb, ab):
-        assert torch.all(buf[:64] == sentinel) and torch.all(buf[-64:] == sentinel)
+    assert torch.all(ob[:64] == sentinel) and torch.all(ob[-64:] == sentinel)
     G.assert_forward_f32(out.double().cpu().numpy(), G.oracle_forward(inp))
     rv, rl, ra = G.oracle_backward(inp)
-    G.assert_backward_f32(gv.double().cpu().numpy(), rv, "grad_value")
-    G.assert_backward_f32(gl.double().cpu().numpy(), rl, "grad_sampling_locations")
-    G.assert_backward_f32(ga.double().cpu().numpy(), ra, "grad_attention_weights")
+    need = binding.workspace_size(B, S, M, D, Lq, L, K)
+    for path in G.BACKWARD_PATHS:
+        vb, gv = _guarded((B, S, M, D), sentinel)
+        lb, gl = _guarded((B, Lq, M, L, K, 2), sentinel)
+        ab, ga = _guarded((B, Lq, M, L, K), sentinel)
+        # The workspace sits between two guard bands of its own (256-byte aligned).
+        wb = torch.full((need + 2 * 512,), 0x5A, dtype=torch.uint8, device="cuda")
+        ws = wb[512:512 + need] if path == "sorted" else None
+        binding.backward(d["value"], d["spatial_shapes"], d["level_start_index"],
+                         d["sampling_locations"], d["attention_weights"], d["grad_output"],
+                         grad_value=gv, grad_sampling_locations=gl, grad_attention_weights=ga,
+                         workspace=ws)
+        torch.cuda.synchronize()
+        for buf in (vb, lb, ab):
+            assert torch.all(buf[:64] == sentinel) and torch.all(buf[-64:] == sentinel), path
+        assert torch.all(wb[:512] == 0x5A) and torch.all(wb[-512:] == 0x5A), path
+        G.assert_backward_f32(gv.double().cpu().numpy(), rv, f"grad_value ({path})")
+        G.assert_backward_f32(gl.double().cpu().numpy(), rl, f"grad_sampling_locations ({path})")
+        G.assert_backward_f32(ga.double().cpu().numpy(), ra, f"grad_attention_weights ({path})")
+
+
+def test_workspace_too_small_is_rejected():
+    inp = random_inputs(15, B=1, M=2, D=8, K=2, shapes=SHAPES[0], Lq=4)
+    d = G.device_inputs(inp)
+    B, S, M, D = inp.value.shape
+    need = binding.workspace_size(B, S, M, D, 4, 1, 2)
+    small = torch.empty(need - 256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(binding.MSDAError) as e:
+        binding.backward(d["value"], d["spatial_shapes"], d["level_start_index"],
+                         d["sampling_locations"], d["attention_weights"], d["grad_output"],
+                         workspace=small)
+    assert e.value.status == 6
 
 
 def test_misaligned_pointer_is_rejected():
@@ -207,8 +213,9 @@ def test_inconsistent_device_metadata_is_memory_safe():
     attn[:, :, :, 2, :] = 0.0
     ref = G.oracle_forward(dataclasses.replace(inp, attention_weights=attn))
     G.assert_forward_f32(got, ref, "forward with an overrunning level")
-    gv, gl, ga = G.gpu_backward(d)
-    assert np.all(gl[:, :, :, 2] == 0.0) and np.all(ga[:, :, :, 2] == 0.0)
+    for path in G.BACKWARD_PATHS:
+        gv, gl, ga = G.gpu_backward(d, path)
+        assert np.all(gl[:, :, :, 2] == 0.0) and np.all(ga[:, :, :, 2] == 0.0), path
 
 
 def test_host_metadata_is_checked():

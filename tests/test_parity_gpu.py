@@ -28,11 +28,24 @@ def test_forward_matches_oracle_full_size(name):
 def test_backward_matches_oracle_full_size(name):
     cfg = W.CONFIGS[name]
     inp = W.make_inputs(cfg, seed=0)
-    gv, gl, ga = G.gpu_backward(G.device_inputs(inp))
+    d = G.device_inputs(inp)
     rv, rl, ra = G.oracle_backward(inp)
-    G.assert_backward_f32(gv, rv, f"{name} grad_value")
-    G.assert_backward_f32(gl, rl, f"{name} grad_sampling_locations")
-    G.assert_backward_f32(ga, ra, f"{name} grad_attention_weights")
+    for path in G.BACKWARD_PATHS:
+        gv, gl, ga = G.gpu_backward(d, path)
+        G.assert_backward_f32(gv, rv, f"{name} grad_value ({path})")
+        G.assert_backward_f32(gl, rl, f"{name} grad_sampling_locations ({path})")
+        G.assert_backward_f32(ga, ra, f"{name} grad_attention_weights ({path})")
+
+
+def test_sorted_backward_location_gradients_are_deterministic():
+    """Per-point gradients of the cell-sorted path do not depend on the order
+    the atomics give the points inside a cell."""
+    inp = W.make_inputs(W.CONFIGS["encoder_train_fp32"].with_batch(1), seed=2)
+    d = G.device_inputs(inp)
+    first = G.gpu_backward(d, "sorted")
+    for _ in range(2):
+        again = G.gpu_backward(d, "sorted")
+        assert np.array_equal(first[1], again[1]) and np.array_equal(first[2], again[2])
 
 
 @pytest.mark.parametrize("name", ["encoder_fp32", "decoder_fp32"])
