@@ -53,9 +53,8 @@ FORWARD_WORKLOAD = "encoder_fp32"
 METRIC = "MSDeformAttn fwd/bwd queries/sec and achieved HBM GB/s vs B200 peak (1 GPU)"
 FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
-# msda_backward with a workspace: zero grad_value, zero cell counts, bin, three
-# scan passes, place, cells.
-BACKWARD_LAUNCHES = 8
+# msda_backward without a workspace (the timed path): zero grad_value, backward.
+BACKWARD_LAUNCHES = 2
 KERNEL_SOURCES = os.path.join(ROOT, "scale_deformable_attention_backward_b200", "csrc")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 
@@ -265,11 +264,11 @@ def run_b200(args, world, rank, local):
         binding.forward(d["value"], d["spatial_shapes"], d["level_start_index"],
                         d["sampling_locations"], d["attention_weights"], output=out)
 
-    def step_bwd():
+    def step_bwd(workspace=None):
         binding.backward(d["value"], d["spatial_shapes"], d["level_start_index"],
                          d["sampling_locations"], d["attention_weights"], d["grad_output"],
                          grad_value=gv, grad_sampling_locations=gl, grad_attention_weights=ga,
-                         workspace=ws)
+                         workspace=workspace)
 
     for _ in range(args.warmup):
         flush.fill_(1.0)
@@ -310,9 +309,8 @@ def run_b200(args, world, rank, local):
     roofline = {
         "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
         "frac": round(achieved / peak, 4), "traffic": recorded_traffic(f"{STEP_WORKLOAD}.{dom}"),
-        "kernel": (f"msda_backward launch sequence ({BACKWARD_LAUNCHES} kernels: zero fills, "
-                   "bin, 3-pass scan, place, cell)" if dom == "backward"
-                   else "msda_forward: forward_kernel"),
+        "kernel": ("msda_backward without workspace: zero_kernel + backward_kernel"
+                   if dom == "backward" else "msda_forward: forward_kernel"),
         "algorithmic_bytes": algo[dom], "mean_ms": round(dom_ms, 4),
         "peak_source": f"{peak_kind} HBM copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
                        if peak_kind == "measured" else "fallback 6.65 TB/s",
@@ -327,6 +325,25 @@ def run_b200(args, world, rank, local):
                          "traffic": recorded_traffic(f"{STEP_WORKLOAD}.backward")},
         },
     }
+
+    # The cell-sorted backward (with a workspace), timed alone for reference.
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        step_bwd(ws)
+    se0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    se1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        se0[i].record(stream)
+        step_bwd(ws)
+        se1[i].record(stream)
+    torch.cuda.synchronize()
+    sorted_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(se0, se1))
+    roofline["other"]["backward_sorted"] = {
+        "mean_ms": round(sorted_ms, 4),
+        "achieved_gbs": round(algo["backward"] / (sorted_ms * 1e-3) / 1e9, 1),
+        "note": "cell-sorted path (msda_backward with a workspace), not the timed step"}
 
     # The encoder self-attention forward alone (B=2), the spec workload.
     fcfg = W.CONFIGS[FORWARD_WORKLOAD]
@@ -438,14 +455,15 @@ def run_case(args, local):
     torch.cuda.set_device(device)
     name = FORWARD_WORKLOAD if args.case == "forward_encoder" else STEP_WORKLOAD
     cfg = W.CONFIGS[name]
-    inp = W.make_inputs(cfg, seed=0, with_grad=args.case == "backward")
+    inp = W.make_inputs(cfg, seed=0, with_grad=args.case.startswith("backward"))
     d = _device_inputs(inp, device)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
 
     def launch():
-        if args.case == "backward":
+        if args.case.startswith("backward"):
             binding.backward(d["value"], d["spatial_shapes"], d["level_start_index"],
-                             d["sampling_locations"], d["attention_weights"], d["grad_output"])
+                             d["sampling_locations"], d["attention_weights"], d["grad_output"],
+                             workspace="auto" if args.case == "backward_sorted" else None)
         else:
             binding.forward(d["value"], d["spatial_shapes"], d["level_start_index"],
                             d["sampling_locations"], d["attention_weights"])
@@ -514,7 +532,8 @@ def parse_args(argv=None):
     p.add_argument("--impl", choices=["b200", "reference"], default="b200")
     p.add_argument("--no-cpu-baseline", action="store_true",
                    help="skip the CPU oracle timing (it takes ~10-20 s)")
-    p.add_argument("--case", choices=["step", "forward", "forward_encoder", "backward"],
+    p.add_argument("--case", choices=["step", "forward", "forward_encoder", "backward",
+                                      "backward_sorted"],
                    default="step",
                    help="time one launch type alone (for profiler captures) instead of "
                         "the full benchmark")

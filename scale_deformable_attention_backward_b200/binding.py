@@ -165,14 +165,15 @@ def backward(value: torch.Tensor, spatial_shapes, level_start_index,
              grad_value: Optional[torch.Tensor] = None,
              grad_sampling_locations: Optional[torch.Tensor] = None,
              grad_attention_weights: Optional[torch.Tensor] = None,
-             workspace="auto",
+             workspace=None,
              ) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
     """MSDeformAttn backward: (grad_value, grad_sampling_locations,
     grad_attention_weights), all float32.
 
-    ``workspace``: ``"auto"`` (default) takes scratch for the cell-sorted path
-    from torch's caching allocator; a uint8 CUDA tensor supplies it; ``None``
-    selects the scratch-free path (one atomic per point corner)."""
+    ``workspace``: ``None`` (default) selects the scratch-free path (one vector
+    atomic per point corner), the faster one on the encoder workloads;
+    ``"auto"`` takes scratch for the cell-sorted path from torch's caching
+    allocator, and a uint8 CUDA tensor supplies that scratch."""
     dev = value.device
     B, S, M, D, Lq, L, K = _dims(value, sampling_locations, attention_weights)
     _require(value, "value", torch.float32, dev)

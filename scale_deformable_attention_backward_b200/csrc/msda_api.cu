@@ -197,11 +197,10 @@ msda_status msda_backward_workspace_size(int64_t B, int64_t S, int64_t M, int64_
   Common c;
   const msda_status st = check_common(B, S, M, D, Lq, L, K, &c);
   if (st != MSDA_OK) return st;
-  // Cell ids, slots and point ids are 32-bit in the sorted pass.
-  const int64_t cells = 2 * S + 2 * L;
-  int64_t bins = 0;
-  if (!product_ok({B, M, cells}, &bins) || bins + 1 >= (int64_t(1) << 31) ||
-      c.point_elems / 2 >= (int64_t(1) << 31))
+  // Point ids, record positions and cell keys are 32-bit in the sorted pass.
+  int64_t keys = 0;
+  if (c.point_elems / 2 >= (int64_t(1) << 31) || !product_ok({B, M, 2 * S + 2 * L}, &keys) ||
+      keys >= (int64_t(1) << 31))
     return MSDA_ERR_UNSUPPORTED;
   *bytes = static_cast<size_t>(
       msda::sorted_layout(B, S, M, Lq, static_cast<int>(L), static_cast<int>(K)).bytes);

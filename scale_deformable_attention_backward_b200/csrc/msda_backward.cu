@@ -161,20 +161,6 @@ cudaError_t launch_zero(float* p, long long n, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-__global__ void zero_words_kernel(int* __restrict__ p, long long n) {
-  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
-       i += static_cast<long long>(gridDim.x) * blockDim.x)
-    p[i] = 0;
-}
-
-cudaError_t launch_zero_words(int* p, long long n, cudaStream_t stream) {
-  if (n <= 0) return cudaSuccess;
-  long long blocks = (n + 255) / 256;
-  if (blocks > 148 * 16) blocks = 148 * 16;
-  zero_words_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p, n);
-  return cudaGetLastError();
-}
-
 template <int LANES>
 static cudaError_t launch_backward_t(const BackwardArgs& a, cudaStream_t stream) {
   constexpr int kThreads = 256;

@@ -12,26 +12,44 @@
 //     grad_loc.x = A W (hy (G10 - G00) + fy (G11 - G01))
 //     grad_loc.y = A H (hx (G01 - G00) + fx (G11 - G10))
 // and its grad_value contribution to corner ij is A w_ij gO.  Points that
-// share a cell (the same (b, m, level, x0, y0)) share the four corner rows of
-// value and the four target rows of grad_value, so they are processed together:
+// share a cell (the same (b, m, level, x0, y0)) add to the same four rows of
+// grad_value, so they are summed in registers first.
 //
-//   1. bin     one thread per point: the cell of the point, a slot in it
-//              (atomic increment of the cell's count); points with no corner in
-//              the map get their (zero or NaN) gradients here and no slot;
-//   2. scan    exclusive prefix sum of the counts (three small launches);
-//   3. place   one thread per point: its (id, A, fx, fy) record at
-//              offset[cell] + slot;
-//   4. cells   a sub-warp per cell: the four corner rows loaded once, then for
-//              every point of the cell one 16-byte load of grad_output per lane,
-//              the four partial dot products and the four grad_value
-//              accumulators in registers; dot products are reduced for a batch
-//              of points at once (reduce-scatter across the lanes, so lane j
-//              finishes point j), and each corner gets one vector atomic per
-//              cell instead of one per point.
+// Why sort: measured on B200, L2 serves about 4.8e10 atomic requests per second
+// (one request = one 128-byte line, whether it carries a 16-byte vector
+// reduction from each of 8 lanes or a bulk TMA reduction), i.e. about 1.5e12
+// float adds/s.  One atomic per point corner costs ~0.85 ms on the encoder
+// training workload; one per cell corner a few tens of microseconds.  Global
+// atomics are kept out of the sort as well (a per-point global counter costs as
+// much as the scatter it replaces).
 //
-// Scratch (caller-provided workspace, see msda_backward_workspace_size): cell
-// counts / offsets, scan block sums, one (cell, slot) pair and one 16-byte
-// record per point.
+// A segment is one (b, m, level); it holds Lq * K points, cut into chunks of
+// kChunkPoints.  The cells of a segment are indexed (y0 + 1)(W + 1) + (x0 + 1),
+// x0 in [-1, W-1], y0 in [-1, H-1]; key = (b * M + m) * cells_per_bm + base_l +
+// cell identifies a cell globally (base_l: cells of the levels before l).
+//
+//   1. hist    one block per (segment, chunk): the cell of each point and its slot
+//              among the chunk's points of that cell (shared-memory atomic);
+//              the chunk's per-cell counts go to counts[key][chunk].  Points with
+//              no corner in the map get their (zero or NaN) gradients here.
+//   2. scan    exclusive prefix sum over counts (three launches): the position of
+//              every (cell, chunk) run in the sorted record array.
+//   3. place   one block per (segment, chunk): each point's record (id, A, fx,
+//              fy) and key at counts[key][chunk] + slot.
+//   4. cells   every sub-warp takes a fixed run of consecutive records, so the
+//              work is balanced whatever the cell sizes.  For a batch of records
+//              it issues all their corner and grad_output loads at once (in sorted
+//              order the corners are mostly L1 hits), forms the four dot
+//              products and adds A w_ij gO into four accumulators that belong to
+//              the current cell; when the cell changes they are flushed with one
+//              16-byte vector atomic per lane and corner (two when the next cell
+//              is the right neighbour, whose left column they share).  Dot
+//              products are reduced for a batch at once (reduce-scatter across
+//              the lanes; lane j finishes record j).
+//
+// Scratch (caller-provided workspace, see msda_backward_workspace_size): counts
+// per (cell, chunk), scan tile sums, the slot of every point, and the sorted
+// records (16 bytes) and keys (4 bytes).
 #include "msda_device.cuh"
 #include "msda_launch.h"
 
@@ -40,15 +58,19 @@ namespace msda {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kScanItems = 8;                        // per thread
-constexpr int kScanTile = kThreads * kScanItems;     // elements per scan block
+constexpr int kUnroll = 4;                    // points in flight per thread (hist / place)
+constexpr int kChunkPoints = 16384;           // points of a segment per hist / place block
+constexpr int kHistCells = 48 * 1024;         // shared counters per band (192 KB)
+constexpr int kScanItems = 8;                 // per thread
+constexpr int kScanTile = kThreads * kScanItems;
+constexpr int kRunRecords = 64;               // records per sub-warp in the cell pass
+constexpr int kCellChannels = 4;              // channels per lane in the cell pass
 
-// Cells of level l occupy [base[l], base[l] + count[l]) inside the segment of
-// one (b, m), count[l] = (H_l + 1)(W_l + 1); cell (x0, y0), x0 in [-1, W-1],
-// y0 in [-1, H-1], is at (y0 + 1)(W + 1) + (x0 + 1).  With consistent metadata
-// the levels fill at most 2 S + 2 L cells, the segment length; a level that would
-// reach past the segment (possible only when levels overlap in `value`) gets
-// count 0, so its points are never binned and no cell index leaves the array.
+// Cells of level l occupy [base[l], base[l] + count[l]) of a (b, m) block of
+// keys, count[l] = (H_l + 1)(W_l + 1).  With consistent metadata the levels fill
+// at most 2 S + 2 L keys (the block length); a level that would reach past it
+// (possible only when levels overlap in `value`) gets count 0, so its points
+// are never binned and no key leaves the array.
 struct CellLevels {
   int base[kMaxLevels];
   int count[kMaxLevels];
@@ -69,55 +91,121 @@ __device__ __forceinline__ void stage_cells(CellLevels& cl, const Levels& lv, in
   __syncthreads();
 }
 
-struct PointIndex {
-  long long bq;
-  int m, l;
+// Exact floor(n / d) for 0 <= n < 2^31 and 1 <= d < 2^31 with one 64-bit
+// multiply: magic = ceil(2^(32+s) / d), s = ceil(log2 d).  The rounding error of
+// magic adds less than n / 2^(32+s) < 1 / (2d) to n / d, which never carries past
+// the next integer.
+struct FastDiv {
+  unsigned long long magic;
+  int shift;
 };
 
-__device__ __forceinline__ PointIndex split_point(long long p, int LK, int K, int M) {
-  PointIndex r;
-  const long long bqm = p / LK;
-  r.l = static_cast<int>(p - bqm * LK) / K;
-  r.m = static_cast<int>(bqm % M);
-  r.bq = bqm / M;
-  return r;
+FastDiv make_fastdiv(long long d) {
+  FastDiv f;
+  int s = 0;
+  while ((1ll << s) < d) ++s;
+  f.shift = 32 + s;
+  f.magic = ((1ull << f.shift) + static_cast<unsigned long long>(d) - 1) /
+            static_cast<unsigned long long>(d);
+  return f;
+}
+
+__device__ __forceinline__ int fast_div(int n, const FastDiv& f) {
+  return static_cast<int>((static_cast<unsigned long long>(n) * f.magic) >> f.shift);
+}
+
+// Segment seg = (b * M + m) * L + l; its point i = q * K + k is sampling point
+// p = ((b * Lq + q) * M + m) * L * K + l * K + k.
+struct Segment {
+  long long b;
+  int m, l;
+  long long p_base;  // p of point 0
+  long long p_q;     // p stride between queries: M * L * K
+};
+
+__device__ __forceinline__ Segment segment_of(long long seg, int M, int L, int K, long long Lq) {
+  Segment s;
+  s.l = static_cast<int>(seg % L);
+  const long long bm = seg / L;
+  s.m = static_cast<int>(bm % M);
+  s.b = bm / M;
+  s.p_q = static_cast<long long>(M) * L * K;
+  s.p_base = (s.b * Lq * M + s.m) * static_cast<long long>(L) * K + static_cast<long long>(s.l) * K;
+  return s;
+}
+
+// The cell of one point, or -1 when none of its corners is in the map.
+__device__ __forceinline__ int point_cell(const Cell& c, int W) {
+  return ((c.vx0 || c.vx1) && (c.vy0 || c.vy1)) ? (c.y0 + 1) * (W + 1) + (c.x0 + 1) : -1;
 }
 
 __global__ void __launch_bounds__(kThreads)
-bin_kernel(const int64_t* __restrict__ spatial_shapes, const int64_t* __restrict__ level_start,
-           const float* __restrict__ sampling_locations,
-           const float* __restrict__ attention_weights, float* __restrict__ grad_loc,
-           float* __restrict__ grad_attn, int* __restrict__ counts, int2* __restrict__ bin_slot,
-           long long S, int M, long long Lq, int L, int K, long long cells_per_bm,
-           long long points) {
+hist_kernel(const int64_t* __restrict__ spatial_shapes, const int64_t* __restrict__ level_start,
+            const float* __restrict__ sampling_locations,
+            const float* __restrict__ attention_weights, float* __restrict__ grad_loc,
+            float* __restrict__ grad_attn, int* __restrict__ counts, int* __restrict__ slots,
+            long long S, int M, long long Lq, int L, int K, long long cells_per_bm,
+            int chunks) {
+  extern __shared__ int hist[];
   __shared__ Levels lv;
   __shared__ CellLevels cl;
   stage_levels(lv, spatial_shapes, level_start, L, S);
   stage_cells(cl, lv, L, cells_per_bm);
-  const int LK = L * K;
-  for (long long p = blockIdx.x * static_cast<long long>(kThreads) + threadIdx.x; p < points;
-       p += static_cast<long long>(gridDim.x) * kThreads) {
-    const PointIndex pi = split_point(p, LK, K, M);
-    const int H = lv.H[pi.l], W = lv.W[pi.l];
-    const float2 xy = __ldg(reinterpret_cast<const float2*>(sampling_locations) + p);
-    const Cell c = locate(xy.x, xy.y, H, W);
-    if ((c.vx0 || c.vx1) && (c.vy0 || c.vy1) && cl.count[pi.l] > 0) {
-      const long long b = pi.bq / Lq;
-      const long long bin = (b * M + pi.m) * cells_per_bm + cl.base[pi.l] +
-                            static_cast<long long>(c.y0 + 1) * (W + 1) + (c.x0 + 1);
-      const int slot = atomicAdd(counts + bin, 1);
-      bin_slot[p] = make_int2(static_cast<int>(bin), slot);
-    } else {
-      // No corner in the map: every corner dot product is 0.  The products with
-      // the weights keep the NaN of a non-finite location, as the oracle does.
-      bin_slot[p] = make_int2(-1, 0);
-      const float a = __ldg(attention_weights + p);
-      grad_attn[p] = 0.0f * (c.fx + c.fy);
-      reinterpret_cast<float2*>(grad_loc)[p] =
-          make_float2(a * static_cast<float>(W) * (0.0f * c.fy),
-                      a * static_cast<float>(H) * (0.0f * c.fx));
+  const long long seg = blockIdx.x / chunks;
+  const int chunk = static_cast<int>(blockIdx.x - seg * chunks);
+  const Segment sg = segment_of(seg, M, L, K, Lq);
+  const int H = lv.H[sg.l], W = lv.W[sg.l];
+  const int ncells = cl.count[sg.l];
+  const long long seg_len = Lq * K;
+  const long long i_begin = static_cast<long long>(chunk) * kChunkPoints;
+  const long long i_end = min(seg_len, i_begin + kChunkPoints);
+  // counts index of (cell, chunk): key * chunks + chunk.
+  const long long key0 = (sg.b * M + sg.m) * cells_per_bm + cl.base[sg.l];
+
+  int lo = 0;
+  do {
+    const int span = min(kHistCells, ncells - lo);
+    for (int c = threadIdx.x; c < span; c += kThreads) hist[c] = 0;
+    __syncthreads();
+    for (long long i0 = i_begin + threadIdx.x; i0 < i_end; i0 += kThreads * kUnroll) {
+      float2 xy[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const long long i = i0 + u * kThreads;
+        if (i < i_end) {
+          const long long q = i / K;
+          xy[u] = __ldg(reinterpret_cast<const float2*>(sampling_locations) + sg.p_base +
+                        q * sg.p_q + (i - q * K));
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const long long i = i0 + u * kThreads;
+        if (i >= i_end) continue;
+        const long long q = i / K;
+        const long long p = sg.p_base + q * sg.p_q + (i - q * K);
+        const Cell c = locate(xy[u].x, xy[u].y, H, W);
+        const int cell = ncells > 0 ? point_cell(c, W) : -1;
+        if (cell >= lo && cell < lo + span) {
+          slots[p] = atomicAdd(hist + (cell - lo), 1);
+        } else if (cell < 0 && lo == 0) {
+          // No corner in the map: every corner dot product is 0.  The products
+          // with the weights keep the NaN of a non-finite location, as the
+          // oracle does.
+          const float a = __ldg(attention_weights + p);
+          grad_attn[p] = 0.0f * (c.fx + c.fy);
+          reinterpret_cast<float2*>(grad_loc)[p] =
+              make_float2(a * static_cast<float>(W) * (0.0f * c.fy),
+                          a * static_cast<float>(H) * (0.0f * c.fx));
+        }
+      }
     }
-  }
+    __syncthreads();
+    for (int c = threadIdx.x; c < span; c += kThreads)
+      counts[(key0 + lo + c) * chunks + chunk] = hist[c];
+    lo += kHistCells;
+    __syncthreads();
+  } while (lo < ncells);
 }
 
 // Exclusive scan, pass 1: each block scans its tile in place and records the
@@ -134,7 +222,6 @@ scan_tiles_kernel(int* __restrict__ data, int* __restrict__ tile_sums, long long
     v[i] = (base + i < n) ? data[base + i] : 0;
     total += v[i];
   }
-  // Block-wide exclusive scan of the per-thread totals.
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int incl = total;
 #pragma unroll
@@ -212,163 +299,301 @@ __global__ void __launch_bounds__(kThreads)
 place_kernel(const int64_t* __restrict__ spatial_shapes, const int64_t* __restrict__ level_start,
              const float* __restrict__ sampling_locations,
              const float* __restrict__ attention_weights, const int* __restrict__ offsets,
-             const int2* __restrict__ bin_slot, float4* __restrict__ records, long long S,
-             int M, int L, int K, long long points) {
-  __shared__ Levels lv;
-  stage_levels(lv, spatial_shapes, level_start, L, S);
-  const int LK = L * K;
-  for (long long p = blockIdx.x * static_cast<long long>(kThreads) + threadIdx.x; p < points;
-       p += static_cast<long long>(gridDim.x) * kThreads) {
-    const int2 bs = bin_slot[p];
-    if (bs.x < 0) continue;
-    const int l = static_cast<int>(p % LK) / K;
-    const float2 xy = __ldg(reinterpret_cast<const float2*>(sampling_locations) + p);
-    const Cell c = locate(xy.x, xy.y, lv.H[l], lv.W[l]);
-    const float a = __ldg(attention_weights + p);
-    records[offsets[bs.x] + bs.y] =
-        make_float4(__int_as_float(static_cast<int>(p)), a, c.fx, c.fy);
-  }
-}
-
-__device__ __forceinline__ float dot4(const float4& a, const float4& b) {
-  return fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, a.w * b.w)));
-}
-
-__device__ __forceinline__ void axpy4(float w, const float4& x, float4& y) {
-  y.x = fmaf(w, x.x, y.x);
-  y.y = fmaf(w, x.y, y.y);
-  y.z = fmaf(w, x.z, y.z);
-  y.w = fmaf(w, x.w, y.w);
-}
-
-// Cell pass.  LANES lanes per cell, 4 channels per lane (D <= 4 * LANES); NB =
-// min(LANES, 8) points per batch.
-template <int LANES>
-__global__ void __launch_bounds__(kThreads)
-cell_kernel(const float* __restrict__ value, const int64_t* __restrict__ spatial_shapes,
-            const int64_t* __restrict__ level_start, const float* __restrict__ grad_output,
-            const int* __restrict__ offsets, const float4* __restrict__ records,
-            float* __restrict__ grad_value, float* __restrict__ grad_loc,
-            float* __restrict__ grad_attn, long long S, int M, int D, long long Lq, int L,
-            int K, long long cells_per_bm, long long bins) {
-  constexpr int NB = LANES < 8 ? LANES : 8;
+             const int* __restrict__ slots, float4* __restrict__ records,
+             int* __restrict__ record_keys, long long S, int M, long long Lq, int L, int K,
+             long long cells_per_bm, int chunks) {
   __shared__ Levels lv;
   __shared__ CellLevels cl;
   stage_levels(lv, spatial_shapes, level_start, L, S);
   stage_cells(cl, lv, L, cells_per_bm);
-  const int lane = threadIdx.x % LANES;
-  const int per_block = kThreads / LANES;
-  const int LK = L * K;
-  const int MD = M * D;
-  const int ch = lane * 4;
-  // Sub-warps work on different cells with different point counts, so their
-  // shuffles name only their own lanes.
-  const unsigned sub_mask =
-      LANES == 32 ? kFullMask
-                  : ((1u << (LANES & 31)) - 1u) << ((threadIdx.x & 31) & ~(LANES - 1));
-
-  for (long long bin0 = blockIdx.x * static_cast<long long>(per_block); bin0 < bins;
-       bin0 += static_cast<long long>(gridDim.x) * per_block) {
-    const long long bin = bin0 + threadIdx.x / LANES;
-    // Every lane of a sub-warp sees the same bin, so the sub-warp stays converged.
-    const int begin = bin < bins ? offsets[bin] : 0;
-    const int end = bin < bins ? offsets[bin + 1] : 0;
-    if (begin >= end) continue;
-    const long long seg = bin / cells_per_bm;
-    const int within = static_cast<int>(bin - seg * cells_per_bm);
-    const int m = static_cast<int>(seg % M);
-    const long long b = seg / M;
-    // The level whose cell range holds this (non-empty) bin.
-    int l = 0;
-    while (l + 1 < L && !(within >= cl.base[l] && within < cl.base[l] + cl.count[l])) ++l;
-    const int H = lv.H[l], W = lv.W[l];
-    const int cell = within - cl.base[l];
-    const int y0 = cell / (W + 1) - 1, x0 = cell % (W + 1) - 1;
-    const bool vx0 = x0 >= 0, vx1 = x0 + 1 < W, vy0 = y0 >= 0, vy1 = y0 + 1 < H;
-    const bool lane_on = ch < D;
-    const long long vofs = (b * S * M + m) * static_cast<long long>(D) + ch;
-    const long long pix = lv.start[l] + static_cast<long long>(y0) * W + x0;
-    // Corner rows of this cell: c00 = V(x0, y0), c10 = V(x0+1, y0), c01 = V(x0, y0+1), ...
-    const float4 zero = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-    float4 c00 = zero, c10 = zero, c01 = zero, c11 = zero;
-    if (lane_on) {
-      if (vx0 && vy0) c00 = __ldg(reinterpret_cast<const float4*>(value + vofs + pix * MD));
-      if (vx1 && vy0) c10 = __ldg(reinterpret_cast<const float4*>(value + vofs + (pix + 1) * MD));
-      if (vx0 && vy1) c01 = __ldg(reinterpret_cast<const float4*>(value + vofs + (pix + W) * MD));
-      if (vx1 && vy1)
-        c11 = __ldg(reinterpret_cast<const float4*>(value + vofs + (pix + W + 1) * MD));
-    }
-    float4 a00 = zero, a10 = zero, a01 = zero, a11 = zero;  // grad_value accumulators
-
-    for (int i0 = begin; i0 < end; i0 += NB) {
-      // Lane j < NB holds record i0 + j.
-      float4 rec = make_float4(__int_as_float(-1), 0.0f, 0.0f, 0.0f);
-      if (lane < NB && i0 + lane < end) rec = records[i0 + lane];
-      float part[4][NB];
+  const long long seg = blockIdx.x / chunks;
+  const int chunk = static_cast<int>(blockIdx.x - seg * chunks);
+  const Segment sg = segment_of(seg, M, L, K, Lq);
+  const int H = lv.H[sg.l], W = lv.W[sg.l];
+  const int ncells = cl.count[sg.l];
+  if (ncells == 0) return;
+  const long long seg_len = Lq * K;
+  const long long i_begin = static_cast<long long>(chunk) * kChunkPoints;
+  const long long i_end = min(seg_len, i_begin + kChunkPoints);
+  const long long key0 = (sg.b * M + sg.m) * cells_per_bm + cl.base[sg.l];
+  for (long long i0 = i_begin + threadIdx.x; i0 < i_end; i0 += kThreads * kUnroll) {
+    float2 xy[kUnroll];
+    float a[kUnroll];
 #pragma unroll
-      for (int j = 0; j < NB; ++j) {
-        const int p = __float_as_int(__shfl_sync(sub_mask, rec.x, j, LANES));
-        const float a = __shfl_sync(sub_mask, rec.y, j, LANES);
-        const float fx = __shfl_sync(sub_mask, rec.z, j, LANES);
-        const float fy = __shfl_sync(sub_mask, rec.w, j, LANES);
-        float4 go = zero;
-        if (p >= 0 && lane_on) {
-          const long long bq = static_cast<long long>(p) / (static_cast<long long>(M) * LK);
-          go = __ldg(reinterpret_cast<const float4*>(grad_output + bq * MD +
-                                                     static_cast<long long>(m) * D + ch));
-        }
-        part[0][j] = dot4(go, c00);
-        part[1][j] = dot4(go, c10);
-        part[2][j] = dot4(go, c01);
-        part[3][j] = dot4(go, c11);
-        const float hx = 1.0f - fx, hy = 1.0f - fy;
-        axpy4(a * hx * hy, go, a00);
-        axpy4(a * fx * hy, go, a10);
-        axpy4(a * hx * fy, go, a01);
-        axpy4(a * fx * fy, go, a11);
-      }
-      // Full butterfly over the lane bits above the batch, then a reduce-scatter
-      // so that lane j (< NB) ends with the totals of point j.
-#pragma unroll
-      for (int o = LANES / 2; o >= NB; o >>= 1) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-#pragma unroll
-          for (int j = 0; j < NB; ++j) part[q][j] += __shfl_xor_sync(sub_mask, part[q][j], o, LANES);
-      }
-#pragma unroll
-      for (int o = NB / 2; o >= 1; o >>= 1) {
-        const bool upper = (lane & o) != 0;
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-#pragma unroll
-          for (int j = 0; j < o; ++j) {
-            // Keep indices with bit o equal to this lane's bit; send the others.
-            const float send = upper ? part[q][j] : part[q][j + o];
-            const float keep = upper ? part[q][j + o] : part[q][j];
-            part[q][j] = keep + __shfl_xor_sync(sub_mask, send, o, LANES);
-          }
-      }
-      // part[q][0] now holds the totals of point `lane` (for lane < NB).
-      const int p = __float_as_int(rec.x);
-      if (lane < NB && p >= 0) {
-        const float a = rec.y, fx = rec.z, fy = rec.w;
-        const float hx = 1.0f - fx, hy = 1.0f - fy;
-        const float g00 = part[0][0], g10 = part[1][0], g01 = part[2][0], g11 = part[3][0];
-        grad_attn[p] = fmaf(hy, fmaf(fx, g10, hx * g00), fy * fmaf(fx, g11, hx * g01));
-        reinterpret_cast<float2*>(grad_loc)[p] = make_float2(
-            a * static_cast<float>(W) * fmaf(hy, g10 - g00, fy * (g11 - g01)),
-            a * static_cast<float>(H) * fmaf(hx, g01 - g00, fx * (g11 - g10)));
+    for (int u = 0; u < kUnroll; ++u) {
+      const long long i = i0 + u * kThreads;
+      if (i < i_end) {
+        const long long q = i / K;
+        const long long p = sg.p_base + q * sg.p_q + (i - q * K);
+        xy[u] = __ldg(reinterpret_cast<const float2*>(sampling_locations) + p);
+        a[u] = __ldg(attention_weights + p);
       }
     }
-    if (lane_on) {
-      float* gv = grad_value + vofs;
-      if (vx0 && vy0) atomicAdd(reinterpret_cast<float4*>(gv + pix * MD), a00);
-      if (vx1 && vy0) atomicAdd(reinterpret_cast<float4*>(gv + (pix + 1) * MD), a10);
-      if (vx0 && vy1) atomicAdd(reinterpret_cast<float4*>(gv + (pix + W) * MD), a01);
-      if (vx1 && vy1) atomicAdd(reinterpret_cast<float4*>(gv + (pix + W + 1) * MD), a11);
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const long long i = i0 + u * kThreads;
+      if (i >= i_end) continue;
+      const long long q = i / K;
+      const long long p = sg.p_base + q * sg.p_q + (i - q * K);
+      const Cell c = locate(xy[u].x, xy[u].y, H, W);
+      const int cell = point_cell(c, W);
+      if (cell < 0) continue;
+      const long long key = key0 + cell;
+      const int pos = offsets[key * chunks + chunk] + slots[p];
+      records[pos] = make_float4(__int_as_float(static_cast<int>(p)), a[u], c.fx, c.fy);
+      record_keys[pos] = static_cast<int>(key);
     }
   }
+}
+
+// A lane's CPL consecutive channels of one row (CPL = 4 or 8), moved as float4s;
+// `on[h]` tells whether float4 h of the lane lies inside the D channels.
+template <int CPL>
+struct Row {
+  float v[CPL];
+};
+
+template <int CPL>
+__device__ __forceinline__ Row<CPL> zero_row() {
+  Row<CPL> r;
+#pragma unroll
+  for (int i = 0; i < CPL; ++i) r.v[i] = 0.0f;
+  return r;
+}
+
+template <int CPL>
+__device__ __forceinline__ Row<CPL> load_row(const float* p, const bool (&on)[CPL / 4]) {
+  Row<CPL> r = zero_row<CPL>();
+#pragma unroll
+  for (int h = 0; h < CPL / 4; ++h)
+    if (on[h]) {
+      const float4 x = __ldg(reinterpret_cast<const float4*>(p + 4 * h));
+      r.v[4 * h + 0] = x.x;
+      r.v[4 * h + 1] = x.y;
+      r.v[4 * h + 2] = x.z;
+      r.v[4 * h + 3] = x.w;
+    }
+  return r;
+}
+
+template <int CPL>
+__device__ __forceinline__ void red_row(float* p, const Row<CPL>& r, const bool (&on)[CPL / 4]) {
+#pragma unroll
+  for (int h = 0; h < CPL / 4; ++h)
+    if (on[h])
+      atomicAdd(reinterpret_cast<float4*>(p + 4 * h),
+                make_float4(r.v[4 * h], r.v[4 * h + 1], r.v[4 * h + 2], r.v[4 * h + 3]));
+}
+
+template <int CPL>
+__device__ __forceinline__ float dot_row(const Row<CPL>& a, const Row<CPL>& b) {
+  float s = a.v[0] * b.v[0];
+#pragma unroll
+  for (int i = 1; i < CPL; ++i) s = fmaf(a.v[i], b.v[i], s);
+  return s;
+}
+
+template <int CPL>
+__device__ __forceinline__ void axpy_row(float w, const Row<CPL>& x, Row<CPL>& y) {
+#pragma unroll
+  for (int i = 0; i < CPL; ++i) y.v[i] = fmaf(w, x.v[i], y.v[i]);
+}
+
+// The geometry of the cell behind a key, with this lane's value / grad_value
+// row offset of pixel (x0, y0) and the element strides to its neighbours.
+struct CellGeom {
+  int m, W, H, x0;
+  bool vx0, vx1, vy0, vy1;
+  long long ofs;  // ((b * S + start + y0 * W + x0) * M + m) * D + ch
+  long long dy;   // W * M * D
+};
+
+__device__ __forceinline__ CellGeom decode_key(int key, long long cells_per_bm, int M, int L,
+                                               long long S, int D, int ch, const Levels& lv,
+                                               const CellLevels& cl) {
+  CellGeom g;
+  const long long bm = key / cells_per_bm;
+  const int within = static_cast<int>(key - bm * cells_per_bm);
+  g.m = static_cast<int>(bm % M);
+  const long long b = bm / M;
+  int l = 0;
+  while (l + 1 < L && !(within >= cl.base[l] && within < cl.base[l] + cl.count[l])) ++l;
+  g.W = lv.W[l];
+  g.H = lv.H[l];
+  const int cell = within - cl.base[l];
+  const int y0 = cell / (g.W + 1) - 1;
+  g.x0 = cell - (y0 + 1) * (g.W + 1) - 1;
+  g.vx0 = g.x0 >= 0;
+  g.vx1 = g.x0 + 1 < g.W;
+  g.vy0 = y0 >= 0;
+  g.vy1 = y0 + 1 < g.H;
+  const long long MD = static_cast<long long>(M) * D;
+  const long long pix = lv.start[l] + static_cast<long long>(y0) * g.W + g.x0;
+  g.ofs = (b * S + pix) * MD + static_cast<long long>(g.m) * D + ch;
+  g.dy = g.W * MD;
+  return g;
+}
+
+// Cell pass.  LANES lanes per sub-warp, CPL channels per lane (D <= CPL * LANES);
+// records are reduced NB = min(LANES, 4) at a time.
+template <int LANES, int CPL>
+__global__ void __launch_bounds__(kThreads)
+cell_kernel(const float* __restrict__ value, const int64_t* __restrict__ spatial_shapes,
+            const int64_t* __restrict__ level_start, const float* __restrict__ grad_output,
+            const int* __restrict__ total_records, const float4* __restrict__ records,
+            const int* __restrict__ record_keys, float* __restrict__ grad_value,
+            float* __restrict__ grad_loc, float* __restrict__ grad_attn, long long S, int M,
+            int D, int L, long long cells_per_bm, FastDiv per_bq) {
+  constexpr int NB = LANES < 4 ? LANES : 4;
+  using R = Row<CPL>;
+  __shared__ Levels lv;
+  __shared__ CellLevels cl;
+  stage_levels(lv, spatial_shapes, level_start, L, S);
+  stage_cells(cl, lv, L, cells_per_bm);
+
+  const int lane = threadIdx.x % LANES;
+  // Sub-warps follow their own runs, so their shuffles name only their lanes.
+  const unsigned mask =
+      LANES == 32 ? kFullMask
+                  : ((1u << (LANES & 31)) - 1u) << ((threadIdx.x & 31) & ~(LANES - 1));
+  const long long run = (blockIdx.x * static_cast<long long>(kThreads) + threadIdx.x) / LANES;
+  const int total = *total_records;
+  if (run * kRunRecords >= total) return;
+  const int r0 = static_cast<int>(run * kRunRecords);
+  const int r1 = min(r0 + kRunRecords, total);
+  const int ch = lane * CPL;
+  bool on[CPL / 4];
+#pragma unroll
+  for (int h = 0; h < CPL / 4; ++h) on[h] = ch + 4 * h < D;
+  const long long MD = static_cast<long long>(M) * D;
+
+  // The current cell (key cur): corner rows cIJ = V(x0 + I, y0 + J) of value and
+  // the grad_value accumulators aIJ of the same corners.
+  int cur = -1;
+  CellGeom g{};
+  R c00 = zero_row<CPL>(), c10 = zero_row<CPL>(), c01 = zero_row<CPL>(), c11 = zero_row<CPL>();
+  R a00 = zero_row<CPL>(), a10 = zero_row<CPL>(), a01 = zero_row<CPL>(), a11 = zero_row<CPL>();
+  auto flush = [&](bool keep_right) {
+    float* gv = grad_value + g.ofs;
+    if (g.vx0 && g.vy0) red_row(gv, a00, on);
+    if (g.vx0 && g.vy1) red_row(gv + g.dy, a01, on);
+    if (!keep_right) {
+      if (g.vx1 && g.vy0) red_row(gv + MD, a10, on);
+      if (g.vx1 && g.vy1) red_row(gv + g.dy + MD, a11, on);
+    }
+  };
+  auto enter = [&](int key) {
+    const CellGeom ng = decode_key(key, cells_per_bm, M, L, S, D, ch, lv, cl);
+    // Moving right along a row keeps the shared column: values and sums.
+    const bool right = cur >= 0 && key == cur + 1 && ng.x0 >= 0;
+    if (cur >= 0) flush(right);
+    if (right) {
+      c00 = c10;
+      c01 = c11;
+      a00 = a10;
+      a01 = a11;
+    } else {
+      c00 = (ng.vx0 && ng.vy0) ? load_row<CPL>(value + ng.ofs, on) : zero_row<CPL>();
+      c01 = (ng.vx0 && ng.vy1) ? load_row<CPL>(value + ng.ofs + ng.dy, on) : zero_row<CPL>();
+      a00 = zero_row<CPL>();
+      a01 = zero_row<CPL>();
+    }
+    c10 = (ng.vx1 && ng.vy0) ? load_row<CPL>(value + ng.ofs + MD, on) : zero_row<CPL>();
+    c11 = (ng.vx1 && ng.vy1) ? load_row<CPL>(value + ng.ofs + ng.dy + MD, on) : zero_row<CPL>();
+    a10 = zero_row<CPL>();
+    a11 = zero_row<CPL>();
+    // Records come in row order: the next cell is most often the right
+    // neighbour, whose new column is prefetched into L1 now.
+    if (ng.x0 + 2 < ng.W && on[0]) {
+      const float* nx = value + ng.ofs + 2 * MD;
+      if (ng.vy0) asm volatile("prefetch.global.L1 [%0];" ::"l"(nx));
+      if (ng.vy1) asm volatile("prefetch.global.L1 [%0];" ::"l"(nx + ng.dy));
+    }
+    g = ng;
+    cur = key;
+  };
+
+  for (int i0 = r0; i0 < r1; i0 += NB) {
+    // Lane j (< NB) holds record i0 + j.
+    float4 rec = make_float4(__int_as_float(-1), 0.0f, 0.0f, 0.0f);
+    int rkey = -1;
+    if (lane < NB && i0 + lane < r1) {
+      rec = records[i0 + lane];
+      rkey = record_keys[i0 + lane];
+    }
+    // The batch's grad_output rows first, so that their loads overlap.
+    int keys[NB];
+    R go[NB];
+#pragma unroll
+    for (int j = 0; j < NB; ++j) {
+      keys[j] = __shfl_sync(mask, rkey, j, LANES);
+      const int p = __float_as_int(__shfl_sync(mask, rec.x, j, LANES));
+      go[j] = zero_row<CPL>();
+      if (keys[j] >= 0) {
+        const int bq = fast_div(p, per_bq);
+        const int m = static_cast<int>((keys[j] / cells_per_bm) % M);
+        go[j] = load_row<CPL>(grad_output + static_cast<long long>(bq) * MD +
+                                  static_cast<long long>(m) * D + ch,
+                              on);
+      }
+    }
+    float part[4][NB];
+    float myW = 0.0f, myH = 0.0f;
+#pragma unroll
+    for (int j = 0; j < NB; ++j) {
+      const float a = __shfl_sync(mask, rec.y, j, LANES);
+      const float fx = __shfl_sync(mask, rec.z, j, LANES);
+      const float fy = __shfl_sync(mask, rec.w, j, LANES);
+      part[0][j] = part[1][j] = part[2][j] = part[3][j] = 0.0f;
+      if (keys[j] < 0) continue;  // past the end of the run (uniform in the sub-warp)
+      if (keys[j] != cur) enter(keys[j]);
+      if (lane == j) {
+        myW = static_cast<float>(g.W);
+        myH = static_cast<float>(g.H);
+      }
+      part[0][j] = dot_row(go[j], c00);
+      part[1][j] = dot_row(go[j], c10);
+      part[2][j] = dot_row(go[j], c01);
+      part[3][j] = dot_row(go[j], c11);
+      const float hx = 1.0f - fx, hy = 1.0f - fy;
+      axpy_row(a * hx * hy, go[j], a00);
+      axpy_row(a * fx * hy, go[j], a10);
+      axpy_row(a * hx * fy, go[j], a01);
+      axpy_row(a * fx * fy, go[j], a11);
+    }
+    // Butterfly over the lane bits above the batch, then a reduce-scatter so that
+    // lane j (< NB) ends with the totals of record j.
+#pragma unroll
+    for (int o = LANES / 2; o >= NB; o >>= 1)
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int j = 0; j < NB; ++j) part[q][j] += __shfl_xor_sync(mask, part[q][j], o, LANES);
+#pragma unroll
+    for (int o = NB / 2; o >= 1; o >>= 1) {
+      const bool upper = (lane & o) != 0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int j = 0; j < o; ++j) {
+          // Keep the indices whose bit o matches this lane's; send the others.
+          const float send = upper ? part[q][j] : part[q][j + o];
+          const float keep = upper ? part[q][j + o] : part[q][j];
+          part[q][j] = keep + __shfl_xor_sync(mask, send, o, LANES);
+        }
+    }
+    if (lane < NB && rkey >= 0) {
+      const int p = __float_as_int(rec.x);
+      const float a = rec.y, fx = rec.z, fy = rec.w;
+      const float hx = 1.0f - fx, hy = 1.0f - fy;
+      const float g00 = part[0][0], g10 = part[1][0], g01 = part[2][0], g11 = part[3][0];
+      grad_attn[p] = fmaf(hy, fmaf(fx, g10, hx * g00), fy * fmaf(fx, g11, hx * g01));
+      reinterpret_cast<float2*>(grad_loc)[p] =
+          make_float2(a * myW * fmaf(hy, g10 - g00, fy * (g11 - g01)),
+                      a * myH * fmaf(hx, g01 - g00, fx * (g11 - g10)));
+    }
+  }
+  if (cur >= 0) flush(false);
 }
 
 template <typename T>
@@ -384,13 +609,15 @@ unsigned grid_for(long long items, long long per_block) {
   return static_cast<unsigned>(blocks < 1 ? 1 : blocks);
 }
 
-template <int LANES>
-cudaError_t launch_cells(const BackwardArgs& a, const SortedLayout& w, const int* offsets,
-                         const float4* records, cudaStream_t stream) {
-  cell_kernel<LANES><<<grid_for(w.bins, kThreads / LANES), kThreads, 0, stream>>>(
-      a.value, a.spatial_shapes, a.level_start_index, a.grad_output, offsets, records,
-      a.grad_value, a.grad_sampling_locations, a.grad_attention_weights, a.S, a.M, a.D, a.Lq,
-      a.L, a.K, w.cells_per_bm, w.bins);
+template <int LANES, int CPL>
+cudaError_t launch_cells(const BackwardArgs& a, const SortedLayout& w, const int* total,
+                         const float4* records, const int* record_keys, cudaStream_t stream) {
+  const long long runs = (w.points + kRunRecords - 1) / kRunRecords;
+  const FastDiv per_bq = make_fastdiv(static_cast<long long>(a.M) * a.L * a.K);
+  cell_kernel<LANES, CPL><<<grid_for(runs * LANES, kThreads), kThreads, 0, stream>>>(
+      a.value, a.spatial_shapes, a.level_start_index, a.grad_output, total, records, record_keys,
+      a.grad_value, a.grad_sampling_locations, a.grad_attention_weights, a.S, a.M, a.D, a.L,
+      w.cells_per_bm, per_bq);
   return cudaGetLastError();
 }
 
@@ -400,11 +627,16 @@ SortedLayout sorted_layout(long long B, long long S, long long M, long long Lq, 
   SortedLayout w;
   // sum_l (H_l + 1)(W_l + 1) <= 2 S + 2 L, because H + W <= H W + 1 for H, W >= 1.
   w.cells_per_bm = 2 * S + 2 * L;
-  w.bins = B * M * w.cells_per_bm;
-  w.points = B * Lq * M * L * K;
-  w.scan_tiles = (w.bins + 1 + kScanTile - 1) / kScanTile;
+  w.segments = B * M * L;
+  w.segment_len = Lq * K;
+  w.chunks = (w.segment_len + kChunkPoints - 1) / kChunkPoints;
+  if (w.chunks < 1) w.chunks = 1;
+  w.points = w.segments * w.segment_len;
+  w.counts = B * M * w.cells_per_bm * w.chunks;
+  w.scan_tiles = (w.counts + 1 + kScanTile - 1) / kScanTile;
   auto up = [](long long bytes) { return (bytes + 255) / 256 * 256; };
-  w.bytes = up(4 * (w.bins + 1)) + up(4 * w.scan_tiles) + up(8 * w.points) + up(16 * w.points);
+  w.bytes = up(4 * (w.counts + 1)) + up(4 * w.scan_tiles) + up(4 * w.points) +
+            up(16 * w.points) + up(4 * w.points);
   return w;
 }
 
@@ -412,40 +644,62 @@ cudaError_t launch_backward_sorted(const BackwardArgs& a, void* workspace,
                                    cudaStream_t stream) {
   const SortedLayout w = sorted_layout(a.B, a.S, a.M, a.Lq, a.L, a.K);
   char* cursor = static_cast<char*>(workspace);
-  int* counts = carve<int>(cursor, w.bins + 1);
+  int* counts = carve<int>(cursor, w.counts + 1);
   int* tile_sums = carve<int>(cursor, w.scan_tiles);
-  int2* bin_slot = carve<int2>(cursor, w.points);
+  int* slots = carve<int>(cursor, w.points);
   float4* records = carve<float4>(cursor, w.points);
+  int* record_keys = carve<int>(cursor, w.points);
 
   cudaError_t err = launch_zero(a.grad_value, a.value_elements, stream);
-  if (err != cudaSuccess) return err;
-  err = launch_zero_words(counts, w.bins + 1, stream);
   if (err != cudaSuccess || w.points == 0) return err;
+  // Counts of cells that no block writes (keys past a segment's levels) stay 0;
+  // the zero fill covers whole float4s, which the 256-byte carve leaves room for.
+  if ((err = launch_zero(reinterpret_cast<float*>(counts), (w.counts + 1 + 3) / 4 * 4,
+                         stream)) != cudaSuccess)
+    return err;
 
-  bin_kernel<<<grid_for(w.points, kThreads), kThreads, 0, stream>>>(
+  // The hist kernel's counters exceed the default 48 KB of dynamic shared
+  // memory; the opt-in is set once per device.
+  const size_t hist_smem = sizeof(int) * static_cast<size_t>(kHistCells);
+  static bool smem_set[64] = {};
+  int dev = 0;
+  if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
+  if (dev < 0 || dev >= 64 || !smem_set[dev]) {
+    err = cudaFuncSetAttribute(hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(hist_smem));
+    if (err != cudaSuccess) return err;
+    if (dev >= 0 && dev < 64) smem_set[dev] = true;
+  }
+  const unsigned blocks = static_cast<unsigned>(w.segments * w.chunks);
+  const int chunks = static_cast<int>(w.chunks);
+  hist_kernel<<<blocks, kThreads, hist_smem, stream>>>(
       a.spatial_shapes, a.level_start_index, a.sampling_locations, a.attention_weights,
-      a.grad_sampling_locations, a.grad_attention_weights, counts, bin_slot, a.S, a.M, a.Lq,
-      a.L, a.K, w.cells_per_bm, w.points);
+      a.grad_sampling_locations, a.grad_attention_weights, counts, slots, a.S, a.M, a.Lq, a.L,
+      a.K, w.cells_per_bm, chunks);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   scan_tiles_kernel<<<static_cast<unsigned>(w.scan_tiles), kThreads, 0, stream>>>(
-      counts, tile_sums, w.bins + 1);
+      counts, tile_sums, w.counts + 1);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   scan_sums_kernel<<<1, 1024, 0, stream>>>(tile_sums, static_cast<int>(w.scan_tiles));
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   scan_add_kernel<<<static_cast<unsigned>(w.scan_tiles), kThreads, 0, stream>>>(
-      counts, tile_sums, w.bins + 1);
+      counts, tile_sums, w.counts + 1);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  place_kernel<<<grid_for(w.points, kThreads), kThreads, 0, stream>>>(
+  place_kernel<<<blocks, kThreads, 0, stream>>>(
       a.spatial_shapes, a.level_start_index, a.sampling_locations, a.attention_weights, counts,
-      bin_slot, records, a.S, a.M, a.L, a.K, w.points);
+      slots, records, record_keys, a.S, a.M, a.Lq, a.L, a.K, w.cells_per_bm, chunks);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  switch (a.lanes) {
-    case 1: return launch_cells<1>(a, w, counts, records, stream);
-    case 2: return launch_cells<2>(a, w, counts, records, stream);
-    case 4: return launch_cells<4>(a, w, counts, records, stream);
-    case 8: return launch_cells<8>(a, w, counts, records, stream);
-    case 16: return launch_cells<16>(a, w, counts, records, stream);
-    case 32: return launch_cells<32>(a, w, counts, records, stream);
+  // counts[w.counts] now holds the number of records.
+  const int* total = counts + w.counts;
+  int lanes = 1;
+  while (lanes * kCellChannels < a.D) lanes <<= 1;
+  switch (lanes) {
+    case 1: return launch_cells<1, kCellChannels>(a, w, total, records, record_keys, stream);
+    case 2: return launch_cells<2, kCellChannels>(a, w, total, records, record_keys, stream);
+    case 4: return launch_cells<4, kCellChannels>(a, w, total, records, record_keys, stream);
+    case 8: return launch_cells<8, kCellChannels>(a, w, total, records, record_keys, stream);
+    case 16: return launch_cells<16, kCellChannels>(a, w, total, records, record_keys, stream);
+    case 32: return launch_cells<32, kCellChannels>(a, w, total, records, record_keys, stream);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -22,10 +22,15 @@
 //            read-only loads and accumulates in float32 with packed two-wide
 //            FMAs.
 // The per-point index arithmetic is thus done once per point instead of once
-// per lane.  Consecutive groups are consecutive heads of consecutive queries and
-// a block owns one tile, so the blocks resident at a time work on neighbouring
-// queries, whose samples overlap in L2.  (Head-major tiles and per-block tile
-// ranges, which favour L1 reuse, measured slower on the encoder workload.)
+// per lane.  The grid holds as many blocks as are resident at once; block i
+// takes tiles i, i + grid, i + 2 grid, ..., so at any moment the blocks work on
+// one window of neighbouring queries (consecutive groups are consecutive heads
+// of consecutive queries), whose samples overlap in L2.  The setup table is
+// double-buffered: the locations and weights of a block's next unit (chunk of a
+// tile) are loaded before the current unit's gathers and turned into setups
+// after them, so their HBM latency hides behind the gathers and one barrier
+// per unit suffices.  (Head-major tiles and contiguous per-block tile ranges,
+// which favour L1 reuse, measured slower on the encoder workload.)
 #include "msda_device.cuh"
 #include "msda_launch.h"
 
@@ -134,79 +139,132 @@ forward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial_
                long long groups) {
   using C = Corner<T>;
   constexpr int E = C::N;
-  constexpr int G = kThreads / LANES;   // groups per block
-  constexpr int PC = kChunkPoints / G;  // points per group per chunk (= 2 * LANES)
+  constexpr int G = kThreads / LANES;
+  constexpr int PC = kChunkPoints / G;
+  constexpr int PER = kChunkPoints / kThreads;  // points set up per thread
   static_assert(G >= 8, "the shared-memory swizzle needs at least 8 groups per block");
   __shared__ Levels lv;
-  __shared__ int4 s_off[kChunkPoints];
-  __shared__ float4 s_w[kChunkPoints];
+  __shared__ int4 s_off[2][kChunkPoints];
+  __shared__ float4 s_w[2][kChunkPoints];
   stage_levels(lv, spatial_shapes, level_start_index, L, S);
 
   const int lane = threadIdx.x % LANES;
   const int gi = threadIdx.x / LANES;
   const int LK = L * K;
   const int MD = M * D;
+  const long long tiles = (groups + G - 1) / G;
+  long long tile = blockIdx.x;
+  if (tile >= tiles) return;
+  int p0 = 0;
 
-  for (long long g0 = static_cast<long long>(blockIdx.x) * G; g0 < groups;
-       g0 += static_cast<long long>(gridDim.x) * G) {
-    const long long g_raw = g0 + gi;
+  // Prefetched inputs of the next unit's points.
+  float2 pxy[PER];
+  float pa[PER];
+  auto prefetch = [&](long long t_, int q0) {
+    const int pc = min(PC, LK - q0);
+#pragma unroll
+    for (int r = 0; r < PER; ++r) {
+      const int t = threadIdx.x + r * kThreads;
+      const int tg = t / PC, tj = t % PC;
+      const long long g = t_ * G + tg;
+      if (tj < pc && g < groups) {
+        const long long bqm = g / chunks;
+        pxy[r] = __ldg(reinterpret_cast<const float2*>(sampling_locations) + bqm * LK + q0 + tj);
+        pa[r] = __ldg(attention_weights + bqm * LK + q0 + tj);
+      }
+    }
+  };
+  auto setup = [&](long long t_, int q0, int buf) {
+    const int pc = min(PC, LK - q0);
+#pragma unroll
+    for (int r = 0; r < PER; ++r) {
+      const int t = threadIdx.x + r * kThreads;
+      const int tg = t / PC, tj = t % PC;
+      const long long g = t_ * G + tg;
+      if (tj < pc && g < groups) {
+        const int l = (q0 + tj) / K;
+        const PointSetup su = setup_point(pxy[r].x, pxy[r].y, pa[r], lv.H[l], lv.W[l], lv.start[l], MD);
+        const int slot = tj * G + (tg ^ (tj & 7));
+        s_off[buf][slot] = su.off;
+        s_w[buf][slot] = su.w;
+      }
+    }
+  };
+
+  prefetch(tile, 0);
+  setup(tile, 0, 0);
+  __syncthreads();
+  int buf = 0;
+  float2 acc[E / 2];
+#pragma unroll
+  for (int e = 0; e < E / 2; ++e) acc[e] = make_float2(0.0f, 0.0f);
+  while (true) {
+    // The unit after this one: the next chunk of this tile, or the next tile.
+    long long ntile = tile;
+    int np0 = p0 + PC;
+    if (np0 >= LK) {
+      ntile = tile + gridDim.x;
+      np0 = 0;
+    }
+    const bool more = ntile < tiles;
+    if (more) prefetch(ntile, np0);
+    const long long g_raw = tile * G + gi;
     const bool active = g_raw < groups;
     const Group grp = decompose(active ? g_raw : groups - 1, chunks, M, Lq);
     const int ch = (grp.chunk * LANES + lane) * E;
-    const bool lane_on = active && ch < D;  // clamped tail groups touch no memory
+    const bool lane_on = active && ch < D;
     const T* vbase = value + (grp.b * S * M + grp.m) * static_cast<long long>(D) + ch;
-
-    float2 acc[E / 2];
-#pragma unroll
-    for (int e = 0; e < E / 2; ++e) acc[e] = make_float2(0.0f, 0.0f);
-
-    for (int p0 = 0; p0 < LK; p0 += PC) {
-      const int pc = min(PC, LK - p0);
-      // Phase 1: setups of this chunk's points; thread t takes point tj of group tg.
-#pragma unroll
-      for (int t = threadIdx.x; t < kChunkPoints; t += kThreads) {
-        const int tg = t / PC, tj = t % PC;
-        const long long g = g0 + tg;
-        if (tj < pc && g < groups) {
-          const long long bqm = g / chunks;
-          const int p = p0 + tj;
-          const int l = p / K;
-          const float2 xy = __ldg(reinterpret_cast<const float2*>(sampling_locations) +
-                                  bqm * LK + p);
-          const float a = __ldg(attention_weights + bqm * LK + p);
-          const PointSetup su = setup_point(xy.x, xy.y, a, lv.H[l], lv.W[l], lv.start[l], MD);
-          const int slot = tj * G + (tg ^ (tj & 7));
-          s_off[slot] = su.off;
-          s_w[slot] = su.w;
-        }
-      }
-      __syncthreads();
-      // Phase 2: gather and accumulate.
-      if (lane_on) {
+    const int pc = min(PC, LK - p0);
+    if (lane_on) {
 #pragma unroll 4
-        for (int j = 0; j < pc; ++j) {
-          const int slot = j * G + (gi ^ (j & 7));
-          const int4 o = s_off[slot];
-          const float4 w = s_w[slot];
-          if (o.x >= 0) C::accumulate(vbase + o.x, w.x, acc);
-          if (o.y >= 0) C::accumulate(vbase + o.y, w.y, acc);
-          if (o.z >= 0) C::accumulate(vbase + o.z, w.z, acc);
-          if (o.w >= 0) C::accumulate(vbase + o.w, w.w, acc);
-        }
+      for (int j = 0; j < pc; ++j) {
+        const int slot = j * G + (gi ^ (j & 7));
+        const int4 o = s_off[buf][slot];
+        const float4 w = s_w[buf][slot];
+        if (o.x >= 0) C::accumulate(vbase + o.x, w.x, acc);
+        if (o.y >= 0) C::accumulate(vbase + o.y, w.y, acc);
+        if (o.z >= 0) C::accumulate(vbase + o.z, w.z, acc);
+        if (o.w >= 0) C::accumulate(vbase + o.w, w.w, acc);
       }
-      __syncthreads();
     }
-    if (lane_on) C::store(output + grp.bq * MD + static_cast<long long>(grp.m) * D + ch, acc);
+    if (p0 + PC >= LK) {
+      if (lane_on) C::store(output + grp.bq * MD + static_cast<long long>(grp.m) * D + ch, acc);
+#pragma unroll
+      for (int e = 0; e < E / 2; ++e) acc[e] = make_float2(0.0f, 0.0f);
+    }
+    if (more) setup(ntile, np0, buf ^ 1);
+    __syncthreads();
+    if (!more) break;
+    tile = ntile;
+    p0 = np0;
+    buf ^= 1;
   }
 }
 
-// One block per tile: the block scheduler hands tiles out in order as SMs free
-// up, so the resident blocks always cover a window of neighbouring queries.
+// Blocks of this kernel that are resident on the current device at once
+// (SM count x blocks per SM), cached per device.
+template <typename T, int LANES>
+static long long resident_blocks() {
+  static long long cached[64] = {};
+  int dev = 0, sms = 0, per_sm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev >= 0 && dev < 64 && cached[dev] > 0) return cached[dev];
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, forward_kernel<T, LANES>, kThreads,
+                                                    0) != cudaSuccess ||
+      sms <= 0 || per_sm <= 0)
+    return 148;
+  const long long n = static_cast<long long>(sms) * per_sm;
+  if (dev >= 0 && dev < 64) cached[dev] = n;
+  return n;
+}
+
 template <typename T, int LANES>
 static cudaError_t launch_forward_t(const ForwardArgs& a, cudaStream_t stream) {
   constexpr int G = kThreads / LANES;
-  long long blocks = (a.groups + G - 1) / G;
-  if (blocks > (1ll << 30)) blocks = 1ll << 30;
+  const long long tiles = (a.groups + G - 1) / G;
+  long long blocks = resident_blocks<T, LANES>();
+  if (blocks > tiles) blocks = tiles;
   forward_kernel<T, LANES><<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(
       static_cast<const T*>(a.value), a.spatial_shapes, a.level_start_index,
       a.sampling_locations, a.attention_weights, static_cast<T*>(a.output), a.S, a.M, a.D,

@@ -45,9 +45,12 @@ struct BackwardArgs {
 
 // Scratch layout of the cell-sorted backward (msda_backward_sorted.cu).
 struct SortedLayout {
-  long long cells_per_bm;  // bound on sum_l (H_l + 1)(W_l + 1) from S and L alone
-  long long bins;          // B * M * cells_per_bm
+  long long cells_per_bm;  // keys per (b, m): bound on sum_l (H_l + 1)(W_l + 1) from S, L
+  long long segments;      // B * M * L: one (b, m, level) each
+  long long segment_len;   // Lq * K points per segment
+  long long chunks;        // hist / place blocks per segment
   long long points;        // B * Lq * M * L * K
+  long long counts;        // B * M * cells_per_bm * chunks (cell, chunk) counters
   long long scan_tiles;
   long long bytes;         // workspace bytes
 };
@@ -60,6 +63,5 @@ cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t stream);
 // Backward with the points grouped by cell; `workspace` holds sorted_layout().bytes.
 cudaError_t launch_backward_sorted(const BackwardArgs& a, void* workspace, cudaStream_t stream);
 cudaError_t launch_zero(float* p, long long n, cudaStream_t stream);
-cudaError_t launch_zero_words(int* p, long long n, cudaStream_t stream);
 
 }  // namespace msda

@@ -138,9 +138,10 @@ def test_workspace_size(lib):
     st, need = _ws_size(lib, B=4, S=19947, M=8, D=32, Lq=19947, L=4, K=4)
     assert st == OK
     points = 4 * 19947 * 8 * 16
-    bins = 4 * 8 * (2 * 19947 + 8)
-    assert need >= 24 * points + 4 * (bins + 1)
-    assert need < 24 * points + 4 * (bins + 1) + 64 * 1024
+    chunks = -(-19947 * 4 // 16384)
+    counts = 4 * 8 * (2 * 19947 + 2 * 4) * chunks
+    # slot 4 B + record 16 B + record key 4 B per point; one counter per (cell, chunk).
+    assert 24 * points + 4 * counts <= need < 24 * points + 4 * counts + 64 * 1024
     assert _ws_size(lib, B=-1)[0] == BAD
-    assert _ws_size(lib, B=1 << 20, S=1 << 12, M=8)[0] == UNSUP  # 32-bit cell ids overflow
+    assert _ws_size(lib, B=1 << 14, Lq=1 << 14, M=8)[0] == UNSUP  # 32-bit point ids overflow
     assert lib.msda_backward_workspace_size(1, 80, 2, 8, 80, 2, 2, None) == NULLP
