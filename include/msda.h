@@ -154,6 +154,46 @@ msda_status msda_backward_workspace_size(int64_t B, int64_t S, int64_t M, int64_
                                          size_t *bytes);
 
 /*
+ * Size of the fixed device scratch of msda_backward_noalloc: 32 MiB, held by
+ * every GPU that loads this library until the process exits.
+ */
+#define MSDA_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+
+/*
+ * msda_backward without a workspace argument and without any allocation.  The
+ * pages have no counterpart: this entry point exists for callers that cannot
+ * allocate device memory at the time they call the op -- for instance a host
+ * framework that owns the whole device memory pool and admits no other
+ * allocator, or code on a latency-critical path where cudaMalloc / cudaFree
+ * would block or synchronize the device.
+ *
+ * It computes what msda_backward computes with a workspace (the cell-sorted
+ * path; arguments, layouts, ownership of the tensors and status codes as for
+ * msda_backward), taking the scratch from one array of
+ * MSDA_NOALLOC_SCRATCH_BYTES that the library holds on each device.  It calls
+ * no cudaMalloc, cudaFree or other allocating routine.
+ *   - Sizes whose msda_backward_workspace_size exceeds MSDA_NOALLOC_SCRATCH_BYTES
+ *     are rejected with MSDA_ERR_WORKSPACE before anything is enqueued (for
+ *     example B=1, S=19947, M=8, D=32, L=K=4 fits up to Lq = 9600 queries).
+ *   - The first call on a device looks up the array's device address (set-up,
+ *     once per device, with that device current); make that first call before
+ *     any stream capture.
+ *   - Every call on a device uses the same array, and the array keeps the last
+ *     call's contents; each call clears what it needs at zero.  Calls that
+ *     overlap on the GPU (other streams, other host threads) race on it and must
+ *     be serialized by the caller.
+ */
+msda_status msda_backward_noalloc(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq,
+                                  int64_t L, int64_t K, msda_dtype value_dtype,
+                                  const void *value, const int64_t *spatial_shapes,
+                                  const int64_t *level_start_index,
+                                  const float *sampling_locations,
+                                  const float *attention_weights,
+                                  const float *grad_output, float *grad_value,
+                                  float *grad_sampling_locations,
+                                  float *grad_attention_weights, void *stream);
+
+/*
  * Host-side metadata check, for callers that hold host copies of the metadata
  * (the pages' layer asserts sum_l H_l * W_l == S before calling the op;
  * "Deformable DETR模型解读", MultiScaleDeformableAttention.forward).

@@ -34,6 +34,7 @@ SIGNATURES = {
     "msda_forward": (_I32, [_I64] * 7 + [_I32] + [_VP] * 7),
     "msda_backward": (_I32, [_I64] * 7 + [_I32] + [_VP] * 10 + [_SZ, _VP]),
     "msda_backward_workspace_size": (_I32, [_I64] * 7 + [ctypes.POINTER(_SZ)]),
+    "msda_backward_noalloc": (_I32, [_I64] * 7 + [_I32] + [_VP] * 10),
     "msda_check_metadata": (_I32, [_I64, _I64, _VP, _VP]),
     "msda_status_string": (ctypes.c_char_p, [_I32]),
     "msda_version": (_I32, []),
