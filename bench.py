@@ -78,23 +78,24 @@ def algorithmic_bytes(cfg: W.Config, inp: W.Inputs) -> dict:
     return {"forward": fwd, "backward": bwd}
 
 
-def source_digest() -> str:
+def source_digest(files) -> str:
+    """Digest of the kernel sources a recorded measurement depends on."""
     h = hashlib.sha256()
-    for name in sorted(os.listdir(KERNEL_SOURCES)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(KERNEL_SOURCES, name), "rb") as f:
-                h.update(name.encode() + f.read())
+    for name in sorted(files):
+        with open(os.path.join(KERNEL_SOURCES, name), "rb") as f:
+            h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 
 def recorded_traffic(key: str):
-    """ncu DRAM bytes per launch recorded for the current kernel sources, or None."""
+    """ncu DRAM bytes per launch recorded in profiles/traffic.json for `key`, or
+    None when there is no record or the kernel's sources changed since."""
     try:
         with open(TRAFFIC_FILE) as f:
             rec = json.load(f).get(key)
-    except (OSError, ValueError):
-        return None
-    if not rec or rec.get("source_digest") != source_digest():
+        if not rec or rec.get("source_digest") != source_digest(rec["files"]):
+            return None
+    except (OSError, ValueError, KeyError):
         return None
     return rec.get("dram_bytes_per_launch")
 
