@@ -60,7 +60,7 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kUnroll = 4;                    // points in flight per thread (hist / place)
 constexpr int kChunkPoints = 16384;           // points of a segment per hist / place block
-constexpr int kHistCells = 48 * 1024;         // shared counters per band (192 KB)
+constexpr int kHistCells = 16 * 1024;         // shared counters per band (64 KB: 3 blocks / SM)
 constexpr int kScanItems = 8;                 // per thread
 constexpr int kScanTile = kThreads * kScanItems;
 constexpr int kRunRecords = 64;               // records per sub-warp in the cell pass
@@ -145,7 +145,7 @@ hist_kernel(const int64_t* __restrict__ spatial_shapes, const int64_t* __restric
             const float* __restrict__ attention_weights, float* __restrict__ grad_loc,
             float* __restrict__ grad_attn, int* __restrict__ counts, int* __restrict__ slots,
             long long S, int M, long long Lq, int L, int K, long long cells_per_bm,
-            int chunks) {
+            int chunks, long long keys) {
   extern __shared__ int hist[];
   __shared__ Levels lv;
   __shared__ CellLevels cl;
@@ -174,8 +174,8 @@ hist_kernel(const int64_t* __restrict__ spatial_shapes, const int64_t* __restric
         const long long i = i0 + u * kThreads;
         if (i < i_end) {
           const long long q = i / K;
-          xy[u] = __ldg(reinterpret_cast<const float2*>(sampling_locations) + sg.p_base +
-                        q * sg.p_q + (i - q * K));
+          xy[u] = __ldcs(reinterpret_cast<const float2*>(sampling_locations) + sg.p_base +
+                         q * sg.p_q + (i - q * K));
         }
       }
 #pragma unroll
@@ -187,7 +187,7 @@ hist_kernel(const int64_t* __restrict__ spatial_shapes, const int64_t* __restric
         const Cell c = locate(xy[u].x, xy[u].y, H, W);
         const int cell = ncells > 0 ? point_cell(c, W) : -1;
         if (cell >= lo && cell < lo + span) {
-          slots[p] = atomicAdd(hist + (cell - lo), 1);
+          __stcs(slots + p, atomicAdd(hist + (cell - lo), 1));
         } else if (cell < 0 && lo == 0) {
           // No corner in the map: every corner dot product is 0.  The products
           // with the weights keep the NaN of a non-finite location, as the
@@ -202,7 +202,7 @@ hist_kernel(const int64_t* __restrict__ spatial_shapes, const int64_t* __restric
     }
     __syncthreads();
     for (int c = threadIdx.x; c < span; c += kThreads)
-      counts[(key0 + lo + c) * chunks + chunk] = hist[c];
+      counts[chunk * keys + key0 + lo + c] = hist[c];
     lo += kHistCells;
     __syncthreads();
   } while (lo < ncells);
@@ -301,7 +301,8 @@ place_kernel(const int64_t* __restrict__ spatial_shapes, const int64_t* __restri
              const float* __restrict__ attention_weights, const int* __restrict__ offsets,
              const int* __restrict__ slots, float4* __restrict__ records,
              int* __restrict__ record_keys, long long S, int M, long long Lq, int L, int K,
-             long long cells_per_bm, int chunks) {
+             long long cells_per_bm, int chunks, long long keys) {
+  extern __shared__ int s_off[];  // this chunk's offsets of the band's cells
   __shared__ Levels lv;
   __shared__ CellLevels cl;
   stage_levels(lv, spatial_shapes, level_start, L, S);
@@ -316,6 +317,11 @@ place_kernel(const int64_t* __restrict__ spatial_shapes, const int64_t* __restri
   const long long i_begin = static_cast<long long>(chunk) * kChunkPoints;
   const long long i_end = min(seg_len, i_begin + kChunkPoints);
   const long long key0 = (sg.b * M + sg.m) * cells_per_bm + cl.base[sg.l];
+  const int* chunk_offsets = offsets + chunk * keys + key0;
+  for (int lo = 0; lo < ncells; lo += kHistCells) {
+  const int span = min(kHistCells, ncells - lo);
+  for (int c = threadIdx.x; c < span; c += kThreads) s_off[c] = chunk_offsets[lo + c];
+  __syncthreads();
   for (long long i0 = i_begin + threadIdx.x; i0 < i_end; i0 += kThreads * kUnroll) {
     float2 xy[kUnroll];
     float a[kUnroll];
@@ -325,8 +331,10 @@ place_kernel(const int64_t* __restrict__ spatial_shapes, const int64_t* __restri
       if (i < i_end) {
         const long long q = i / K;
         const long long p = sg.p_base + q * sg.p_q + (i - q * K);
-        xy[u] = __ldg(reinterpret_cast<const float2*>(sampling_locations) + p);
-        a[u] = __ldg(attention_weights + p);
+        // One-touch streams are marked evict-first, so that the randomly read
+        // offsets stay in L2.
+        xy[u] = __ldcs(reinterpret_cast<const float2*>(sampling_locations) + p);
+        a[u] = __ldcs(attention_weights + p);
       }
     }
 #pragma unroll
@@ -337,11 +345,41 @@ place_kernel(const int64_t* __restrict__ spatial_shapes, const int64_t* __restri
       const long long p = sg.p_base + q * sg.p_q + (i - q * K);
       const Cell c = locate(xy[u].x, xy[u].y, H, W);
       const int cell = point_cell(c, W);
-      if (cell < 0) continue;
-      const long long key = key0 + cell;
-      const int pos = offsets[key * chunks + chunk] + slots[p];
-      records[pos] = make_float4(__int_as_float(static_cast<int>(p)), a[u], c.fx, c.fy);
-      record_keys[pos] = static_cast<int>(key);
+      if (cell < lo || cell >= lo + span) continue;
+      const int pos = s_off[cell - lo] + __ldcs(slots + p);
+      __stcs(records + pos, make_float4(__int_as_float(static_cast<int>(p)), a[u], c.fx, c.fy));
+      __stcs(record_keys + pos, static_cast<int>(key0 + cell));
+    }
+  }
+  __syncthreads();  // s_off is reloaded for the next band
+  }
+}
+
+// Per-key totals over the chunks of the chunk-major counts[chunk][key].
+__global__ void __launch_bounds__(kThreads)
+column_totals_kernel(const int* __restrict__ counts, int* __restrict__ totals, long long keys,
+                     int chunks) {
+  for (long long k = blockIdx.x * static_cast<long long>(kThreads) + threadIdx.x; k <= keys;
+       k += static_cast<long long>(gridDim.x) * kThreads) {
+    int s = 0;
+    if (k < keys)
+      for (int c = 0; c < chunks; ++c) s += counts[c * keys + k];
+    totals[k] = s;  // totals[keys] = 0: after the exclusive scan, the record count
+  }
+}
+
+// counts[chunk][key] -> position of the (key, chunk) run: the key's base (scanned
+// totals) plus the counts of the key's earlier chunks.
+__global__ void __launch_bounds__(kThreads)
+finalize_offsets_kernel(int* __restrict__ counts, const int* __restrict__ bases, long long keys,
+                        int chunks) {
+  for (long long k = blockIdx.x * static_cast<long long>(kThreads) + threadIdx.x; k < keys;
+       k += static_cast<long long>(gridDim.x) * kThreads) {
+    int run = bases[k];
+    for (int c = 0; c < chunks; ++c) {
+      const int v = counts[c * keys + k];
+      counts[c * keys + k] = run;
+      run += v;
     }
   }
 }
@@ -408,14 +446,26 @@ struct CellGeom {
   long long dy;   // W * M * D
 };
 
-__device__ __forceinline__ CellGeom decode_key(int key, long long cells_per_bm, int M, int L,
+// The divisions by cells_per_bm and M use precomputed magic numbers.
+struct KeyDiv {
+  FastDiv per_cells;  // key -> b * M + m
+  FastDiv per_m;      // b * M + m -> b
+  int cells_per_bm;
+};
+
+__device__ __forceinline__ int key_head(int key, const KeyDiv& kd, int M) {
+  const int bm = fast_div(key, kd.per_cells);
+  return bm - fast_div(bm, kd.per_m) * M;
+}
+
+__device__ __forceinline__ CellGeom decode_key(int key, const KeyDiv& kd, int M, int L,
                                                long long S, int D, int ch, const Levels& lv,
                                                const CellLevels& cl) {
   CellGeom g;
-  const long long bm = key / cells_per_bm;
-  const int within = static_cast<int>(key - bm * cells_per_bm);
-  g.m = static_cast<int>(bm % M);
-  const long long b = bm / M;
+  const int bm = fast_div(key, kd.per_cells);
+  const int within = key - bm * kd.cells_per_bm;
+  const int b = fast_div(bm, kd.per_m);
+  g.m = bm - b * M;
   int l = 0;
   while (l + 1 < L && !(within >= cl.base[l] && within < cl.base[l] + cl.count[l])) ++l;
   g.W = lv.W[l];
@@ -429,7 +479,7 @@ __device__ __forceinline__ CellGeom decode_key(int key, long long cells_per_bm, 
   g.vy1 = y0 + 1 < g.H;
   const long long MD = static_cast<long long>(M) * D;
   const long long pix = lv.start[l] + static_cast<long long>(y0) * g.W + g.x0;
-  g.ofs = (b * S + pix) * MD + static_cast<long long>(g.m) * D + ch;
+  g.ofs = (static_cast<long long>(b) * S + pix) * MD + static_cast<long long>(g.m) * D + ch;
   g.dy = g.W * MD;
   return g;
 }
@@ -443,7 +493,7 @@ cell_kernel(const float* __restrict__ value, const int64_t* __restrict__ spatial
             const int* __restrict__ total_records, const float4* __restrict__ records,
             const int* __restrict__ record_keys, float* __restrict__ grad_value,
             float* __restrict__ grad_loc, float* __restrict__ grad_attn, long long S, int M,
-            int D, int L, long long cells_per_bm, FastDiv per_bq) {
+            int D, int L, long long cells_per_bm, KeyDiv kd, FastDiv per_bq) {
   constexpr int NB = LANES < 4 ? LANES : 4;
   using R = Row<CPL>;
   __shared__ Levels lv;
@@ -483,7 +533,7 @@ cell_kernel(const float* __restrict__ value, const int64_t* __restrict__ spatial
     }
   };
   auto enter = [&](int key) {
-    const CellGeom ng = decode_key(key, cells_per_bm, M, L, S, D, ch, lv, cl);
+    const CellGeom ng = decode_key(key, kd, M, L, S, D, ch, lv, cl);
     // Moving right along a row keeps the shared column: values and sums.
     const bool right = cur >= 0 && key == cur + 1 && ng.x0 >= 0;
     if (cur >= 0) flush(right);
@@ -513,53 +563,89 @@ cell_kernel(const float* __restrict__ value, const int64_t* __restrict__ spatial
     cur = key;
   };
 
-  for (int i0 = r0; i0 < r1; i0 += NB) {
-    // Lane j (< NB) holds record i0 + j.
-    float4 rec = make_float4(__int_as_float(-1), 0.0f, 0.0f, 0.0f);
-    int rkey = -1;
-    if (lane < NB && i0 + lane < r1) {
-      rec = records[i0 + lane];
-      rkey = record_keys[i0 + lane];
+  // Software pipeline: the records of batch b + 1 sit in registers and their
+  // grad_output slices are being copied (cp.async) into shared memory while
+  // batch b is computed.  Each lane copies exactly the 16-byte slices it later
+  // reads, so the copies need no barrier, only the lane's own wait.
+  __shared__ float4 ring[2][NB][CPL / 4][kThreads];
+  const int nb = (r1 - r0 + NB - 1) / NB;
+  auto load_batch = [&](int bb, float4& rec, int& key) {
+    rec = make_float4(__int_as_float(-1), 0.0f, 0.0f, 0.0f);
+    key = -1;
+    const int i = r0 + bb * NB + lane;
+    if (lane < NB && bb < nb && i < r1) {
+      key = __ldcs(record_keys + i);
+      rec = __ldcs(records + i);
     }
-    // The batch's grad_output rows first, so that their loads overlap.
-    int keys[NB];
-    R go[NB];
+  };
+  auto issue_go = [&](const float4& rec, int key, int stage) {
 #pragma unroll
     for (int j = 0; j < NB; ++j) {
-      keys[j] = __shfl_sync(mask, rkey, j, LANES);
-      const int p = __float_as_int(__shfl_sync(mask, rec.x, j, LANES));
-      go[j] = zero_row<CPL>();
-      if (keys[j] >= 0) {
-        const int bq = fast_div(p, per_bq);
-        const int m = static_cast<int>((keys[j] / cells_per_bm) % M);
-        go[j] = load_row<CPL>(grad_output + static_cast<long long>(bq) * MD +
-                                  static_cast<long long>(m) * D + ch,
-                              on);
+      const int kj = __shfl_sync(mask, key, j, LANES);
+      const int pj = __float_as_int(__shfl_sync(mask, rec.x, j, LANES));
+      if (kj >= 0) {
+        const int bq = fast_div(pj, per_bq);
+        const int m = key_head(kj, kd, M);
+        const float* src = grad_output + static_cast<long long>(bq) * MD +
+                           static_cast<long long>(m) * D + ch;
+#pragma unroll
+        for (int h = 0; h < CPL / 4; ++h)
+          if (on[h]) {
+            const unsigned dst =
+                static_cast<unsigned>(__cvta_generic_to_shared(&ring[stage][j][h][threadIdx.x]));
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src + 4 * h)
+                         : "memory");
+          }
       }
     }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+
+  float4 rec_cur, rec_nxt, rec_nn;
+  int key_cur, key_nxt, key_nn;
+  load_batch(0, rec_cur, key_cur);
+  issue_go(rec_cur, key_cur, 0);
+  load_batch(1, rec_nxt, key_nxt);
+  for (int b = 0; b < nb; ++b) {
+    const int stage = b & 1;
+    issue_go(rec_nxt, key_nxt, stage ^ 1);  // batch b + 1
+    load_batch(b + 2, rec_nn, key_nn);
+    asm volatile("cp.async.wait_group 1;" ::: "memory");  // batch b's slices are in
+
     float part[4][NB];
     float myW = 0.0f, myH = 0.0f;
 #pragma unroll
     for (int j = 0; j < NB; ++j) {
-      const float a = __shfl_sync(mask, rec.y, j, LANES);
-      const float fx = __shfl_sync(mask, rec.z, j, LANES);
-      const float fy = __shfl_sync(mask, rec.w, j, LANES);
+      const int kj = __shfl_sync(mask, key_cur, j, LANES);
+      const float a = __shfl_sync(mask, rec_cur.y, j, LANES);
+      const float fx = __shfl_sync(mask, rec_cur.z, j, LANES);
+      const float fy = __shfl_sync(mask, rec_cur.w, j, LANES);
       part[0][j] = part[1][j] = part[2][j] = part[3][j] = 0.0f;
-      if (keys[j] < 0) continue;  // past the end of the run (uniform in the sub-warp)
-      if (keys[j] != cur) enter(keys[j]);
+      if (kj < 0) continue;  // past the end of the run (uniform in the sub-warp)
+      if (kj != cur) enter(kj);
       if (lane == j) {
         myW = static_cast<float>(g.W);
         myH = static_cast<float>(g.H);
       }
-      part[0][j] = dot_row(go[j], c00);
-      part[1][j] = dot_row(go[j], c10);
-      part[2][j] = dot_row(go[j], c01);
-      part[3][j] = dot_row(go[j], c11);
+      R go = zero_row<CPL>();
+#pragma unroll
+      for (int h = 0; h < CPL / 4; ++h)
+        if (on[h]) {
+          const float4 x = ring[stage][j][h][threadIdx.x];
+          go.v[4 * h + 0] = x.x;
+          go.v[4 * h + 1] = x.y;
+          go.v[4 * h + 2] = x.z;
+          go.v[4 * h + 3] = x.w;
+        }
+      part[0][j] = dot_row(go, c00);
+      part[1][j] = dot_row(go, c10);
+      part[2][j] = dot_row(go, c01);
+      part[3][j] = dot_row(go, c11);
       const float hx = 1.0f - fx, hy = 1.0f - fy;
-      axpy_row(a * hx * hy, go[j], a00);
-      axpy_row(a * fx * hy, go[j], a10);
-      axpy_row(a * hx * fy, go[j], a01);
-      axpy_row(a * fx * fy, go[j], a11);
+      axpy_row(a * hx * hy, go, a00);
+      axpy_row(a * fx * hy, go, a10);
+      axpy_row(a * hx * fy, go, a01);
+      axpy_row(a * fx * fy, go, a11);
     }
     // Butterfly over the lane bits above the batch, then a reduce-scatter so that
     // lane j (< NB) ends with the totals of record j.
@@ -582,9 +668,9 @@ cell_kernel(const float* __restrict__ value, const int64_t* __restrict__ spatial
           part[q][j] = keep + __shfl_xor_sync(mask, send, o, LANES);
         }
     }
-    if (lane < NB && rkey >= 0) {
-      const int p = __float_as_int(rec.x);
-      const float a = rec.y, fx = rec.z, fy = rec.w;
+    if (lane < NB && key_cur >= 0) {
+      const int p = __float_as_int(rec_cur.x);
+      const float a = rec_cur.y, fx = rec_cur.z, fy = rec_cur.w;
       const float hx = 1.0f - fx, hy = 1.0f - fy;
       const float g00 = part[0][0], g10 = part[1][0], g01 = part[2][0], g11 = part[3][0];
       grad_attn[p] = fmaf(hy, fmaf(fx, g10, hx * g00), fy * fmaf(fx, g11, hx * g01));
@@ -592,7 +678,12 @@ cell_kernel(const float* __restrict__ value, const int64_t* __restrict__ spatial
           make_float2(a * myW * fmaf(hy, g10 - g00, fy * (g11 - g01)),
                       a * myH * fmaf(hx, g01 - g00, fx * (g11 - g10)));
     }
+    rec_cur = rec_nxt;
+    key_cur = key_nxt;
+    rec_nxt = rec_nn;
+    key_nxt = key_nn;
   }
+  asm volatile("cp.async.wait_all;" ::: "memory");
   if (cur >= 0) flush(false);
 }
 
@@ -614,10 +705,14 @@ cudaError_t launch_cells(const BackwardArgs& a, const SortedLayout& w, const int
                          const float4* records, const int* record_keys, cudaStream_t stream) {
   const long long runs = (w.points + kRunRecords - 1) / kRunRecords;
   const FastDiv per_bq = make_fastdiv(static_cast<long long>(a.M) * a.L * a.K);
+  KeyDiv kd;
+  kd.per_cells = make_fastdiv(w.cells_per_bm);
+  kd.per_m = make_fastdiv(a.M);
+  kd.cells_per_bm = static_cast<int>(w.cells_per_bm);
   cell_kernel<LANES, CPL><<<grid_for(runs * LANES, kThreads), kThreads, 0, stream>>>(
       a.value, a.spatial_shapes, a.level_start_index, a.grad_output, total, records, record_keys,
       a.grad_value, a.grad_sampling_locations, a.grad_attention_weights, a.S, a.M, a.D, a.L,
-      w.cells_per_bm, per_bq);
+      w.cells_per_bm, kd, per_bq);
   return cudaGetLastError();
 }
 
@@ -627,15 +722,16 @@ SortedLayout sorted_layout(long long B, long long S, long long M, long long Lq, 
   SortedLayout w;
   // sum_l (H_l + 1)(W_l + 1) <= 2 S + 2 L, because H + W <= H W + 1 for H, W >= 1.
   w.cells_per_bm = 2 * S + 2 * L;
+  w.keys = B * M * w.cells_per_bm;
   w.segments = B * M * L;
   w.segment_len = Lq * K;
   w.chunks = (w.segment_len + kChunkPoints - 1) / kChunkPoints;
   if (w.chunks < 1) w.chunks = 1;
   w.points = w.segments * w.segment_len;
-  w.counts = B * M * w.cells_per_bm * w.chunks;
-  w.scan_tiles = (w.counts + 1 + kScanTile - 1) / kScanTile;
+  w.counts = w.keys * w.chunks;
+  w.scan_tiles = (w.keys + 1 + kScanTile - 1) / kScanTile;
   auto up = [](long long bytes) { return (bytes + 255) / 256 * 256; };
-  w.bytes = up(4 * (w.counts + 1)) + up(4 * w.scan_tiles) + up(4 * w.points) +
+  w.bytes = up(4 * w.counts) + up(4 * (w.keys + 1)) + up(4 * w.scan_tiles) + up(4 * w.points) +
             up(16 * w.points) + up(4 * w.points);
   return w;
 }
@@ -644,7 +740,8 @@ cudaError_t launch_backward_sorted(const BackwardArgs& a, void* workspace,
                                    cudaStream_t stream) {
   const SortedLayout w = sorted_layout(a.B, a.S, a.M, a.Lq, a.L, a.K);
   char* cursor = static_cast<char*>(workspace);
-  int* counts = carve<int>(cursor, w.counts + 1);
+  int* counts = carve<int>(cursor, w.counts);      // counts[chunk][key], then run offsets
+  int* totals = carve<int>(cursor, w.keys + 1);    // per-key totals, then key bases
   int* tile_sums = carve<int>(cursor, w.scan_tiles);
   int* slots = carve<int>(cursor, w.points);
   float4* records = carve<float4>(cursor, w.points);
@@ -652,45 +749,55 @@ cudaError_t launch_backward_sorted(const BackwardArgs& a, void* workspace,
 
   cudaError_t err = launch_zero(a.grad_value, a.value_elements, stream);
   if (err != cudaSuccess || w.points == 0) return err;
-  // Counts of cells that no block writes (keys past a segment's levels) stay 0;
+  // Counts of keys that no block writes (keys past a segment's levels) stay 0;
   // the zero fill covers whole float4s, which the 256-byte carve leaves room for.
-  if ((err = launch_zero(reinterpret_cast<float*>(counts), (w.counts + 1 + 3) / 4 * 4,
-                         stream)) != cudaSuccess)
+  if ((err = launch_zero(reinterpret_cast<float*>(counts), (w.counts + 3) / 4 * 4, stream)) !=
+      cudaSuccess)
     return err;
 
-  // The hist kernel's counters exceed the default 48 KB of dynamic shared
-  // memory; the opt-in is set once per device.
-  const size_t hist_smem = sizeof(int) * static_cast<size_t>(kHistCells);
+  // The hist and place kernels' per-cell tables exceed the default 48 KB of
+  // dynamic shared memory; the opt-in is set once per device.
+  const size_t cell_smem = sizeof(int) * static_cast<size_t>(kHistCells);
   static bool smem_set[64] = {};
   int dev = 0;
   if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
   if (dev < 0 || dev >= 64 || !smem_set[dev]) {
-    err = cudaFuncSetAttribute(hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(hist_smem));
-    if (err != cudaSuccess) return err;
+    if ((err = cudaFuncSetAttribute(hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    static_cast<int>(cell_smem))) != cudaSuccess ||
+        (err = cudaFuncSetAttribute(place_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    static_cast<int>(cell_smem))) != cudaSuccess)
+      return err;
     if (dev >= 0 && dev < 64) smem_set[dev] = true;
   }
   const unsigned blocks = static_cast<unsigned>(w.segments * w.chunks);
   const int chunks = static_cast<int>(w.chunks);
-  hist_kernel<<<blocks, kThreads, hist_smem, stream>>>(
+  hist_kernel<<<blocks, kThreads, cell_smem, stream>>>(
       a.spatial_shapes, a.level_start_index, a.sampling_locations, a.attention_weights,
       a.grad_sampling_locations, a.grad_attention_weights, counts, slots, a.S, a.M, a.Lq, a.L,
-      a.K, w.cells_per_bm, chunks);
+      a.K, w.cells_per_bm, chunks, w.keys);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  // Key-major positions from the chunk-major counts: per-key totals, their
+  // exclusive scan, then each (key, chunk) run's offset.
+  column_totals_kernel<<<grid_for(w.keys + 1, kThreads), kThreads, 0, stream>>>(
+      counts, totals, w.keys, chunks);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   scan_tiles_kernel<<<static_cast<unsigned>(w.scan_tiles), kThreads, 0, stream>>>(
-      counts, tile_sums, w.counts + 1);
+      totals, tile_sums, w.keys + 1);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   scan_sums_kernel<<<1, 1024, 0, stream>>>(tile_sums, static_cast<int>(w.scan_tiles));
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   scan_add_kernel<<<static_cast<unsigned>(w.scan_tiles), kThreads, 0, stream>>>(
-      counts, tile_sums, w.counts + 1);
+      totals, tile_sums, w.keys + 1);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  place_kernel<<<blocks, kThreads, 0, stream>>>(
+  finalize_offsets_kernel<<<grid_for(w.keys, kThreads), kThreads, 0, stream>>>(
+      counts, totals, w.keys, chunks);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  place_kernel<<<blocks, kThreads, cell_smem, stream>>>(
       a.spatial_shapes, a.level_start_index, a.sampling_locations, a.attention_weights, counts,
-      slots, records, record_keys, a.S, a.M, a.Lq, a.L, a.K, w.cells_per_bm, chunks);
+      slots, records, record_keys, a.S, a.M, a.Lq, a.L, a.K, w.cells_per_bm, chunks, w.keys);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  // counts[w.counts] now holds the number of records.
-  const int* total = counts + w.counts;
+  // totals[keys] now holds the number of records.
+  const int* total = totals + w.keys;
   int lanes = 1;
   while (lanes * kCellChannels < a.D) lanes <<= 1;
   switch (lanes) {

@@ -46,11 +46,12 @@ struct BackwardArgs {
 // Scratch layout of the cell-sorted backward (msda_backward_sorted.cu).
 struct SortedLayout {
   long long cells_per_bm;  // keys per (b, m): bound on sum_l (H_l + 1)(W_l + 1) from S, L
+  long long keys;          // B * M * cells_per_bm cell keys
   long long segments;      // B * M * L: one (b, m, level) each
   long long segment_len;   // Lq * K points per segment
   long long chunks;        // hist / place blocks per segment
   long long points;        // B * Lq * M * L * K
-  long long counts;        // B * M * cells_per_bm * chunks (cell, chunk) counters
+  long long counts;        // keys * chunks (chunk, cell) counters
   long long scan_tiles;
   long long bytes;         // workspace bytes
 };

@@ -139,9 +139,12 @@ def test_workspace_size(lib):
     assert st == OK
     points = 4 * 19947 * 8 * 16
     chunks = -(-19947 * 4 // 16384)
-    counts = 4 * 8 * (2 * 19947 + 2 * 4) * chunks
-    # slot 4 B + record 16 B + record key 4 B per point; one counter per (cell, chunk).
-    assert 24 * points + 4 * counts <= need < 24 * points + 4 * counts + 64 * 1024
+    keys = 4 * 8 * (2 * 19947 + 2 * 4)
+    counts = keys * chunks
+    # slot 4 B + record 16 B + record key 4 B per point; one counter per (chunk, cell)
+    # and one total per cell.
+    fixed = 24 * points + 4 * counts + 4 * keys
+    assert fixed <= need < fixed + 64 * 1024
     assert _ws_size(lib, B=-1)[0] == BAD
     assert _ws_size(lib, B=1 << 14, Lq=1 << 14, M=8)[0] == UNSUP  # 32-bit point ids overflow
     assert lib.msda_backward_workspace_size(1, 80, 2, 8, 80, 2, 2, None) == NULLP
