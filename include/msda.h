@@ -144,7 +144,7 @@ msda_status msda_backward(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq
  * Bytes of workspace msda_backward needs for these sizes (host only; no device
  * access).  The bound depends on the sizes alone: a level of H x W pixels has
  * (H + 1)(W + 1) bilinear cells, and sum_l (H_l + 1)(W_l + 1) <= 2 S + 2 L.
- * For B=4, S=Lq=19947, M=8, L=K=4 it is about 250 MB.  Returns
+ * For B=4, S=Lq=19947, M=8, L=K=4 it is about 276 MB.  Returns
  * MSDA_ERR_UNSUPPORTED when the sorted path's 32-bit cell and point ids would
  * overflow (B*M*(2S+2L) or B*Lq*M*L*K at 2^31 or more); the scratch-free path
  * still accepts those sizes.
@@ -174,7 +174,7 @@ msda_status msda_backward_workspace_size(int64_t B, int64_t S, int64_t M, int64_
  * no cudaMalloc, cudaFree or other allocating routine.
  *   - Sizes whose msda_backward_workspace_size exceeds MSDA_NOALLOC_SCRATCH_BYTES
  *     are rejected with MSDA_ERR_WORKSPACE before anything is enqueued (for
- *     example B=1, S=19947, M=8, D=32, L=K=4 fits up to Lq = 9600 queries).
+ *     example B=1, S=19947, M=8, D=32, L=K=4 fits up to Lq = 9259 queries).
  *   - The first call on a device looks up the array's device address (set-up,
  *     once per device, with that device current); make that first call before
  *     any stream capture.

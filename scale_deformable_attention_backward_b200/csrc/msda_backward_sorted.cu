@@ -30,12 +30,15 @@
 //
 //   1. hist    one block per (segment, chunk): the cell of each point and its slot
 //              among the chunk's points of that cell (shared-memory atomic);
-//              the chunk's per-cell counts go to counts[key][chunk].  Points with
-//              no corner in the map get their (zero or NaN) gradients here.
-//   2. scan    exclusive prefix sum over counts (three launches): the position of
-//              every (cell, chunk) run in the sorted record array.
-//   3. place   one block per (segment, chunk): each point's record (id, A, fx,
-//              fy) and key at counts[key][chunk] + slot.
+//              the chunk's per-cell counts go to counts[chunk][key] (coalesced
+//              rows).  Points with no corner in the map get their (zero or NaN)
+//              gradients here.
+//   2. offsets per-key totals over the chunks, their exclusive prefix sum (three
+//              launches), then counts[chunk][key] becomes the position of the
+//              (key, chunk) run in the sorted record array.
+//   3. place   one block per (segment, chunk): the chunk's run offsets of the
+//              segment's cells are staged in shared memory; each point's record
+//              (id, A, fx, fy) and key go to offset + slot.
 //   4. cells   every sub-warp takes a fixed run of consecutive records, so the
 //              work is balanced whatever the cell sizes.  For a batch of records
 //              it issues all their corner and grad_output loads at once (in sorted
@@ -48,8 +51,8 @@
 //              the lanes; lane j finishes record j).
 //
 // Scratch (caller-provided workspace, see msda_backward_workspace_size): counts
-// per (cell, chunk), scan tile sums, the slot of every point, and the sorted
-// records (16 bytes) and keys (4 bytes).
+// per (chunk, cell), per-cell totals, scan tile sums, the slot of every point,
+// and the sorted records (16 bytes) and keys (4 bytes).
 #include "msda_device.cuh"
 #include "msda_launch.h"
 
@@ -159,7 +162,7 @@ hist_kernel(const int64_t* __restrict__ spatial_shapes, const int64_t* __restric
   const long long seg_len = Lq * K;
   const long long i_begin = static_cast<long long>(chunk) * kChunkPoints;
   const long long i_end = min(seg_len, i_begin + kChunkPoints);
-  // counts index of (cell, chunk): key * chunks + chunk.
+  // counts index of (chunk, cell): chunk * keys + key.
   const long long key0 = (sg.b * M + sg.m) * cells_per_bm + cl.base[sg.l];
 
   int lo = 0;

@@ -94,6 +94,18 @@ __device__ __forceinline__ Cell locate(float lx, float ly, int H, int W) {
   return c;
 }
 
+// Packed float32 pair FMA (sm_100): d = a * b + c on both halves, each rounded
+// once as fmaf would.
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;"
+      : "=l"(d)
+      : "l"(*reinterpret_cast<unsigned long long*>(&a)),
+        "l"(*reinterpret_cast<unsigned long long*>(&b)),
+        "l"(*reinterpret_cast<unsigned long long*>(&c)));
+  return *reinterpret_cast<float2*>(&d);
+}
+
 // ---------------------------------------------------------------------------
 // 16-byte lane vectors: 4 x float32 or 8 x bfloat16, widened to float32.
 // ---------------------------------------------------------------------------

@@ -74,17 +74,6 @@ __device__ __forceinline__ PointSetup setup_point(float lx, float ly, float a, i
   return s;
 }
 
-// Packed float32 pair FMA (sm_100): d = a * b + c on both halves.
-__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
-  unsigned long long d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;"
-      : "=l"(d)
-      : "l"(*reinterpret_cast<unsigned long long*>(&a)),
-        "l"(*reinterpret_cast<unsigned long long*>(&b)),
-        "l"(*reinterpret_cast<unsigned long long*>(&c)));
-  return *reinterpret_cast<float2*>(&d);
-}
-
 template <typename T>
 struct Corner;
 
