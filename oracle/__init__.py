@@ -33,6 +33,14 @@ class Oracle:
         lib.msda_oracle_backward.restype = ctypes.c_int
         lib.msda_oracle_backward.argtypes = [_I64] * 7 + [_PD, _PI, _PI, _PD, _PD, _PD,
                                                           _PD, _PD, _PD]
+        if hasattr(lib, "msda_oracle_fused_forward"):
+            lib.msda_oracle_fused_forward.restype = ctypes.c_int
+            lib.msda_oracle_fused_forward.argtypes = ([_I64] * 8 + [ctypes.c_int] +
+                                                      [_PD, _PI, _PI, _PD, _PD, _PD, _PD])
+            lib.msda_oracle_fused_backward.restype = ctypes.c_int
+            lib.msda_oracle_fused_backward.argtypes = ([_I64] * 8 + [ctypes.c_int] +
+                                                       [_PD, _PI, _PI, _PD, _PD, _PD, _PD,
+                                                        _PD, _PD, _PD, _PD])
         self.lib = lib
         self.path = library_path
 
@@ -97,6 +105,64 @@ class Oracle:
         return gv, gl, ga
 
 
+    @staticmethod
+    def _fused_dims(value, spatial_shapes, reference_points, sampling_offsets,
+                    attention_logits):
+        B, S, M, D = value.shape
+        Bq, Lq, Mq, L, K, two = sampling_offsets.shape
+        if (Bq, Mq, two) != (B, M, 2):
+            raise ValueError("sampling_offsets must be [B, Lq, M, L, K, 2]")
+        if reference_points.ndim != 4 or reference_points.shape[:3] != (B, Lq, L):
+            raise ValueError("reference_points must be [B, Lq, L, R]")
+        R = reference_points.shape[3]
+        if R not in (2, 4):
+            raise ValueError("reference_points must have 2 or 4 components")
+        if attention_logits.shape != (B, Lq, M, L * K):
+            raise ValueError("attention_logits must be [B, Lq, M, L*K]")
+        if spatial_shapes.shape != (L, 2):
+            raise ValueError("spatial_shapes must be [L, 2]")
+        return B, S, M, D, Lq, L, K, R
+
+    def fused_forward(self, value, spatial_shapes, level_start_index, reference_points,
+                      sampling_offsets, attention_logits, round_f32=True):
+        """Output [B, Lq, M*D] float64 of the op fed with raw reference points,
+        offsets and logits (locations in float32 when ``round_f32``)."""
+        v, sh, st = self._f64(value), self._i64(spatial_shapes), self._i64(level_start_index)
+        ref, off = self._f64(reference_points), self._f64(sampling_offsets)
+        z = self._f64(attention_logits)
+        B, S, M, D, Lq, L, K, R = self._fused_dims(v, sh, ref, off, z)
+        out = np.empty((B, Lq, M * D), dtype=np.float64)
+        rc = self.lib.msda_oracle_fused_forward(
+            B, S, M, D, Lq, L, K, R, int(bool(round_f32)), self._p(v, _PD), self._p(sh, _PI),
+            self._p(st, _PI), self._p(ref, _PD), self._p(off, _PD), self._p(z, _PD),
+            self._p(out, _PD))
+        if rc != 0:
+            raise ValueError(f"oracle fused forward failed (rc={rc})")
+        return out
+
+    def fused_backward(self, value, spatial_shapes, level_start_index, reference_points,
+                       sampling_offsets, attention_logits, grad_output, round_f32=True):
+        """Return (grad_value, grad_sampling_offsets, grad_attention_logits,
+        grad_reference_points), all float64."""
+        v, sh, st = self._f64(value), self._i64(spatial_shapes), self._i64(level_start_index)
+        ref, off = self._f64(reference_points), self._f64(sampling_offsets)
+        z = self._f64(attention_logits)
+        B, S, M, D, Lq, L, K, R = self._fused_dims(v, sh, ref, off, z)
+        go = self._f64(grad_output).reshape(B, Lq, M * D)
+        gv = np.empty((B, S, M, D), dtype=np.float64)
+        goff = np.empty((B, Lq, M, L, K, 2), dtype=np.float64)
+        gz = np.empty((B, Lq, M, L * K), dtype=np.float64)
+        gref = np.empty((B, Lq, L, R), dtype=np.float64)
+        rc = self.lib.msda_oracle_fused_backward(
+            B, S, M, D, Lq, L, K, R, int(bool(round_f32)), self._p(v, _PD), self._p(sh, _PI),
+            self._p(st, _PI), self._p(ref, _PD), self._p(off, _PD), self._p(z, _PD),
+            self._p(go, _PD), self._p(gv, _PD), self._p(goff, _PD), self._p(gz, _PD),
+            self._p(gref, _PD))
+        if rc != 0:
+            raise ValueError(f"oracle fused backward failed (rc={rc})")
+        return gv, goff, gz, gref
+
+
 _DEFAULT = None
 
 
@@ -116,4 +182,12 @@ def backward(*args, **kwargs):
     return default().backward(*args, **kwargs)
 
 
-__all__ = ["Oracle", "default", "forward", "backward"]
+def fused_forward(*args, **kwargs):
+    return default().fused_forward(*args, **kwargs)
+
+
+def fused_backward(*args, **kwargs):
+    return default().fused_backward(*args, **kwargs)
+
+
+__all__ = ["Oracle", "default", "forward", "backward", "fused_forward", "fused_backward"]

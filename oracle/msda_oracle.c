@@ -46,10 +46,13 @@
  *   attention_weights   [B, Lq, M, L, K]
  *   output              [B, Lq, M * D]
  *
- * Return value of every entry point: 0 on success, -1 if a shape is negative.
+ * Return value of every entry point: 0 on success, -1 if a shape is negative
+ * (or, for the fused entry points, R is neither 2 nor 4), -2 if scratch memory
+ * could not be allocated.
  */
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 
 /* Integer pixel coordinate of a corner, or -1 if the corner lies outside [0, n). */
 static int64_t corner_index(double c, int64_t n)
@@ -193,4 +196,192 @@ int msda_oracle_backward(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq,
         }
     }
     return 0;
+}
+
+/* ------------------------------------------------------------------------
+ * The step before the core: sampling locations and attention weights formed
+ * from the raw inputs, then the core above.
+ *
+ * Sources (same pages): [walk] MultiScaleDeformableAttention.forward and the
+ * Deformable DETR MSDeformAttn.forward printed on "Deformable DETR模型解读
+ * （附源码+论文）" and on the phdsky.com notes:
+ *  - attention weights: a softmax over the L*K logits of each (b, q, m);
+ *  - reference points with 2 components (x, y): loc = ref + off / (W_l, H_l);
+ *  - reference points with 4 components (box centre x, y and size w, h):
+ *    loc = ref[0:2] + off / K * ref[2:4] * 0.5.
+ * Readings (listed in the design doc):
+ *  - with round_f32 = 1 the location is formed in float32, every operation
+ *    rounded once in the pages' order (division by the normaliser, then the
+ *    addition; for boxes the division by K, the product with the size, the
+ *    product with 0.5, then the addition), as the pages' float32 tensors
+ *    compute it; with round_f32 = 0 it is formed in float64 (used by the
+ *    finite-difference checks).  The softmax is float64 either way.
+ *  - the backward differentiates the real-number formula (the float32
+ *    rounding is not differentiated): d loc / d off = 1 / (W_l, H_l), or
+ *    ref[2:4] * 0.5 / K for boxes; d loc / d ref[0:2] = 1; for boxes
+ *    d loc / d ref[2:4] = off * 0.5 / K; the softmax gives
+ *    d z_i = A_i * (gA_i - sum_j A_j gA_j) over the (b, q, m) group.
+ *
+ * Extra layouts:
+ *   reference_points    [B, Lq, L, R]          R = 2 or 4
+ *   sampling_offsets    [B, Lq, M, L, K, 2]
+ *   attention_logits    [B, Lq, M, L * K]
+ * ------------------------------------------------------------------------ */
+
+static double form_location(double ref_c, double size_c, double off_c, int64_t n,
+                            int64_t K, int64_t R, int round_f32)
+{
+    if (round_f32) {
+        float t;
+        if (R == 2) {
+            t = (float)off_c / (float)n;
+        } else {
+            t = (float)off_c / (float)K;
+            t = t * (float)size_c;
+            t = t * 0.5f;
+        }
+        return (double)((float)ref_c + t);
+    }
+    if (R == 2)
+        return ref_c + off_c / (double)n;
+    return ref_c + off_c / (double)K * size_c * 0.5;
+}
+
+/* loc [B, Lq, M, L, K, 2] and A [B, Lq, M, L, K] from the raw inputs. */
+static void fused_inputs(int64_t B, int64_t Lq, int64_t M, int64_t L, int64_t K,
+                         int64_t R, int round_f32, const int64_t *spatial_shapes,
+                         const double *ref, const double *off, const double *logits,
+                         double *loc, double *A)
+{
+    int64_t LK = L * K;
+    for (int64_t b = 0; b < B; ++b)
+    for (int64_t q = 0; q < Lq; ++q)
+    for (int64_t m = 0; m < M; ++m) {
+        int64_t g = (b * Lq + q) * M + m;
+        const double *z = logits + g * LK;
+        double zmax = z[0];
+        for (int64_t i = 1; i < LK; ++i)
+            if (z[i] > zmax || isnan(z[i]))
+                zmax = z[i];
+        double sum = 0.0;
+        for (int64_t i = 0; i < LK; ++i)
+            sum += exp(z[i] - zmax);
+        for (int64_t i = 0; i < LK; ++i)
+            A[g * LK + i] = exp(z[i] - zmax) / sum;
+        for (int64_t l = 0; l < L; ++l) {
+            const double *r = ref + ((b * Lq + q) * L + l) * R;
+            int64_t H = spatial_shapes[2 * l + 0];
+            int64_t W = spatial_shapes[2 * l + 1];
+            for (int64_t k = 0; k < K; ++k) {
+                int64_t p = g * LK + l * K + k;
+                loc[2 * p + 0] = form_location(r[0], R == 4 ? r[2] : 0.0, off[2 * p + 0], W,
+                                               K, R, round_f32);
+                loc[2 * p + 1] = form_location(r[1], R == 4 ? r[3] : 0.0, off[2 * p + 1], H,
+                                               K, R, round_f32);
+            }
+        }
+    }
+}
+
+int msda_oracle_fused_forward(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq,
+                              int64_t L, int64_t K, int64_t R, int round_f32,
+                              const double *value, const int64_t *spatial_shapes,
+                              const int64_t *level_start_index,
+                              const double *reference_points,
+                              const double *sampling_offsets,
+                              const double *attention_logits, double *output)
+{
+    if (B < 0 || S < 0 || M < 0 || D < 0 || Lq < 0 || L < 0 || K < 0 || (R != 2 && R != 4))
+        return -1;
+    int64_t n = B * Lq * M * L * K;
+    double *loc = malloc(sizeof(double) * (size_t)(2 * n + 1));
+    double *A = malloc(sizeof(double) * (size_t)(n + 1));
+    if (loc == NULL || A == NULL) {
+        free(loc);
+        free(A);
+        return -2;
+    }
+    fused_inputs(B, Lq, M, L, K, R, round_f32, spatial_shapes, reference_points,
+                 sampling_offsets, attention_logits, loc, A);
+    int rc = msda_oracle_forward(B, S, M, D, Lq, L, K, value, spatial_shapes,
+                                 level_start_index, loc, A, output);
+    free(loc);
+    free(A);
+    return rc;
+}
+
+int msda_oracle_fused_backward(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq,
+                               int64_t L, int64_t K, int64_t R, int round_f32,
+                               const double *value, const int64_t *spatial_shapes,
+                               const int64_t *level_start_index,
+                               const double *reference_points,
+                               const double *sampling_offsets,
+                               const double *attention_logits, const double *grad_output,
+                               double *grad_value, double *grad_sampling_offsets,
+                               double *grad_attention_logits,
+                               double *grad_reference_points)
+{
+    if (B < 0 || S < 0 || M < 0 || D < 0 || Lq < 0 || L < 0 || K < 0 || (R != 2 && R != 4))
+        return -1;
+    int64_t n = B * Lq * M * L * K;
+    int64_t LK = L * K;
+    double *loc = malloc(sizeof(double) * (size_t)(2 * n + 1));
+    double *A = malloc(sizeof(double) * (size_t)(n + 1));
+    double *gloc = malloc(sizeof(double) * (size_t)(2 * n + 1));
+    double *gA = malloc(sizeof(double) * (size_t)(n + 1));
+    if (loc == NULL || A == NULL || gloc == NULL || gA == NULL) {
+        free(loc);
+        free(A);
+        free(gloc);
+        free(gA);
+        return -2;
+    }
+    fused_inputs(B, Lq, M, L, K, R, round_f32, spatial_shapes, reference_points,
+                 sampling_offsets, attention_logits, loc, A);
+    int rc = msda_oracle_backward(B, S, M, D, Lq, L, K, value, spatial_shapes,
+                                  level_start_index, loc, A, grad_output, grad_value,
+                                  gloc, gA);
+    if (rc == 0) {
+        if (grad_reference_points != NULL)
+            for (int64_t i = 0; i < B * Lq * L * R; ++i)
+                grad_reference_points[i] = 0.0;
+        for (int64_t b = 0; b < B; ++b)
+        for (int64_t q = 0; q < Lq; ++q)
+        for (int64_t m = 0; m < M; ++m) {
+            int64_t g = (b * Lq + q) * M + m;
+            /* Softmax: d z_i = A_i (gA_i - sum_j A_j gA_j). */
+            double s = 0.0;
+            for (int64_t i = 0; i < LK; ++i)
+                s += A[g * LK + i] * gA[g * LK + i];
+            for (int64_t i = 0; i < LK; ++i)
+                grad_attention_logits[g * LK + i] = A[g * LK + i] * (gA[g * LK + i] - s);
+            for (int64_t l = 0; l < L; ++l) {
+                const double *r = reference_points + ((b * Lq + q) * L + l) * R;
+                double *gr = grad_reference_points == NULL
+                                 ? NULL
+                                 : grad_reference_points + ((b * Lq + q) * L + l) * R;
+                int64_t H = spatial_shapes[2 * l + 0];
+                int64_t W = spatial_shapes[2 * l + 1];
+                for (int64_t k = 0; k < K; ++k) {
+                    int64_t p = g * LK + l * K + k;
+                    for (int c = 0; c < 2; ++c) {
+                        double gl = gloc[2 * p + c];
+                        double dloc_doff = R == 2 ? 1.0 / (double)(c == 0 ? W : H)
+                                                  : r[2 + c] * 0.5 / (double)K;
+                        grad_sampling_offsets[2 * p + c] = gl * dloc_doff;
+                        if (gr != NULL) {
+                            gr[c] += gl;
+                            if (R == 4)
+                                gr[2 + c] += gl * sampling_offsets[2 * p + c] * 0.5 / (double)K;
+                        }
+                    }
+                }
+            }
+        }
+    }
+    free(loc);
+    free(A);
+    free(gloc);
+    free(gA);
+    return rc;
 }

@@ -388,18 +388,15 @@ def pin_finite_differences(orc):
 # P-9: the library routine the pages build on (torch grid_sample, float64, CPU)
 # ----------------------------------------------------------------------------
 
-def grid_sample_reference(value, shapes, start, loc, attn, grad=None):
-    """Forward (and, with ``grad``, autograd gradients) written with
-    ``torch.nn.functional.grid_sample(mode='bilinear', padding_mode='zeros',
-    align_corners=False)`` on float64 CPU tensors, one call per level with grid =
-    2*loc - 1 -- the formulation of ms_deform_attn_core_pytorch ("Deformable
-    DETR模型解读").  Test-only cross-check of the oracle."""
+def grid_sample_core(v, lo, at, shapes, start):
+    """The core on torch float64 CPU tensors (differentiable): value [B,S,M,D],
+    locations [B,Lq,M,L,K,2], weights [B,Lq,M,L,K] -> output [B,Lq,M*D], written
+    with ``torch.nn.functional.grid_sample(mode='bilinear', padding_mode='zeros',
+    align_corners=False)``, one call per level with grid = 2*loc - 1 -- the
+    formulation of ms_deform_attn_core_pytorch ("Deformable DETR模型解读")."""
     import torch
     import torch.nn.functional as F
 
-    v = torch.tensor(value, dtype=torch.float64, requires_grad=grad is not None)
-    lo = torch.tensor(loc, dtype=torch.float64, requires_grad=grad is not None)
-    at = torch.tensor(attn, dtype=torch.float64, requires_grad=grad is not None)
     B, S, M, D = v.shape
     _, Lq, _, L, K, _ = lo.shape
     acc = torch.zeros(B * M, D, Lq, dtype=torch.float64)
@@ -411,7 +408,20 @@ def grid_sample_reference(value, shapes, start, loc, attn, grad=None):
                             align_corners=False)                     # [B*M, D, Lq, K]
         wts = at[:, :, :, l].permute(0, 2, 1, 3).reshape(B * M, 1, Lq, K)
         acc = acc + (smp * wts).sum(-1)
-    out = acc.reshape(B, M, D, Lq).permute(0, 3, 1, 2).reshape(B, Lq, M * D)
+    return acc.reshape(B, M, D, Lq).permute(0, 3, 1, 2).reshape(B, Lq, M * D)
+
+
+def grid_sample_reference(value, shapes, start, loc, attn, grad=None):
+    """Forward (and, with ``grad``, autograd gradients) of :func:`grid_sample_core`
+    on float64 CPU tensors.  Test-only cross-check of the oracle."""
+    import torch
+
+    v = torch.tensor(value, dtype=torch.float64, requires_grad=grad is not None)
+    lo = torch.tensor(loc, dtype=torch.float64, requires_grad=grad is not None)
+    at = torch.tensor(attn, dtype=torch.float64, requires_grad=grad is not None)
+    B, S, M, D = v.shape
+    Lq = lo.shape[1]
+    out = grid_sample_core(v, lo, at, shapes, start)
     if grad is None:
         return out.detach().numpy()
     out.backward(torch.tensor(grad, dtype=torch.float64).reshape(B, Lq, M * D))

@@ -13,6 +13,7 @@ import pytest
 import oracle
 from oracle import build as oracle_build
 import oracle_pins
+import fused_pins
 
 SOURCE = open(oracle_build.SOURCE).read()
 
@@ -42,6 +43,21 @@ MUTANTS = [
     ("grad_value_column_major", "start + c.yi[j] * W + c.xi[i]", "start + (c.xi[i] * H + c.yi[j]) % (H * W)", False),
     ("grad_value_wrong_corner_weight", "A * wx[i] * wy[j] * gO;", "A * wx[1 - i] * wy[j] * gO;", False),
     ("grad_value_drops_lower_row", "if (c.xi[i] >= 0 && c.yi[j] >= 0)", "if (c.xi[i] >= 0 && c.yi[j] >= 0 && j == 0)", False),
+    # The step before the core (fused entry points).
+    ("fused_normaliser_swapped", "off[2 * p + 0], W,", "off[2 * p + 0], H,", False),
+    ("fused_reference_components_swapped", "form_location(r[0], R == 4 ? r[2] : 0.0",
+     "form_location(r[1], R == 4 ? r[2] : 0.0", False),
+    ("fused_box_half_dropped_f32", "t = t * 0.5f;", "t = t * 1.0f;", False),
+    ("fused_box_size_swapped", "R == 4 ? r[2] : 0.0, off[2 * p + 0]", "R == 4 ? r[3] : 0.0, off[2 * p + 0]", False),
+    ("fused_softmax_unnormalised", "A[g * LK + i] = exp(z[i] - zmax) / sum;", "A[g * LK + i] = exp(z[i] - zmax);", False),
+    ("fused_softmax_no_max", "sum += exp(z[i] - zmax);", "sum += exp(z[i]);", False),
+    ("fused_logit_grad_not_centred", "* (gA[g * LK + i] - s);", "* gA[g * LK + i];", False),
+    ("fused_offset_grad_unscaled", "grad_sampling_offsets[2 * p + c] = gl * dloc_doff;",
+     "grad_sampling_offsets[2 * p + c] = gl;", False),
+    ("fused_offset_grad_wrong_axis", "1.0 / (double)(c == 0 ? W : H)", "1.0 / (double)(c == 0 ? H : W)", False),
+    ("fused_box_size_grad_half_dropped", "gl * sampling_offsets[2 * p + c] * 0.5 / (double)K;",
+     "gl * sampling_offsets[2 * p + c] / (double)K;", False),
+    ("fused_reference_grad_dropped", "gr[c] += gl;", "gr[c] += 0.0 * gl;", False),
 ]
 
 
@@ -66,5 +82,5 @@ def test_mutant_is_caught(tmp_path, name, before, after, every):
     src.write_text(_mutate(before, after, every))
     lib = oracle_build.compile_source(str(src), str(tmp_path / f"libmutant_{name}.so"))
     orc = oracle.Oracle(lib)
-    failed = _failing_pins(orc, oracle_pins.FIRST_PRINCIPLES_PINS)
+    failed = _failing_pins(orc, oracle_pins.FIRST_PRINCIPLES_PINS + fused_pins.FIRST_PRINCIPLES_PINS)
     assert failed, f"mutant {name} passes every first-principles pin"
