@@ -125,7 +125,8 @@ msda_status msda_forward(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq,
  *                 are grouped by bilinear cell first, so each cell's corners are
  *                 read once and each grad_value row gets one atomic per cell
  *                 instead of one per point.  workspace == NULL selects the
- *                 scratch-free path (one atomic per point corner; slower).  A
+ *                 scratch-free path (one atomic per point corner), which
+ *                 measured faster on the encoder training workload.  A
  *                 workspace that is too small returns MSDA_ERR_WORKSPACE.  Two
  *                 calls that overlap on the GPU must not share a workspace.
  */
@@ -139,6 +140,73 @@ msda_status msda_backward(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq
                           float *grad_sampling_locations,
                           float *grad_attention_weights, void *workspace,
                           size_t workspace_bytes, void *stream);
+
+/*
+ * The op fused with the step before it: the sampling locations and attention
+ * weights are formed inside the kernels from the raw reference points,
+ * sampling offsets and attention logits, so neither is written to or read
+ * from memory.  "Deformable DETR模型解读（附源码+论文）",
+ * MultiScaleDeformableAttention.forward, and MSDeformAttn.forward on the
+ * phdsky.com notes of "Deformable DETR Deformable Transformers for End-to-End
+ * Object Detection":
+ *
+ *   A[b,q,m,:]  = softmax over the L*K logits attention_logits[b,q,m,:]
+ *   R == 2:  loc[b,q,m,l,k] = ref[b,q,l] + off[b,q,m,l,k] / (W_l, H_l)
+ *   R == 4:  loc[b,q,m,l,k] = ref[b,q,l,0:2] + off[b,q,m,l,k] / K * ref[b,q,l,2:4] * 0.5
+ *            (a box reference: centre x, y and size w, h, all normalised)
+ *
+ * then out = msda_forward(value, ..., loc, A).  loc is formed in float32 with
+ * each operation rounded once in the order written (the pages' float32
+ * tensors compute it so), so its pixel cell is the one they get.
+ *
+ *   reference_points    [B, Lq, L, R]        float32, R = 2 or 4 (else
+ *                                             MSDA_ERR_BAD_SHAPE)
+ *   sampling_offsets    [B, Lq, M, L, K, 2]  float32, 8-byte aligned; pixels of
+ *                                             level l for R == 2
+ *   attention_logits    [B, Lq, M, L * K]    float32
+ *   value, spatial_shapes, level_start_index, output, stream: as msda_forward.
+ */
+msda_status msda_fused_forward(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq,
+                               int64_t L, int64_t K, int64_t R, msda_dtype value_dtype,
+                               const void *value, const int64_t *spatial_shapes,
+                               const int64_t *level_start_index,
+                               const float *reference_points,
+                               const float *sampling_offsets,
+                               const float *attention_logits, void *output, void *stream);
+
+/*
+ * Backward of msda_fused_forward: the gradients of <grad_output, output> with
+ * respect to value, sampling_offsets, attention_logits and (optionally)
+ * reference_points.  With dloc, dA the core's gradients (msda_backward):
+ *   d off          = dloc / (W_l, H_l)                (R == 2)
+ *                  = dloc * ref[2:4] * 0.5 / K        (R == 4)
+ *   d logits_i     = A_i * (dA_i - sum_j A_j dA_j)    over each (b, q, m)
+ *   d ref[0:2]     = sum over (m, k) of dloc
+ *   d ref[2:4]     = sum over (m, k) of dloc * off * 0.5 / K   (R == 4)
+ * The derivative is that of the real-number formula (the float32 rounding of
+ * loc is not differentiated); the pages print no backward.
+ *
+ *   value_dtype must be MSDA_F32, D <= 128 (as msda_backward)
+ *   grad_value               [B, S, M, D]          overwritten (zeroed, then
+ *                                                  atomics; 16-byte aligned)
+ *   grad_sampling_offsets    [B, Lq, M, L, K, 2]   overwritten (8-byte aligned)
+ *   grad_attention_logits    [B, Lq, M, L * K]     overwritten
+ *   grad_reference_points    [B, Lq, L, R]         overwritten (zeroed, then
+ *                                                  atomics), or NULL to skip it
+ *                                                  (reference points are often
+ *                                                  detached)
+ * The scratch-free path of msda_backward is used; there is no workspace.
+ */
+msda_status msda_fused_backward(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq,
+                                int64_t L, int64_t K, int64_t R, msda_dtype value_dtype,
+                                const void *value, const int64_t *spatial_shapes,
+                                const int64_t *level_start_index,
+                                const float *reference_points,
+                                const float *sampling_offsets,
+                                const float *attention_logits, const float *grad_output,
+                                float *grad_value, float *grad_sampling_offsets,
+                                float *grad_attention_logits,
+                                float *grad_reference_points, void *stream);
 
 /*
  * Bytes of workspace msda_backward needs for these sizes (host only; no device

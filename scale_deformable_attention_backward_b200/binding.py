@@ -35,6 +35,8 @@ SIGNATURES = {
     "msda_backward": (_I32, [_I64] * 7 + [_I32] + [_VP] * 10 + [_SZ, _VP]),
     "msda_backward_workspace_size": (_I32, [_I64] * 7 + [ctypes.POINTER(_SZ)]),
     "msda_backward_noalloc": (_I32, [_I64] * 7 + [_I32] + [_VP] * 10),
+    "msda_fused_forward": (_I32, [_I64] * 8 + [_I32] + [_VP] * 8),
+    "msda_fused_backward": (_I32, [_I64] * 8 + [_I32] + [_VP] * 12),
     "msda_check_metadata": (_I32, [_I64, _I64, _VP, _VP]),
     "msda_status_string": (ctypes.c_char_p, [_I32]),
     "msda_version": (_I32, []),
@@ -253,3 +255,118 @@ def ms_deform_attn(value, spatial_shapes, level_start_index, sampling_locations,
     """Differentiable MSDeformAttn core (value float32 for the backward)."""
     return MSDeformAttnFunction.apply(value, spatial_shapes, level_start_index,
                                       sampling_locations, attention_weights, im2col_step)
+
+
+def _fused_dims(value, reference_points, sampling_offsets, attention_logits):
+    if value.dim() != 4:
+        raise ValueError("value must be [B, S, M, D]")
+    B, S, M, D = value.shape
+    if sampling_offsets.dim() != 6 or sampling_offsets.shape[-1] != 2:
+        raise ValueError("sampling_offsets must be [B, Lq, M, L, K, 2]")
+    Bq, Lq, Mq, L, K, _ = sampling_offsets.shape
+    if (Bq, Mq) != (B, M):
+        raise ValueError("sampling_offsets batch / head dims do not match value")
+    if reference_points.dim() != 4 or tuple(reference_points.shape[:3]) != (B, Lq, L):
+        raise ValueError("reference_points must be [B, Lq, L, R]")
+    R = reference_points.shape[3]
+    if tuple(attention_logits.shape) != (B, Lq, M, L * K):
+        raise ValueError("attention_logits must be [B, Lq, M, L*K]")
+    return B, S, M, D, Lq, L, K, R
+
+
+def fused_forward(value: torch.Tensor, spatial_shapes, level_start_index,
+                  reference_points: torch.Tensor, sampling_offsets: torch.Tensor,
+                  attention_logits: torch.Tensor,
+                  output: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """The op fed with raw reference points ([B, Lq, L, 2] or box [B, Lq, L, 4]),
+    sampling offsets and attention logits (``msda_fused_forward``): returns
+    ``[B, Lq, M*D]`` in value's dtype."""
+    dev = value.device
+    B, S, M, D, Lq, L, K, R = _fused_dims(value, reference_points, sampling_offsets,
+                                          attention_logits)
+    _require(value, "value", None, dev)
+    code = _value_code(value)
+    for t, name in ((reference_points, "reference_points"), (sampling_offsets, "sampling_offsets"),
+                    (attention_logits, "attention_logits")):
+        _require(t, name, torch.float32, dev)
+    ss, st = _metadata(spatial_shapes, level_start_index, S, dev)
+    if ss.shape != (L, 2) or st.shape != (L,):
+        raise ValueError("spatial_shapes must be [L, 2] and level_start_index [L]")
+    if output is None:
+        output = torch.empty((B, Lq, M * D), dtype=value.dtype, device=dev)
+    else:
+        _require(output, "output", value.dtype, dev)
+        if tuple(output.shape) != (B, Lq, M * D):
+            raise ValueError("output must be [B, Lq, M*D]")
+    with torch.cuda.device(dev):
+        stream = torch.cuda.current_stream(dev).cuda_stream
+        _check(library().msda_fused_forward(B, S, M, D, Lq, L, K, R, code, _ptr(value), _ptr(ss),
+                                            _ptr(st), _ptr(reference_points),
+                                            _ptr(sampling_offsets), _ptr(attention_logits),
+                                            _ptr(output), ctypes.c_void_p(stream)),
+               "msda_fused_forward")
+    return output
+
+
+def fused_backward(value: torch.Tensor, spatial_shapes, level_start_index,
+                   reference_points: torch.Tensor, sampling_offsets: torch.Tensor,
+                   attention_logits: torch.Tensor, grad_output: torch.Tensor,
+                   reference_grad: bool = True):
+    """Backward of :func:`fused_forward` (``msda_fused_backward``): returns
+    (grad_value, grad_sampling_offsets, grad_attention_logits,
+    grad_reference_points or None), all float32."""
+    dev = value.device
+    B, S, M, D, Lq, L, K, R = _fused_dims(value, reference_points, sampling_offsets,
+                                          attention_logits)
+    _require(value, "value", torch.float32, dev)
+    for t, name in ((reference_points, "reference_points"), (sampling_offsets, "sampling_offsets"),
+                    (attention_logits, "attention_logits"), (grad_output, "grad_output")):
+        _require(t, name, torch.float32, dev)
+    if tuple(grad_output.shape) != (B, Lq, M * D):
+        raise ValueError("grad_output must be [B, Lq, M*D]")
+    ss, st = _metadata(spatial_shapes, level_start_index, S, dev)
+    if ss.shape != (L, 2) or st.shape != (L,):
+        raise ValueError("spatial_shapes must be [L, 2] and level_start_index [L]")
+    gv = torch.empty((B, S, M, D), dtype=torch.float32, device=dev)
+    goff = torch.empty((B, Lq, M, L, K, 2), dtype=torch.float32, device=dev)
+    gz = torch.empty((B, Lq, M, L * K), dtype=torch.float32, device=dev)
+    gref = torch.empty((B, Lq, L, R), dtype=torch.float32, device=dev) if reference_grad else None
+    with torch.cuda.device(dev):
+        stream = torch.cuda.current_stream(dev).cuda_stream
+        _check(library().msda_fused_backward(B, S, M, D, Lq, L, K, R, MSDA_F32, _ptr(value),
+                                             _ptr(ss), _ptr(st), _ptr(reference_points),
+                                             _ptr(sampling_offsets), _ptr(attention_logits),
+                                             _ptr(grad_output), _ptr(gv), _ptr(goff), _ptr(gz),
+                                             _ptr(gref), ctypes.c_void_p(stream)),
+               "msda_fused_backward")
+    return gv, goff, gz, gref
+
+
+class MSDeformAttnFusedFunction(torch.autograd.Function):
+    """Autograd wrapper of the fused op: forward and backward run in libmsda.so."""
+
+    @staticmethod
+    def forward(ctx, value, spatial_shapes, level_start_index, reference_points,
+                sampling_offsets, attention_logits):
+        out = fused_forward(value, spatial_shapes, level_start_index, reference_points,
+                            sampling_offsets, attention_logits)
+        ctx.save_for_backward(value, reference_points, sampling_offsets, attention_logits)
+        ctx.meta = (spatial_shapes, level_start_index)
+        return out
+
+    @staticmethod
+    def backward(ctx, grad_output):
+        value, ref, off, logits = ctx.saved_tensors
+        ss, st = ctx.meta
+        gv, goff, gz, gref = fused_backward(value, ss, st, ref, off, logits,
+                                            grad_output.contiguous(),
+                                            reference_grad=ctx.needs_input_grad[3])
+        return gv, None, None, gref, goff, gz
+
+
+def ms_deform_attn_fused(value, spatial_shapes, level_start_index, reference_points,
+                         sampling_offsets, attention_logits):
+    """Differentiable op fed with raw reference points, offsets and logits."""
+    return MSDeformAttnFusedFunction.apply(value, spatial_shapes, level_start_index,
+                                           reference_points, sampling_offsets,
+                                           attention_logits)

@@ -190,6 +190,121 @@ msda_status msda_backward(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq
   return err == cudaSuccess ? MSDA_OK : MSDA_ERR_CUDA;
 }
 
+msda_status msda_fused_forward(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq,
+                               int64_t L, int64_t K, int64_t R, msda_dtype value_dtype,
+                               const void* value, const int64_t* spatial_shapes,
+                               const int64_t* level_start_index, const float* reference_points,
+                               const float* sampling_offsets, const float* attention_logits,
+                               void* output, void* stream) {
+  Common c;
+  msda_status st = check_common(B, S, M, D, Lq, L, K, &c);
+  if (st != MSDA_OK) return st;
+  if (R != 2 && R != 4) return MSDA_ERR_BAD_SHAPE;
+  if (value_dtype != MSDA_F32 && value_dtype != MSDA_BF16) return MSDA_ERR_UNSUPPORTED;
+  const int E = value_dtype == MSDA_F32 ? 4 : 8;
+  if (D % E != 0 || M > INT32_MAX || D > INT32_MAX) return MSDA_ERR_UNSUPPORTED;
+  if (c.out_elems == 0) return MSDA_OK;
+  if ((c.value_elems > 0 && value == nullptr) || spatial_shapes == nullptr ||
+      level_start_index == nullptr || reference_points == nullptr ||
+      sampling_offsets == nullptr || attention_logits == nullptr || output == nullptr)
+    return MSDA_ERR_NULL_POINTER;
+  if (!aligned(value, 16) || !aligned(output, 16) || !aligned(sampling_offsets, 8) ||
+      !aligned(reference_points, 4) || !aligned(attention_logits, 4) ||
+      !aligned(spatial_shapes, 8) || !aligned(level_start_index, 8))
+    return MSDA_ERR_MISALIGNED;
+  if (validate_env()) {
+    st = check_device_metadata(S, L, spatial_shapes, level_start_index);
+    if (st != MSDA_OK) return st;
+  }
+  msda::FusedArgs a{};
+  a.value = value;
+  a.spatial_shapes = spatial_shapes;
+  a.level_start_index = level_start_index;
+  a.reference_points = reference_points;
+  a.sampling_offsets = sampling_offsets;
+  a.attention_logits = attention_logits;
+  a.output = output;
+  a.S = S;
+  a.Lq = Lq;
+  a.M = static_cast<int>(M);
+  a.D = static_cast<int>(D);
+  a.L = static_cast<int>(L);
+  a.K = static_cast<int>(K);
+  a.R = static_cast<int>(R);
+  a.bf16 = value_dtype == MSDA_BF16;
+  const int64_t nvec = D / E;
+  a.lanes = pow2_at_least(nvec);
+  a.chunks = static_cast<int>((nvec + a.lanes - 1) / a.lanes);
+  a.groups = B * Lq * M * a.chunks;
+  return msda::launch_fused_forward(a, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? MSDA_OK
+             : MSDA_ERR_CUDA;
+}
+
+msda_status msda_fused_backward(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq,
+                                int64_t L, int64_t K, int64_t R, msda_dtype value_dtype,
+                                const void* value, const int64_t* spatial_shapes,
+                                const int64_t* level_start_index, const float* reference_points,
+                                const float* sampling_offsets, const float* attention_logits,
+                                const float* grad_output, float* grad_value,
+                                float* grad_sampling_offsets, float* grad_attention_logits,
+                                float* grad_reference_points, void* stream) {
+  Common c;
+  msda_status st = check_common(B, S, M, D, Lq, L, K, &c);
+  if (st != MSDA_OK) return st;
+  if (R != 2 && R != 4) return MSDA_ERR_BAD_SHAPE;
+  if (value_dtype != MSDA_F32) return MSDA_ERR_UNSUPPORTED;
+  if (D % 4 != 0 || D > 128 || M > INT32_MAX) return MSDA_ERR_UNSUPPORTED;
+  int64_t ref_elems = 0;
+  if (!product_ok({B, Lq, L, R}, &ref_elems)) return MSDA_ERR_BAD_SHAPE;
+  if (c.value_elems == 0 && c.out_elems == 0) return MSDA_OK;
+  if (c.value_elems > 0 && grad_value == nullptr) return MSDA_ERR_NULL_POINTER;
+  if (!aligned(grad_value, 16) || !aligned(grad_reference_points, 4)) return MSDA_ERR_MISALIGNED;
+  const bool work = c.out_elems > 0;
+  if (work && (value == nullptr || spatial_shapes == nullptr || level_start_index == nullptr ||
+               reference_points == nullptr || sampling_offsets == nullptr ||
+               attention_logits == nullptr || grad_output == nullptr ||
+               grad_sampling_offsets == nullptr || grad_attention_logits == nullptr))
+    return MSDA_ERR_NULL_POINTER;
+  if (work && (!aligned(value, 16) || !aligned(grad_output, 16) ||
+               !aligned(sampling_offsets, 8) || !aligned(grad_sampling_offsets, 8) ||
+               !aligned(reference_points, 4) || !aligned(attention_logits, 4) ||
+               !aligned(grad_attention_logits, 4) || !aligned(spatial_shapes, 8) ||
+               !aligned(level_start_index, 8)))
+    return MSDA_ERR_MISALIGNED;
+  if (work && validate_env()) {
+    st = check_device_metadata(S, L, spatial_shapes, level_start_index);
+    if (st != MSDA_OK) return st;
+  }
+  msda::FusedArgs a{};
+  a.value = value;
+  a.spatial_shapes = spatial_shapes;
+  a.level_start_index = level_start_index;
+  a.reference_points = reference_points;
+  a.sampling_offsets = sampling_offsets;
+  a.attention_logits = attention_logits;
+  a.grad_output = grad_output;
+  a.grad_value = grad_value;
+  a.grad_sampling_offsets = grad_sampling_offsets;
+  a.grad_attention_logits = grad_attention_logits;
+  a.grad_reference_points = work ? grad_reference_points : nullptr;
+  a.S = S;
+  a.Lq = Lq;
+  a.M = static_cast<int>(M);
+  a.D = static_cast<int>(D);
+  a.L = static_cast<int>(L);
+  a.K = static_cast<int>(K);
+  a.R = static_cast<int>(R);
+  a.lanes = pow2_at_least(D / 4);
+  a.chunks = 1;
+  a.groups = work ? B * Lq * M : 0;
+  a.value_elements = c.value_elems;
+  a.reference_elements = ref_elems;
+  return msda::launch_fused_backward(a, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? MSDA_OK
+             : MSDA_ERR_CUDA;
+}
+
 msda_status msda_backward_workspace_size(int64_t B, int64_t S, int64_t M, int64_t D,
                                          int64_t Lq, int64_t L, int64_t K, size_t* bytes) {
   if (bytes == nullptr) return MSDA_ERR_NULL_POINTER;

@@ -32,6 +32,7 @@
 // per unit suffices.  (Head-major tiles and contiguous per-block tile ranges,
 // which favour L1 reuse, measured slower on the encoder workload.)
 #include "msda_device.cuh"
+#include "msda_gather.cuh"
 #include "msda_launch.h"
 
 namespace msda {
@@ -40,81 +41,6 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kChunkPoints = 512;
-
-// The setup of one point: element offsets of its four corners relative to the
-// (b, m, channel) base pointer, -1 for a corner outside the map, in the order
-// V(x0,y0), V(x0+1,y0), V(x0,y0+1), V(x0+1,y0+1); and the four weights
-// A * bilinear in the same order.
-struct PointSetup {
-  int4 off;
-  float4 w;
-};
-
-__device__ __forceinline__ PointSetup setup_point(float lx, float ly, float a, int H, int W,
-                                                  long long start, int MD) {
-  const Cell c = locate(lx, ly, H, W);
-  const float hx = 1.0f - c.fx, hy = 1.0f - c.fy;
-  PointSetup s;
-  s.w = make_float4(a * hx * hy, a * c.fx * hy, a * hx * c.fy, a * c.fx * c.fy);
-  const int base = static_cast<int>(start + static_cast<long long>(c.y0) * W + c.x0);
-  // Offsets are formed only for corners inside the map, where 0 <= pixel < S and
-  // pixel * M * D < 2^31 (checked by the C ABI).
-  s.off.x = (c.vx0 && c.vy0) ? base * MD : -1;
-  s.off.y = (c.vx1 && c.vy0) ? (base + 1) * MD : -1;
-  s.off.z = (c.vx0 && c.vy1) ? (base + W) * MD : -1;
-  s.off.w = (c.vx1 && c.vy1) ? (base + W + 1) * MD : -1;
-  // A point with no corner in the map adds A * 0 to the output, which is NaN when
-  // its weights are not finite (a non-finite location or weight).  Such a point
-  // reads the level's first pixel with a NaN weight, so the NaN reaches the sum.
-  if ((s.off.x & s.off.y & s.off.z & s.off.w) < 0 && W > 0 &&
-      !isfinite(s.w.x + s.w.y + s.w.z + s.w.w)) {
-    s.off.x = static_cast<int>(start) * MD;
-    s.w.x = __int_as_float(0x7fffffff);
-  }
-  return s;
-}
-
-template <typename T>
-struct Corner;
-
-template <>
-struct Corner<float> {
-  static constexpr int N = 4;
-  // acc += w * value[0..3] for one corner inside the map.
-  __device__ __forceinline__ static void accumulate(const float* p, float w, float2 (&acc)[2]) {
-    const float4 v = __ldg(reinterpret_cast<const float4*>(p));
-    const float2 ww = make_float2(w, w);
-    acc[0] = fma2(ww, make_float2(v.x, v.y), acc[0]);
-    acc[1] = fma2(ww, make_float2(v.z, v.w), acc[1]);
-  }
-  __device__ __forceinline__ static void store(float* p, const float2 (&acc)[2]) {
-    *reinterpret_cast<float4*>(p) = make_float4(acc[0].x, acc[0].y, acc[1].x, acc[1].y);
-  }
-};
-
-template <>
-struct Corner<__nv_bfloat16> {
-  static constexpr int N = 8;
-  __device__ __forceinline__ static void accumulate(const __nv_bfloat16* p, float w,
-                                                    float2 (&acc)[4]) {
-    const uint4 r = __ldg(reinterpret_cast<const uint4*>(p));
-    const unsigned u[4] = {r.x, r.y, r.z, r.w};
-    const float2 ww = make_float2(w, w);
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-      acc[i] = fma2(ww, make_float2(__uint_as_float(u[i] << 16),
-                                    __uint_as_float(u[i] & 0xffff0000u)), acc[i]);
-  }
-  __device__ __forceinline__ static void store(__nv_bfloat16* p, const float2 (&acc)[4]) {
-    unsigned u[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const __nv_bfloat162 h = __floats2bfloat162_rn(acc[i].x, acc[i].y);
-      u[i] = *reinterpret_cast<const unsigned*>(&h);
-    }
-    *reinterpret_cast<uint4*>(p) = make_uint4(u[0], u[1], u[2], u[3]);
-  }
-};
 
 }  // namespace
 

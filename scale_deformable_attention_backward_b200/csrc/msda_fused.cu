@@ -1,0 +1,399 @@
+// msda_fused.cu -- the MSDeformAttn core fused with the step before it: the
+// sampling locations and attention weights are formed in registers from the
+// raw reference points, sampling offsets and attention logits (sm_100a).
+//
+// The step before the core ("Deformable DETR模型解读（附源码+论文）",
+// MultiScaleDeformableAttention.forward, and MSDeformAttn.forward on the
+// phdsky.com notes of "Deformable DETR Deformable Transformers for End-to-End
+// Object Detection"):
+//   A[b,q,m,:]   = softmax over the L*K logits of (b, q, m)
+//   R = 2:  loc  = ref[b,q,l] + off[b,q,m,l,k] / (W_l, H_l)
+//   R = 4:  loc  = ref[b,q,l,0:2] + off[b,q,m,l,k] / K * ref[b,q,l,2:4] * 0.5
+// The location is formed in float32 with every operation rounded once in that
+// order (the pages' float32 tensors compute it so), which keeps the floor of
+// the pixel coordinate identical to theirs; the core then runs as in
+// msda_forward.cu / msda_backward.cu.
+//
+// Backward (the derivative of the real-number formula; the pages print none):
+//   d off   = d loc / (W_l, H_l)                      (R = 2)
+//           = d loc * ref[2:4] * 0.5 / K              (R = 4)
+//   d ref   = sum over (m, k) of d loc, and for R = 4 also
+//     d ref[2:4] = sum over (m, k) of d loc * off * 0.5 / K
+//   d z_i   = A_i (dA_i - sum_j A_j dA_j)             over the (b, q, m) group
+// where d loc and dA are the core's grad_sampling_locations and
+// grad_attention_weights.
+#include <cmath>
+
+#include "msda_device.cuh"
+#include "msda_gather.cuh"
+#include "msda_launch.h"
+
+namespace msda {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kChunkPoints = 512;
+
+// The sampling location of one point, formed as the pages' float32 tensors do.
+__device__ __forceinline__ float2 fused_location(const float* __restrict__ ref, float2 off, int R,
+                                                 int W, int H, int K) {
+  if (R == 2)
+    return make_float2(__fadd_rn(__ldg(ref + 0), __fdiv_rn(off.x, static_cast<float>(W))),
+                       __fadd_rn(__ldg(ref + 1), __fdiv_rn(off.y, static_cast<float>(H))));
+  const float fk = static_cast<float>(K);
+  const float tx = __fmul_rn(__fmul_rn(__fdiv_rn(off.x, fk), __ldg(ref + 2)), 0.5f);
+  const float ty = __fmul_rn(__fmul_rn(__fdiv_rn(off.y, fk), __ldg(ref + 3)), 0.5f);
+  return make_float2(__fadd_rn(__ldg(ref + 0), tx), __fadd_rn(__ldg(ref + 1), ty));
+}
+
+// A maximum that keeps NaN, so that a NaN logit makes the whole group's
+// weights NaN (as the softmax does).
+__device__ __forceinline__ float nan_max(float a, float b) { return (b > a || b != b) ? b : a; }
+
+// (max, 1 / sum exp(z - max)) over the LK logits of one group, computed by the
+// LANES lanes of a sub-warp (every lane of the warp takes part).
+template <int LANES>
+__device__ __forceinline__ float2 softmax_norm(const float* __restrict__ z, int LK, int lane) {
+  float m = -INFINITY;
+  for (int i = lane; i < LK; i += LANES) m = nan_max(m, __ldg(z + i));
+#pragma unroll
+  for (int o = LANES / 2; o > 0; o >>= 1) m = nan_max(m, __shfl_xor_sync(kFullMask, m, o, LANES));
+  float s = 0.0f;
+  for (int i = lane; i < LK; i += LANES) s += expf(__ldg(z + i) - m);
+#pragma unroll
+  for (int o = LANES / 2; o > 0; o >>= 1) s += __shfl_xor_sync(kFullMask, s, o, LANES);
+  return make_float2(m, 1.0f / s);
+}
+
+// Forward: the two phases of msda_forward.cu (per-point setup into a swizzled
+// shared table, then sub-warp gathers), preceded per tile by the softmax
+// normaliser of each group.
+template <typename T, int LANES>
+__global__ void __launch_bounds__(kThreads)
+fused_forward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial_shapes,
+                     const int64_t* __restrict__ level_start_index,
+                     const float* __restrict__ reference_points,
+                     const float* __restrict__ sampling_offsets,
+                     const float* __restrict__ attention_logits, T* __restrict__ output,
+                     long long S, int M, int D, long long Lq, int L, int K, int R, int chunks,
+                     long long groups) {
+  using C = Corner<T>;
+  constexpr int E = C::N;
+  constexpr int G = kThreads / LANES;
+  constexpr int PC = kChunkPoints / G;
+  constexpr int PER = kChunkPoints / kThreads;
+  static_assert(G >= 8, "the shared-memory swizzle needs at least 8 groups per block");
+  __shared__ Levels lv;
+  __shared__ int4 s_off[kChunkPoints];
+  __shared__ float4 s_w[kChunkPoints];
+  __shared__ float2 s_norm[G];
+  stage_levels(lv, spatial_shapes, level_start_index, L, S);
+
+  const int lane = threadIdx.x % LANES;
+  const int gi = threadIdx.x / LANES;
+  const int LK = L * K;
+  const int MD = M * D;
+  const long long tiles = (groups + G - 1) / G;
+
+  for (long long tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+    const long long g_raw = tile * G + gi;
+    const bool active = g_raw < groups;
+    const Group grp = decompose(active ? g_raw : groups - 1, chunks, M, Lq);
+    const float2 nz = softmax_norm<LANES>(attention_logits + grp.bqm * LK, LK, lane);
+    if (lane == 0) s_norm[gi] = nz;
+    __syncthreads();
+
+    const int ch = (grp.chunk * LANES + lane) * E;
+    const bool lane_on = active && ch < D;
+    const T* vbase = value + (grp.b * S * M + grp.m) * static_cast<long long>(D) + ch;
+    float2 acc[E / 2];
+#pragma unroll
+    for (int e = 0; e < E / 2; ++e) acc[e] = make_float2(0.0f, 0.0f);
+
+    for (int p0 = 0; p0 < LK; p0 += PC) {
+      const int pc = min(PC, LK - p0);
+#pragma unroll
+      for (int r = 0; r < PER; ++r) {
+        const int t = threadIdx.x + r * kThreads;
+        const int tg = t / PC, tj = t % PC;
+        const long long g = tile * G + tg;
+        if (tj < pc && g < groups) {
+          const long long bqm = g / chunks;
+          const long long bq = bqm / M;
+          const int i = p0 + tj;
+          const int l = i / K;
+          const long long p = bqm * LK + i;
+          const float2 off = __ldg(reinterpret_cast<const float2*>(sampling_offsets) + p);
+          const float2 loc = fused_location(reference_points + (bq * L + l) * R, off, R,
+                                            lv.W[l], lv.H[l], K);
+          const float2 n = s_norm[tg];
+          const float a = expf(__ldg(attention_logits + p) - n.x) * n.y;
+          const PointSetup su = setup_point(loc.x, loc.y, a, lv.H[l], lv.W[l], lv.start[l], MD);
+          const int slot = tj * G + (tg ^ (tj & 7));
+          s_off[slot] = su.off;
+          s_w[slot] = su.w;
+        }
+      }
+      __syncthreads();
+      if (lane_on) {
+#pragma unroll 4
+        for (int j = 0; j < pc; ++j) {
+          const int slot = j * G + (gi ^ (j & 7));
+          const int4 o = s_off[slot];
+          const float4 w = s_w[slot];
+          if (o.x >= 0) C::accumulate(vbase + o.x, w.x, acc);
+          if (o.y >= 0) C::accumulate(vbase + o.y, w.y, acc);
+          if (o.z >= 0) C::accumulate(vbase + o.z, w.z, acc);
+          if (o.w >= 0) C::accumulate(vbase + o.w, w.w, acc);
+        }
+      }
+      __syncthreads();  // the table and s_norm are rewritten next
+    }
+    if (lane_on) C::store(output + grp.bq * MD + static_cast<long long>(grp.m) * D + ch, acc);
+  }
+}
+
+// Backward: the scratch-free backward of msda_backward.cu (a sub-warp per
+// (b, q, m), four corner gathers and one 16-byte vector atomic per lane and
+// corner for each point) with the locations and weights formed from the raw
+// inputs, and the chain rule through them applied per point.  grad_logits
+// holds dA until the group's sum_j A_j dA_j is known, then d z.
+template <int LANES>
+__global__ void __launch_bounds__(kThreads)
+fused_backward_kernel(const float* __restrict__ value, const int64_t* __restrict__ spatial_shapes,
+                      const int64_t* __restrict__ level_start_index,
+                      const float* __restrict__ reference_points,
+                      const float* __restrict__ sampling_offsets,
+                      const float* __restrict__ attention_logits,
+                      const float* __restrict__ grad_output, float* __restrict__ grad_value,
+                      float* __restrict__ grad_offsets, float* __restrict__ grad_logits,
+                      float* __restrict__ grad_reference, long long S, int M, int D,
+                      long long Lq, int L, int K, int R, long long groups) {
+  using V = Vec<float>;
+  constexpr int E = V::N;
+  __shared__ Levels lv;
+  stage_levels(lv, spatial_shapes, level_start_index, L, S);
+
+  const int lane = threadIdx.x % LANES;
+  const int groups_per_block = blockDim.x / LANES;
+  const int LK = L * K;
+  const long long MD = static_cast<long long>(M) * D;
+  const float half_over_k = 0.5f / static_cast<float>(K);
+
+  for (long long g0 = static_cast<long long>(blockIdx.x) * groups_per_block; g0 < groups;
+       g0 += static_cast<long long>(gridDim.x) * groups_per_block) {
+    const long long g_raw = g0 + threadIdx.x / LANES;
+    const bool active = g_raw < groups;
+    const Group grp = decompose(active ? g_raw : groups - 1, 1, M, Lq);
+    const int ch = lane * E;
+    const bool lane_on = active && ch < D;
+    const long long vofs = (grp.b * S * M + grp.m) * static_cast<long long>(D) + ch;
+    const float* vbase = value + vofs;
+    float* gvbase = grad_value + vofs;
+    const float* zg = attention_logits + grp.bqm * LK;
+    const float2 nz = softmax_norm<LANES>(zg, LK, lane);
+
+    float go[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) go[e] = 0.0f;
+    if (lane_on) V::load(grad_output + grp.bq * MD + static_cast<long long>(grp.m) * D + ch, go);
+
+    float sum_adA = 0.0f;  // this lane's share of sum_j A_j dA_j
+    int l = 0, k = 0;
+    int H = lv.H[0], W = lv.W[0];
+    long long start = lv.start[0];
+    for (int p0 = 0; p0 < LK; p0 += LANES) {
+      const int pj = p0 + lane;
+      const int lj = pj / K;
+      float2 xy = make_float2(0.0f, 0.0f), offj = make_float2(0.0f, 0.0f);
+      float aj = 0.0f;
+      if (pj < LK) {
+        offj = __ldg(reinterpret_cast<const float2*>(sampling_offsets) + grp.bqm * LK + pj);
+        xy = fused_location(reference_points + (grp.bq * L + lj) * R, offj, R, lv.W[lj],
+                            lv.H[lj], K);
+        aj = expf(__ldg(zg + pj) - nz.x) * nz.y;
+      }
+      float keep_attn = 0.0f, keep_x = 0.0f, keep_y = 0.0f;
+      const int n = min(LANES, LK - p0);
+      for (int j = 0; j < n; ++j) {
+        const float lx = __shfl_sync(kFullMask, xy.x, j, LANES);
+        const float ly = __shfl_sync(kFullMask, xy.y, j, LANES);
+        const float a = __shfl_sync(kFullMask, aj, j, LANES);
+        const Cell c = locate(lx, ly, H, W);
+        const float hx = 1.0f - c.fx, hy = 1.0f - c.fy;
+        const long long row = static_cast<long long>(W) * MD;
+        const long long off = (start + static_cast<long long>(c.y0) * W + c.x0) * MD;
+        const bool v00 = c.vx0 && c.vy0, v10 = c.vx1 && c.vy0;
+        const bool v01 = c.vx0 && c.vy1, v11 = c.vx1 && c.vy1;
+        float s_attn = 0.0f, s_x = 0.0f, s_y = 0.0f;
+        if (lane_on) {
+          float q00[E], q10[E], q01[E], q11[E];
+#pragma unroll
+          for (int e = 0; e < E; ++e) q00[e] = q10[e] = q01[e] = q11[e] = 0.0f;
+          if (v00) V::load(vbase + off, q00);
+          if (v10) V::load(vbase + off + MD, q10);
+          if (v01) V::load(vbase + off + row, q01);
+          if (v11) V::load(vbase + off + row + MD, q11);
+#pragma unroll
+          for (int e = 0; e < E; ++e) {
+            const float top = fmaf(c.fx, q10[e], hx * q00[e]);
+            const float bot = fmaf(c.fx, q11[e], hx * q01[e]);
+            s_attn = fmaf(go[e], fmaf(c.fy, bot, hy * top), s_attn);
+            s_x = fmaf(go[e], fmaf(c.fy, q11[e] - q01[e], hy * (q10[e] - q00[e])), s_x);
+            s_y = fmaf(go[e], fmaf(c.fx, q11[e] - q10[e], hx * (q01[e] - q00[e])), s_y);
+          }
+          const float w00 = a * hx * hy, w10 = a * c.fx * hy;
+          const float w01 = a * hx * c.fy, w11 = a * c.fx * c.fy;
+          if (v00) atomicAdd(reinterpret_cast<float4*>(gvbase + off),
+                             make_float4(w00 * go[0], w00 * go[1], w00 * go[2], w00 * go[3]));
+          if (v10) atomicAdd(reinterpret_cast<float4*>(gvbase + off + MD),
+                             make_float4(w10 * go[0], w10 * go[1], w10 * go[2], w10 * go[3]));
+          if (v01) atomicAdd(reinterpret_cast<float4*>(gvbase + off + row),
+                             make_float4(w01 * go[0], w01 * go[1], w01 * go[2], w01 * go[3]));
+          if (v11) atomicAdd(reinterpret_cast<float4*>(gvbase + off + row + MD),
+                             make_float4(w11 * go[0], w11 * go[1], w11 * go[2], w11 * go[3]));
+        }
+#pragma unroll
+        for (int o = LANES / 2; o > 0; o >>= 1) {
+          s_attn += __shfl_xor_sync(kFullMask, s_attn, o, LANES);
+          s_x += __shfl_xor_sync(kFullMask, s_x, o, LANES);
+          s_y += __shfl_xor_sync(kFullMask, s_y, o, LANES);
+        }
+        if (lane == j) {
+          keep_attn = s_attn;
+          keep_x = a * s_x;  // grad_loc.x / W of this point
+          keep_y = a * s_y;  // grad_loc.y / H
+        }
+        if (++k == K) {
+          k = 0;
+          if (++l < L) {
+            H = lv.H[l];
+            W = lv.W[l];
+            start = lv.start[l];
+          }
+        }
+      }
+      if (active && pj < LK) {
+        const long long p = grp.bqm * LK + pj;
+        sum_adA = fmaf(aj, keep_attn, sum_adA);
+        grad_logits[p] = keep_attn;  // dA for now
+        const float Wj = static_cast<float>(lv.W[lj]), Hj = static_cast<float>(lv.H[lj]);
+        const float gx = keep_x * Wj, gy = keep_y * Hj;  // grad_loc
+        float2 goff;
+        if (R == 2) {
+          goff = make_float2(keep_x, keep_y);
+        } else {
+          const float* rp = reference_points + (grp.bq * L + lj) * R;
+          goff = make_float2(gx * __ldg(rp + 2) * half_over_k, gy * __ldg(rp + 3) * half_over_k);
+        }
+        reinterpret_cast<float2*>(grad_offsets)[p] = goff;
+        if (grad_reference != nullptr) {
+          float* gr = grad_reference + (grp.bq * L + lj) * R;
+          atomicAdd(gr + 0, gx);
+          atomicAdd(gr + 1, gy);
+          if (R == 4) {
+            atomicAdd(gr + 2, gx * offj.x * half_over_k);
+            atomicAdd(gr + 3, gy * offj.y * half_over_k);
+          }
+        }
+      }
+    }
+    // Softmax Jacobian: d z_j = A_j (dA_j - sum_i A_i dA_i).  Each lane revisits
+    // the points it wrote.
+#pragma unroll
+    for (int o = LANES / 2; o > 0; o >>= 1) sum_adA += __shfl_xor_sync(kFullMask, sum_adA, o, LANES);
+    if (active) {
+      for (int pj = lane; pj < LK; pj += LANES) {
+        const long long p = grp.bqm * LK + pj;
+        const float aj = expf(__ldg(zg + pj) - nz.x) * nz.y;
+        grad_logits[p] = aj * (grad_logits[p] - sum_adA);
+      }
+    }
+  }
+}
+
+template <typename T, int LANES>
+long long resident_forward_blocks() {
+  static long long cached[64] = {};
+  int dev = 0, sms = 0, per_sm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev >= 0 && dev < 64 && cached[dev] > 0) return cached[dev];
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fused_forward_kernel<T, LANES>,
+                                                    kThreads, 0) != cudaSuccess ||
+      sms <= 0 || per_sm <= 0)
+    return 148;
+  const long long n = static_cast<long long>(sms) * per_sm;
+  if (dev >= 0 && dev < 64) cached[dev] = n;
+  return n;
+}
+
+template <typename T, int LANES>
+cudaError_t launch_fused_forward_t(const FusedArgs& a, cudaStream_t stream) {
+  constexpr int G = kThreads / LANES;
+  const long long tiles = (a.groups + G - 1) / G;
+  long long blocks = resident_forward_blocks<T, LANES>();
+  if (blocks > tiles) blocks = tiles;
+  fused_forward_kernel<T, LANES><<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(
+      static_cast<const T*>(a.value), a.spatial_shapes, a.level_start_index, a.reference_points,
+      a.sampling_offsets, a.attention_logits, static_cast<T*>(a.output), a.S, a.M, a.D, a.Lq,
+      a.L, a.K, a.R, a.chunks, a.groups);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t fused_forward_lanes(const FusedArgs& a, cudaStream_t stream) {
+  switch (a.lanes) {
+    case 1: return launch_fused_forward_t<T, 1>(a, stream);
+    case 2: return launch_fused_forward_t<T, 2>(a, stream);
+    case 4: return launch_fused_forward_t<T, 4>(a, stream);
+    case 8: return launch_fused_forward_t<T, 8>(a, stream);
+    case 16: return launch_fused_forward_t<T, 16>(a, stream);
+    case 32: return launch_fused_forward_t<T, 32>(a, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <int LANES>
+cudaError_t launch_fused_backward_t(const FusedArgs& a, cudaStream_t stream) {
+  const long long per_block = kThreads / LANES;
+  long long blocks = (a.groups + per_block - 1) / per_block;
+  if (blocks > (1ll << 30)) blocks = 1ll << 30;
+  fused_backward_kernel<LANES><<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(
+      static_cast<const float*>(a.value), a.spatial_shapes, a.level_start_index,
+      a.reference_points, a.sampling_offsets, a.attention_logits, a.grad_output, a.grad_value,
+      a.grad_sampling_offsets, a.grad_attention_logits, a.grad_reference_points, a.S, a.M, a.D,
+      a.Lq, a.L, a.K, a.R, a.groups);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fused_forward(const FusedArgs& a, cudaStream_t stream) {
+  if (a.groups == 0) return cudaSuccess;
+  return a.bf16 ? fused_forward_lanes<__nv_bfloat16>(a, stream)
+                : fused_forward_lanes<float>(a, stream);
+}
+
+cudaError_t launch_fused_backward(const FusedArgs& a, cudaStream_t stream) {
+  cudaError_t err = launch_zero(a.grad_value, a.value_elements, stream);
+  if (err != cudaSuccess) return err;
+  if (a.grad_reference_points != nullptr && a.reference_elements > 0) {
+    err = cudaMemsetAsync(a.grad_reference_points, 0,
+                          sizeof(float) * static_cast<size_t>(a.reference_elements), stream);
+    if (err != cudaSuccess) return err;
+  }
+  if (a.groups == 0) return cudaSuccess;
+  switch (a.lanes) {
+    case 1: return launch_fused_backward_t<1>(a, stream);
+    case 2: return launch_fused_backward_t<2>(a, stream);
+    case 4: return launch_fused_backward_t<4>(a, stream);
+    case 8: return launch_fused_backward_t<8>(a, stream);
+    case 16: return launch_fused_backward_t<16>(a, stream);
+    case 32: return launch_fused_backward_t<32>(a, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace msda

@@ -43,6 +43,33 @@ struct BackwardArgs {
   long long value_elements;  // B * S * M * D (grad_value is zeroed first)
 };
 
+// The core fed with raw reference points, offsets and logits (msda_fused.cu).
+struct FusedArgs {
+  const void* value;
+  const int64_t* spatial_shapes;
+  const int64_t* level_start_index;
+  const float* reference_points;   // [B, Lq, L, R]
+  const float* sampling_offsets;   // [B, Lq, M, L, K, 2]
+  const float* attention_logits;   // [B, Lq, M, L * K]
+  long long S, Lq;
+  int M, D, L, K, R;
+  bool bf16;
+  int lanes;                       // forward: as ForwardArgs; backward: D <= 4 * lanes
+  int chunks;                      // forward channel chunks per (b, q, m); 1 for the backward
+  long long groups;                // B * Lq * M * chunks
+  void* output;                    // forward
+  const float* grad_output;        // backward
+  float* grad_value;
+  float* grad_sampling_offsets;
+  float* grad_attention_logits;
+  float* grad_reference_points;    // may be null: not computed
+  long long value_elements;        // B * S * M * D
+  long long reference_elements;    // B * Lq * L * R
+};
+
+cudaError_t launch_fused_forward(const FusedArgs& a, cudaStream_t stream);
+cudaError_t launch_fused_backward(const FusedArgs& a, cudaStream_t stream);
+
 // Scratch layout of the cell-sorted backward (msda_backward_sorted.cu).
 struct SortedLayout {
   long long cells_per_bm;  // keys per (b, m): bound on sum_l (H_l + 1)(W_l + 1) from S, L

@@ -51,6 +51,7 @@ class Config:
     K: int
     shapes: Tuple[Tuple[int, int], ...]
     recipe: str            # "uniform" | "encoder" | "decoder" | "encoder_valid_ratio"
+                           # | "decoder_box"
     dtype: str             # value dtype: "f32" | "bf16"
     backward: bool         # whether the workload includes the training backward
     Lq: Optional[int] = None   # None: one query per value token (self-attention)
@@ -98,6 +99,12 @@ CONFIGS: Dict[str, Config] = {
         recipe="encoder", dtype="f32", backward=True,
         description="encoder training fp32 fwd+bwd: B=4 M=8 D=32 K=4 L=4, "
                     "levels (100,150),(50,75),(25,38),(13,19), S=Lq=19947"),
+    "decoder_box_train_fp32": Config(
+        "decoder_box_train_fp32", B=2, M=8, D=32, K=4, shapes=tuple(ENCODER_800x1200),
+        recipe="decoder_box", dtype="f32", backward=True, Lq=300,
+        description="decoder cross-attention with box reference points fp32 fwd+bwd: B=2 "
+                    "Lq=300 M=8 D=32 K=4 L=4 over the 800x1200 encoder levels; box centre "
+                    "U[0.05,0.95]^2, size U[0.05,0.5]^2, offsets N(0,1)*K/2 box units")
 }
 
 
@@ -179,6 +186,17 @@ def _reference_points(cfg: Config, rng: np.random.Generator, Lq: int) -> np.ndar
     raise ValueError(cfg.recipe)
 
 
+def _box_references(rng: np.random.Generator, B: int, Lq: int, L: int) -> np.ndarray:
+    """[B, Lq, L, 4] box reference points (centre x, y, size w, h; normalised),
+    one box per query shared by the levels, as a box-refining decoder layer feeds
+    them ("Deformable DETR模型解读", MultiScaleDeformableAttention.forward, the
+    4-component branch)."""
+    centre = rng.uniform(0.05, 0.95, size=(B, Lq, 2))
+    size = rng.uniform(0.05, 0.5, size=(B, Lq, 2))
+    box = np.concatenate([centre, size], -1)
+    return np.broadcast_to(box[:, :, None, :], (B, Lq, L, 4)).copy()
+
+
 def make_inputs(cfg: Config, seed: int = 0, with_grad: Optional[bool] = None) -> Inputs:
     """Draw one seeded set of inputs for ``cfg``."""
     rng = np.random.default_rng(seed)
@@ -196,6 +214,10 @@ def make_inputs(cfg: Config, seed: int = 0, with_grad: Optional[bool] = None) ->
 
     if cfg.recipe == "uniform":
         loc = rng.uniform(-0.1, 1.1, size=(B, Lq, M, L, K, 2))
+    elif cfg.recipe == "decoder_box":
+        box = _box_references(rng, B, Lq, L)                            # [B, Lq, L, 4]
+        off = rng.standard_normal((B, Lq, M, L, K, 2)) * (K / 2.0)
+        loc = box[:, :, None, :, None, :2] + off / K * box[:, :, None, :, None, 2:] * 0.5
     else:
         ref = _reference_points(cfg, rng, Lq)                        # [B, Lq, L, 2]
         if cfg.recipe == "decoder":
@@ -224,6 +246,77 @@ def make_inputs(cfg: Config, seed: int = 0, with_grad: Optional[bool] = None) ->
         attention_weights=np.ascontiguousarray(attn.astype(np.float32)),
         grad_output=grad,
     )
+
+
+@dataclasses.dataclass
+class FusedInputs:
+    """Host arrays for one call of the fused op (raw reference points, offsets and
+    logits instead of locations and weights)."""
+
+    config: Config
+    value: np.ndarray                  # [B,S,M,D] float32 (bf16-representable for bf16)
+    value_bf16_bits: Optional[np.ndarray]
+    spatial_shapes: np.ndarray         # [L,2] int64 (H, W)
+    level_start_index: np.ndarray      # [L] int64
+    reference_points: np.ndarray       # [B,Lq,L,R] float32, R = 2 or 4 (boxes)
+    sampling_offsets: np.ndarray       # [B,Lq,M,L,K,2] float32
+    attention_logits: np.ndarray       # [B,Lq,M,L*K] float32
+    grad_output: Optional[np.ndarray]  # [B,Lq,M*D] float32, backward workloads only
+
+
+def make_fused_inputs(cfg: Config, seed: int = 0,
+                      with_grad: Optional[bool] = None) -> FusedInputs:
+    """The raw inputs behind :func:`make_inputs` (same draws in the same order):
+    reference points, offsets (pixels of level l for 2-component references,
+    box units for boxes) and the softmax logits.  For the "uniform" recipe the
+    2-component reference points are drawn U[-0.1, 1.1]^2 and the offsets
+    N(0, 1) pixels."""
+    rng = np.random.default_rng(seed)
+    B, M, D, K, L = cfg.B, cfg.M, cfg.D, cfg.K, cfg.L
+    shapes = [tuple(s) for s in cfg.shapes]
+    ss, start = level_metadata(shapes)
+    S, Lq = cfg.S, cfg.queries
+    wh = ss[:, ::-1].astype(np.float64)                               # [L, (W, H)]
+
+    value64 = rng.standard_normal((B, S, M, D))
+    value32 = value64.astype(np.float32)
+    bits = None
+    if cfg.dtype == "bf16":
+        bits = bf16_round_bits(value32)
+        value32 = bf16_to_f32_exact(bits)
+
+    if cfg.recipe == "uniform":
+        ref = rng.uniform(-0.1, 1.1, size=(B, Lq, L, 2))
+        off = rng.standard_normal((B, Lq, M, L, K, 2))
+    elif cfg.recipe == "decoder_box":
+        ref = _box_references(rng, B, Lq, L)
+        off = rng.standard_normal((B, Lq, M, L, K, 2)) * (K / 2.0)
+    else:
+        ref = _reference_points(cfg, rng, Lq)
+        if cfg.recipe == "decoder":
+            off = rng.standard_normal((B, Lq, M, L, K, 2)) * 0.02 * wh[None, None, None, :, None, :]
+        else:
+            off = rng.standard_normal((B, Lq, M, L, K, 2)) * 2.0
+
+    logits = rng.standard_normal((B, Lq, M, L * K))
+    want_grad = cfg.backward if with_grad is None else with_grad
+    grad = rng.standard_normal((B, Lq, M * D)).astype(np.float32) if want_grad else None
+    f32 = lambda a: np.ascontiguousarray(np.asarray(a, dtype=np.float32))
+    return FusedInputs(config=cfg, value=np.ascontiguousarray(value32), value_bf16_bits=bits,
+                       spatial_shapes=ss, level_start_index=start, reference_points=f32(ref),
+                       sampling_offsets=f32(off), attention_logits=f32(logits),
+                       grad_output=grad)
+
+
+def select_fused_queries(inp: FusedInputs, queries: np.ndarray) -> FusedInputs:
+    """The same fused call restricted to a subset of queries (value untouched)."""
+    q = np.asarray(queries, dtype=np.int64)
+    take = lambda a: np.ascontiguousarray(a[:, q])
+    return dataclasses.replace(
+        inp, reference_points=take(inp.reference_points),
+        sampling_offsets=take(inp.sampling_offsets),
+        attention_logits=take(inp.attention_logits),
+        grad_output=None if inp.grad_output is None else take(inp.grad_output))
 
 
 def bf16_to_f32_exact(bits: np.ndarray) -> np.ndarray:

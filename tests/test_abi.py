@@ -148,3 +148,52 @@ def test_workspace_size(lib):
     assert _ws_size(lib, B=-1)[0] == BAD
     assert _ws_size(lib, B=1 << 14, Lq=1 << 14, M=8)[0] == UNSUP  # 32-bit point ids overflow
     assert lib.msda_backward_workspace_size(1, 80, 2, 8, 80, 2, 2, None) == NULLP
+
+
+def _ffwd(lib, R=2, dtype=0, B=1, S=80, M=2, D=8, Lq=80, L=2, K=2, ptrs=None):
+    p = [FAKE] * 7 if ptrs is None else ptrs
+    v = lambda x: None if x is None else ctypes.c_void_p(x)
+    return lib.msda_fused_forward(B, S, M, D, Lq, L, K, R, dtype, *[v(x) for x in p], None)
+
+
+def _fbwd(lib, R=2, dtype=0, B=1, S=80, M=2, D=8, Lq=80, L=2, K=2, ptrs=None):
+    p = [FAKE] * 11 if ptrs is None else ptrs
+    v = lambda x: None if x is None else ctypes.c_void_p(x)
+    return lib.msda_fused_backward(B, S, M, D, Lq, L, K, R, dtype, *[v(x) for x in p], None)
+
+
+def test_fused_argument_errors(lib):
+    # Reference points must have 2 or 4 components.
+    for R in (0, 1, 3, 5):
+        assert _ffwd(lib, R=R) == BAD
+        assert _fbwd(lib, R=R) == BAD
+    # Shared size rules of the core.
+    assert _ffwd(lib, B=-1) == BAD
+    assert _ffwd(lib, L=17) == UNSUP and _fbwd(lib, K=65) == UNSUP
+    assert _ffwd(lib, D=6) == UNSUP
+    # The backward is float32 only, D <= 128; the forward also takes bfloat16.
+    assert _fbwd(lib, dtype=1) == UNSUP
+    assert _fbwd(lib, D=132) == UNSUP
+    # Every required pointer; grad_reference_points (the 11th) may be NULL.
+    for i in range(7):
+        ptrs = [FAKE] * 7
+        ptrs[i] = None
+        assert _ffwd(lib, ptrs=ptrs) == NULLP, i
+    for i in range(10):
+        ptrs = [FAKE] * 11
+        ptrs[i] = None
+        assert _fbwd(lib, ptrs=ptrs) == NULLP, i
+    # Alignment: offsets (index 4) need 8 bytes, value 16, logits 4.
+    for i, off in ((0, 8), (4, 4), (5, 2), (6, 8)):
+        ptrs = [FAKE] * 7
+        ptrs[i] = FAKE + off
+        assert _ffwd(lib, ptrs=ptrs) == MISAL, i
+    ptrs = [FAKE] * 11
+    ptrs[8] = FAKE + 4                      # grad_sampling_offsets
+    assert _fbwd(lib, ptrs=ptrs) == MISAL
+    ptrs = [FAKE] * 11
+    ptrs[10] = FAKE + 2                     # grad_reference_points
+    assert _fbwd(lib, ptrs=ptrs) == MISAL
+    # Empty problems launch nothing.
+    assert _ffwd(lib, Lq=0) == OK
+    assert _fbwd(lib, B=0) == OK

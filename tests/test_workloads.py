@@ -112,3 +112,29 @@ def test_select_queries():
     assert sub.sampling_locations.shape[1] == 3
     assert np.array_equal(sub.sampling_locations[:, 1], inp.sampling_locations[:, 1])
     assert np.array_equal(sub.grad_output[:, 2], inp.grad_output[:, 7])
+
+
+@pytest.mark.parametrize("name", ["tiny_fp32", "encoder_fp32", "decoder_fp32",
+                                  "decoder_box_train_fp32"])
+def test_fused_inputs_reproduce_locations_and_weights(name):
+    """The raw inputs of the fused op, pushed through the pages' formulas in
+    float64, give the locations and weights make_inputs draws (up to their
+    float32 storage)."""
+    cfg = W.CONFIGS[name]
+    f = W.make_fused_inputs(cfg, seed=0)
+    c = W.make_inputs(cfg, seed=0)
+    assert np.array_equal(f.value, c.value)
+    if cfg.recipe == "uniform":
+        return  # the uniform recipe draws locations directly
+    ref = f.reference_points.astype(np.float64)[:, :, None, :, None, :]
+    off = f.sampling_offsets.astype(np.float64)
+    if ref.shape[-1] == 2:
+        wh = f.spatial_shapes[:, ::-1].astype(np.float64)[None, None, None, :, None, :]
+        loc = ref + off / wh
+    else:
+        loc = ref[..., :2] + off / cfg.K * ref[..., 2:] * 0.5
+    assert np.abs(loc - c.sampling_locations).max() < 1e-6
+    z = f.attention_logits.astype(np.float64)
+    e = np.exp(z - z.max(-1, keepdims=True))
+    A = (e / e.sum(-1, keepdims=True)).reshape(c.attention_weights.shape)
+    assert np.abs(A - c.attention_weights).max() < 1e-6
