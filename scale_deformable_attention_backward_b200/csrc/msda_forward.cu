@@ -44,14 +44,20 @@ constexpr int kChunkPoints = 512;
 
 }  // namespace
 
-template <typename T, int LANES>
+// FUSED: the inputs are the step before the core (msda_fused.cu): the
+// locations array holds sampling offsets and the weights array holds the
+// attention logits (same shapes), and reference_points [B, Lq, L, R] is read;
+// the setup forms each point's location and softmax weight in registers.  This
+// needs a group's L*K points in one unit (L*K <= PC <= 32), so the softmax is a
+// shuffle reduction over the PC consecutive threads that set the group up.
+template <typename T, int LANES, bool FUSED>
 __global__ void __launch_bounds__(kThreads)
 forward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial_shapes,
                const int64_t* __restrict__ level_start_index,
                const float* __restrict__ sampling_locations,
                const float* __restrict__ attention_weights, T* __restrict__ output,
                long long S, int M, int D, long long Lq, int L, int K, int chunks,
-               long long groups) {
+               long long groups, const float* __restrict__ reference_points, int R) {
   using C = Corner<T>;
   constexpr int E = C::N;
   constexpr int G = kThreads / LANES;
@@ -96,7 +102,29 @@ forward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial_
       const int t = threadIdx.x + r * kThreads;
       const int tg = t / PC, tj = t % PC;
       const long long g = t_ * G + tg;
-      if (tj < pc && g < groups) {
+      const bool live = tj < pc && g < groups;
+      if constexpr (FUSED) {
+        // Softmax over the group's L*K = pc logits, held by PC consecutive lanes.
+        float z = live ? pa[r] : -INFINITY;
+        float mx = z;
+#pragma unroll
+        for (int o = PC / 2; o > 0; o >>= 1) {
+          const float y = __shfl_xor_sync(kFullMask, mx, o, PC);
+          mx = (y > mx || y != y) ? y : mx;
+        }
+        const float e = live ? expf(z - mx) : 0.0f;
+        float sum = e;
+#pragma unroll
+        for (int o = PC / 2; o > 0; o >>= 1) sum += __shfl_xor_sync(kFullMask, sum, o, PC);
+        pa[r] = e * (1.0f / sum);
+        if (live) {
+          const int l = (q0 + tj) / K;
+          const long long bq = g / chunks / M;
+          pxy[r] = fused_location(reference_points + (bq * L + l) * R, pxy[r], R, lv.W[l],
+                                  lv.H[l], K);
+        }
+      }
+      if (live) {
         const int l = (q0 + tj) / K;
         const PointSetup su = setup_point(pxy[r].x, pxy[r].y, pa[r], lv.H[l], lv.W[l], lv.start[l], MD);
         const int slot = tj * G + (tg ^ (tj & 7));
@@ -158,15 +186,15 @@ forward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial_
 
 // Blocks of this kernel that are resident on the current device at once
 // (SM count x blocks per SM), cached per device.
-template <typename T, int LANES>
+template <typename T, int LANES, bool FUSED>
 static long long resident_blocks() {
   static long long cached[64] = {};
   int dev = 0, sms = 0, per_sm = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
   if (dev >= 0 && dev < 64 && cached[dev] > 0) return cached[dev];
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, forward_kernel<T, LANES>, kThreads,
-                                                    0) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, forward_kernel<T, LANES, FUSED>,
+                                                    kThreads, 0) != cudaSuccess ||
       sms <= 0 || per_sm <= 0)
     return 148;
   const long long n = static_cast<long long>(sms) * per_sm;
@@ -178,13 +206,40 @@ template <typename T, int LANES>
 static cudaError_t launch_forward_t(const ForwardArgs& a, cudaStream_t stream) {
   constexpr int G = kThreads / LANES;
   const long long tiles = (a.groups + G - 1) / G;
-  long long blocks = resident_blocks<T, LANES>();
+  long long blocks = resident_blocks<T, LANES, false>();
   if (blocks > tiles) blocks = tiles;
-  forward_kernel<T, LANES><<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(
+  forward_kernel<T, LANES, false><<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(
       static_cast<const T*>(a.value), a.spatial_shapes, a.level_start_index,
       a.sampling_locations, a.attention_weights, static_cast<T*>(a.output), a.S, a.M, a.D,
-      a.Lq, a.L, a.K, a.chunks, a.groups);
+      a.Lq, a.L, a.K, a.chunks, a.groups, nullptr, 0);
   return cudaGetLastError();
+}
+
+template <typename T, int LANES>
+static cudaError_t launch_fused_pipelined_t(const FusedArgs& a, cudaStream_t stream) {
+  constexpr int G = kThreads / LANES;
+  constexpr int PC = kChunkPoints / G;
+  if (PC > 32 || a.L * a.K > PC) return cudaErrorNotSupported;
+  const long long tiles = (a.groups + G - 1) / G;
+  long long blocks = resident_blocks<T, LANES, true>();
+  if (blocks > tiles) blocks = tiles;
+  forward_kernel<T, LANES, true><<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(
+      static_cast<const T*>(a.value), a.spatial_shapes, a.level_start_index,
+      a.sampling_offsets, a.attention_logits, static_cast<T*>(a.output), a.S, a.M, a.D, a.Lq,
+      a.L, a.K, a.chunks, a.groups, a.reference_points, a.R);
+  return cudaGetLastError();
+}
+
+template <typename T>
+static cudaError_t fused_pipelined_lanes(const FusedArgs& a, cudaStream_t stream) {
+  switch (a.lanes) {
+    case 1: return launch_fused_pipelined_t<T, 1>(a, stream);
+    case 2: return launch_fused_pipelined_t<T, 2>(a, stream);
+    case 4: return launch_fused_pipelined_t<T, 4>(a, stream);
+    case 8: return launch_fused_pipelined_t<T, 8>(a, stream);
+    case 16: return launch_fused_pipelined_t<T, 16>(a, stream);
+    default: return cudaErrorNotSupported;
+  }
 }
 
 template <typename T>
@@ -202,6 +257,11 @@ static cudaError_t dispatch_lanes(const ForwardArgs& a, cudaStream_t stream) {
 
 cudaError_t launch_forward(const ForwardArgs& a, cudaStream_t stream) {
   return a.bf16 ? dispatch_lanes<__nv_bfloat16>(a, stream) : dispatch_lanes<float>(a, stream);
+}
+
+cudaError_t launch_fused_forward_pipelined(const FusedArgs& a, cudaStream_t stream) {
+  return a.bf16 ? fused_pipelined_lanes<__nv_bfloat16>(a, stream)
+                : fused_pipelined_lanes<float>(a, stream);
 }
 
 }  // namespace msda

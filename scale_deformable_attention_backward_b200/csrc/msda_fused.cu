@@ -35,22 +35,6 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kChunkPoints = 512;
 
-// The sampling location of one point, formed as the pages' float32 tensors do.
-__device__ __forceinline__ float2 fused_location(const float* __restrict__ ref, float2 off, int R,
-                                                 int W, int H, int K) {
-  if (R == 2)
-    return make_float2(__fadd_rn(__ldg(ref + 0), __fdiv_rn(off.x, static_cast<float>(W))),
-                       __fadd_rn(__ldg(ref + 1), __fdiv_rn(off.y, static_cast<float>(H))));
-  const float fk = static_cast<float>(K);
-  const float tx = __fmul_rn(__fmul_rn(__fdiv_rn(off.x, fk), __ldg(ref + 2)), 0.5f);
-  const float ty = __fmul_rn(__fmul_rn(__fdiv_rn(off.y, fk), __ldg(ref + 3)), 0.5f);
-  return make_float2(__fadd_rn(__ldg(ref + 0), tx), __fadd_rn(__ldg(ref + 1), ty));
-}
-
-// A maximum that keeps NaN, so that a NaN logit makes the whole group's
-// weights NaN (as the softmax does).
-__device__ __forceinline__ float nan_max(float a, float b) { return (b > a || b != b) ? b : a; }
-
 // (max, 1 / sum exp(z - max)) over the LK logits of one group, computed by the
 // LANES lanes of a sub-warp (every lane of the warp takes part).
 template <int LANES>
@@ -66,9 +50,11 @@ __device__ __forceinline__ float2 softmax_norm(const float* __restrict__ z, int 
   return make_float2(m, 1.0f / s);
 }
 
-// Forward: the two phases of msda_forward.cu (per-point setup into a swizzled
-// shared table, then sub-warp gathers), preceded per tile by the softmax
-// normaliser of each group.
+// Forward for any L*K: the two phases of msda_forward.cu (per-point setup into a
+// swizzled shared table, then sub-warp gathers), preceded per tile by the
+// softmax normaliser of each group.  When a group's L*K points fit one unit of
+// the pipelined forward kernel, that kernel is used instead (FUSED variant in
+// msda_forward.cu).
 template <typename T, int LANES>
 __global__ void __launch_bounds__(kThreads)
 fused_forward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial_shapes,
@@ -160,7 +146,7 @@ fused_forward_kernel(const T* __restrict__ value, const int64_t* __restrict__ sp
 // inputs, and the chain rule through them applied per point.  grad_logits
 // holds dA until the group's sum_j A_j dA_j is known, then d z.
 template <int LANES>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 3)  // 3 blocks per SM, as the core backward
 fused_backward_kernel(const float* __restrict__ value, const int64_t* __restrict__ spatial_shapes,
                       const int64_t* __restrict__ level_start_index,
                       const float* __restrict__ reference_points,
@@ -372,6 +358,9 @@ cudaError_t launch_fused_backward_t(const FusedArgs& a, cudaStream_t stream) {
 
 cudaError_t launch_fused_forward(const FusedArgs& a, cudaStream_t stream) {
   if (a.groups == 0) return cudaSuccess;
+  // The pipelined kernel of msda_forward.cu when a group's points fit one unit.
+  const cudaError_t err = launch_fused_forward_pipelined(a, stream);
+  if (err != cudaErrorNotSupported) return err;
   return a.bf16 ? fused_forward_lanes<__nv_bfloat16>(a, stream)
                 : fused_forward_lanes<float>(a, stream);
 }

@@ -1,6 +1,6 @@
 // msda_gather.cuh -- the per-point setup and the corner accumulation of the
-// gather (forward) kernels: msda_forward.cu and the fused forward in
-// msda_fused.cu (sm_100a).
+// gather (forward) kernels, and the location formula of the fused op:
+// msda_forward.cu and msda_fused.cu (sm_100a).
 //
 // Sampling rule of "Deformable DETR模型解读（附源码+论文）",
 // ms_deform_attn_core_pytorch: a point's four bilinear corners, each weighted
@@ -85,5 +85,21 @@ struct Corner<__nv_bfloat16> {
     *reinterpret_cast<uint4*>(p) = make_uint4(u[0], u[1], u[2], u[3]);
   }
 };
+
+// The sampling location of one point, formed as the pages' float32 tensors do.
+__device__ __forceinline__ float2 fused_location(const float* __restrict__ ref, float2 off, int R,
+                                                 int W, int H, int K) {
+  if (R == 2)
+    return make_float2(__fadd_rn(__ldg(ref + 0), __fdiv_rn(off.x, static_cast<float>(W))),
+                       __fadd_rn(__ldg(ref + 1), __fdiv_rn(off.y, static_cast<float>(H))));
+  const float fk = static_cast<float>(K);
+  const float tx = __fmul_rn(__fmul_rn(__fdiv_rn(off.x, fk), __ldg(ref + 2)), 0.5f);
+  const float ty = __fmul_rn(__fmul_rn(__fdiv_rn(off.y, fk), __ldg(ref + 3)), 0.5f);
+  return make_float2(__fadd_rn(__ldg(ref + 0), tx), __fadd_rn(__ldg(ref + 1), ty));
+}
+
+// A maximum that keeps NaN, so that a NaN logit makes the whole group's
+// weights NaN (as the softmax does).
+__device__ __forceinline__ float nan_max(float a, float b) { return (b > a || b != b) ? b : a; }
 
 }  // namespace msda

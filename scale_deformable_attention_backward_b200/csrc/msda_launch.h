@@ -68,6 +68,9 @@ struct FusedArgs {
 };
 
 cudaError_t launch_fused_forward(const FusedArgs& a, cudaStream_t stream);
+// The pipelined forward kernel forming the inputs in registers; returns
+// cudaErrorNotSupported (having launched nothing) unless L*K <= 2 * lanes <= 32.
+cudaError_t launch_fused_forward_pipelined(const FusedArgs& a, cudaStream_t stream);
 cudaError_t launch_fused_backward(const FusedArgs& a, cudaStream_t stream);
 
 // Scratch layout of the cell-sorted backward (msda_backward_sorted.cu).
