@@ -346,6 +346,67 @@ def run_b200(args, world, rank, local):
         "achieved_gbs": round(algo["backward"] / (sorted_ms * 1e-3) / 1e9, 1),
         "note": "cell-sorted path (msda_backward with a workspace), not the timed step"}
 
+    # The op fused with the step before it (softmax of the logits, locations from
+    # reference points and offsets), one training step on the same workload, against
+    # that step written with torch ops around msda_forward / msda_backward.
+    fz = W.make_fused_inputs(cfg, seed=0)
+    fzd = {k: torch.from_numpy(getattr(fz, k)).to(device) for k in
+           ("value", "spatial_shapes", "level_start_index", "reference_points",
+            "sampling_offsets", "attention_logits", "grad_output")}
+    norm = fzd["spatial_shapes"].flip(-1).to(torch.float32)[None, None, None, :, None, :]
+
+    def fused_step():
+        binding.fused_forward(fzd["value"], fzd["spatial_shapes"], fzd["level_start_index"],
+                              fzd["reference_points"], fzd["sampling_offsets"],
+                              fzd["attention_logits"], output=out)
+        binding.fused_backward(fzd["value"], fzd["spatial_shapes"], fzd["level_start_index"],
+                               fzd["reference_points"], fzd["sampling_offsets"],
+                               fzd["attention_logits"], fzd["grad_output"],
+                               reference_grad=False)
+
+    def unfused_step():
+        A = torch.softmax(fzd["attention_logits"], -1)
+        loc = fzd["reference_points"][:, :, None, :, None, :] + fzd["sampling_offsets"] / norm
+        Av = A.view(B, Lq, M, L, K)
+        binding.forward(fzd["value"], fzd["spatial_shapes"], fzd["level_start_index"], loc, Av,
+                        output=out)
+        _, g_loc, g_a = binding.backward(fzd["value"], fzd["spatial_shapes"],
+                                         fzd["level_start_index"], loc, Av, fzd["grad_output"])
+        g_off = g_loc / norm
+        g_a = g_a.view(B, Lq, M, L * K)
+        g_z = A * (g_a - (A * g_a).sum(-1, keepdim=True))
+        return g_off, g_z
+
+    def time_steps(fn, n):
+        for _ in range(args.warmup):
+            flush.fill_(1.0)
+            fn()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(n)]
+        torch.cuda.synchronize()
+        for i in range(n):
+            flush.fill_(float(i))
+            ev[i][0].record(stream)
+            fn()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        return statistics.mean(a.elapsed_time(b) for a, b in ev)
+
+    n_fused = max(3, min(args.steps, 50))
+    fused_ms = max_over_ranks(time_steps(fused_step, n_fused), world, device)
+    unfused_ms = max_over_ranks(time_steps(unfused_step, n_fused), world, device)
+    fused = {
+        "workload": cfg.description + "; inputs are reference points, offsets (pixels) and "
+                                      "softmax logits",
+        "step": "msda_fused_forward + msda_fused_backward (reference points detached)",
+        "ms_per_step": round(fused_ms, 4),
+        "queries_per_s": round(world * queries / (fused_ms * 1e-3), 1),
+        "unfused_ms_per_step": round(unfused_ms, 4),
+        "unfused": "torch softmax and offset normaliser, msda_forward + msda_backward, "
+                   "torch chain rule (offset scaling, softmax Jacobian)",
+        "steps": n_fused,
+    }
+
     # The encoder self-attention forward alone (B=2), the spec workload.
     fcfg = W.CONFIGS[FORWARD_WORKLOAD]
     finp = W.make_inputs(fcfg, seed=0)
@@ -431,6 +492,7 @@ def run_b200(args, world, rank, local):
                    "timing": "CUDA events per step on the launching stream, max over ranks"},
         "roofline": roofline,
         "forward_encoder": forward_encoder,
+        "fused": fused,
         "e2e": {"value": round(world * queries / (e2e_ms * 1e-3), 1), "unit": "queries/s",
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h)},
@@ -456,12 +518,25 @@ def run_case(args, local):
     torch.cuda.set_device(device)
     name = FORWARD_WORKLOAD if args.case == "forward_encoder" else STEP_WORKLOAD
     cfg = W.CONFIGS[name]
-    inp = W.make_inputs(cfg, seed=0, with_grad=args.case.startswith("backward"))
-    d = _device_inputs(inp, device)
+    if args.case.startswith("fused"):
+        fz = W.make_fused_inputs(cfg, seed=0)
+        d = {k: torch.from_numpy(getattr(fz, k)).to(device) for k in
+             ("value", "spatial_shapes", "level_start_index", "reference_points",
+              "sampling_offsets", "attention_logits", "grad_output")}
+    else:
+        inp = W.make_inputs(cfg, seed=0, with_grad=args.case.startswith("backward"))
+        d = _device_inputs(inp, device)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    fused_args = ("value", "spatial_shapes", "level_start_index", "reference_points",
+                  "sampling_offsets", "attention_logits")
 
     def launch():
-        if args.case.startswith("backward"):
+        if args.case == "fused_forward":
+            binding.fused_forward(*[d[k] for k in fused_args])
+        elif args.case == "fused_backward":
+            binding.fused_backward(*[d[k] for k in fused_args], d["grad_output"],
+                                   reference_grad=False)
+        elif args.case.startswith("backward"):
             binding.backward(d["value"], d["spatial_shapes"], d["level_start_index"],
                              d["sampling_locations"], d["attention_weights"], d["grad_output"],
                              workspace="auto" if args.case == "backward_sorted" else None)
@@ -534,7 +609,7 @@ def parse_args(argv=None):
     p.add_argument("--no-cpu-baseline", action="store_true",
                    help="skip the CPU oracle timing (it takes ~10-20 s)")
     p.add_argument("--case", choices=["step", "forward", "forward_encoder", "backward",
-                                      "backward_sorted"],
+                                      "backward_sorted", "fused_forward", "fused_backward"],
                    default="step",
                    help="time one launch type alone (for profiler captures) instead of "
                         "the full benchmark")
