@@ -229,14 +229,21 @@ def barrier(world: int):
 
 def _device_inputs(inp, device):
     import torch
+
+    def bf16(bits):
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(device)
+
     d = {
-        "value": torch.from_numpy(inp.value).to(device),
+        "value": (bf16(inp.value_bf16_bits) if inp.value_bf16_bits is not None
+                  else torch.from_numpy(inp.value).to(device)),
         "spatial_shapes": torch.from_numpy(inp.spatial_shapes).to(device),
         "level_start_index": torch.from_numpy(inp.level_start_index).to(device),
         "sampling_locations": torch.from_numpy(inp.sampling_locations).to(device),
         "attention_weights": torch.from_numpy(inp.attention_weights).to(device),
     }
-    if inp.grad_output is not None:
+    if inp.grad_output_bf16_bits is not None:
+        d["grad_output"] = bf16(inp.grad_output_bf16_bits)
+    elif inp.grad_output is not None:
         d["grad_output"] = torch.from_numpy(inp.grad_output).to(device)
     return d
 
@@ -407,6 +414,34 @@ def run_b200(args, world, rank, local):
         "steps": n_fused,
     }
 
+    # The bfloat16 training step (value and grad_output bf16; float32 arithmetic and
+    # gradients) on the bf16 encoder geometry.
+    bcfg = W.CONFIGS["encoder_train_bf16"]
+    binp = W.make_inputs(bcfg, seed=0)
+    bd = _device_inputs(binp, device)
+    bout = torch.empty((bcfg.B, bcfg.queries, bcfg.M * bcfg.D), dtype=torch.bfloat16,
+                       device=device)
+    bgv = torch.empty(binp.value.shape, dtype=torch.float32, device=device)
+    bgl = torch.empty_like(bd["sampling_locations"])
+    bga = torch.empty_like(bd["attention_weights"])
+
+    def bf16_step():
+        binding.forward(bd["value"], bd["spatial_shapes"], bd["level_start_index"],
+                        bd["sampling_locations"], bd["attention_weights"], output=bout)
+        binding.backward(bd["value"], bd["spatial_shapes"], bd["level_start_index"],
+                         bd["sampling_locations"], bd["attention_weights"], bd["grad_output"],
+                         grad_value=bgv, grad_sampling_locations=bgl, grad_attention_weights=bga)
+
+    bf16_ms = max_over_ranks(time_steps(bf16_step, n_fused), world, device)
+    bq = bcfg.B * bcfg.queries
+    bf16_train = {
+        "workload": bcfg.description, "step": "msda_forward + msda_backward, bf16 value and "
+                                              "grad_output",
+        "ms_per_step": round(bf16_ms, 4),
+        "queries_per_s": round(world * bq / (bf16_ms * 1e-3), 1),
+        "steps": n_fused,
+    }
+
     # The encoder self-attention forward alone (B=2), the spec workload.
     fcfg = W.CONFIGS[FORWARD_WORKLOAD]
     finp = W.make_inputs(fcfg, seed=0)
@@ -493,6 +528,7 @@ def run_b200(args, world, rank, local):
         "roofline": roofline,
         "forward_encoder": forward_encoder,
         "fused": fused,
+        "bf16_train": bf16_train,
         "e2e": {"value": round(world * queries / (e2e_ms * 1e-3), 1), "unit": "queries/s",
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h)},

@@ -44,7 +44,8 @@
  *    (each lane moves 16 bytes); 1 <= L <= 16; 1 <= K <= 64; every size >= 0,
  *    B*S*M*D and B*Lq*M*L*K*2 below 2^62, S*M*D below 2^31 (one image's value
  *    block is addressed with 32-bit offsets), H_l and W_l below 2^22.  `value`,
- *    `output`, `grad_output` and `grad_value` must be 16-byte aligned,
+ *    `output`, `grad_output` and `grad_value` must be 16-byte aligned (the
+ *    bfloat16 backward's `value` and `grad_output`: 8-byte),
  *    `sampling_locations` 8-byte aligned, the other arrays 4-byte aligned
  *    (8-byte for the int64 metadata).
  *  - B*Lq == 0 (or M == 0, or D == 0) is valid and launches nothing, except that
@@ -109,9 +110,11 @@ msda_status msda_forward(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq,
  * inputs (the softmax before them is not differentiated).
  *
  *   value, spatial_shapes, level_start_index, sampling_locations,
- *   attention_weights   as for msda_forward (value_dtype must be MSDA_F32,
- *                       D <= 128)
- *   grad_output              [B, Lq, M * D]        float32
+ *   attention_weights   as for msda_forward; D <= 128.  value_dtype MSDA_F32,
+ *                       or MSDA_BF16 without a workspace (value and
+ *                       grad_output then only need 8-byte alignment; the
+ *                       arithmetic and every gradient stay float32)
+ *   grad_output              [B, Lq, M * D]        value_dtype
  *   grad_value               [B, S, M, D]          float32  overwritten: zeroed on
  *                                                  `stream`, then accumulated with
  *                                                  atomics (summation order, and so
@@ -136,7 +139,7 @@ msda_status msda_backward(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq
                           const int64_t *level_start_index,
                           const float *sampling_locations,
                           const float *attention_weights,
-                          const float *grad_output, float *grad_value,
+                          const void *grad_output, float *grad_value,
                           float *grad_sampling_locations,
                           float *grad_attention_weights, void *workspace,
                           size_t workspace_bytes, void *stream);

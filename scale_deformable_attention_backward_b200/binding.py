@@ -173,16 +173,19 @@ def backward(value: torch.Tensor, spatial_shapes, level_start_index,
     """MSDeformAttn backward: (grad_value, grad_sampling_locations,
     grad_attention_weights), all float32.
 
+    ``value`` and ``grad_output`` are float32, or both bfloat16 (scratch-free
+    path only; the arithmetic and the gradients stay float32).
     ``workspace``: ``None`` (default) selects the scratch-free path (one vector
     atomic per point corner), the faster one on the encoder workloads;
     ``"auto"`` takes scratch for the cell-sorted path from torch's caching
     allocator, and a uint8 CUDA tensor supplies that scratch."""
     dev = value.device
     B, S, M, D, Lq, L, K = _dims(value, sampling_locations, attention_weights)
-    _require(value, "value", torch.float32, dev)
+    _require(value, "value", None, dev)
+    code = _value_code(value)
     _require(sampling_locations, "sampling_locations", torch.float32, dev)
     _require(attention_weights, "attention_weights", torch.float32, dev)
-    _require(grad_output, "grad_output", torch.float32, dev)
+    _require(grad_output, "grad_output", value.dtype, dev)
     if tuple(grad_output.shape) != (B, Lq, M * D):
         raise ValueError("grad_output must be [B, Lq, M*D]")
     ss, st = _metadata(spatial_shapes, level_start_index, S, dev)
@@ -213,7 +216,7 @@ def backward(value: torch.Tensor, spatial_shapes, level_start_index,
         ws, ws_bytes = workspace, workspace.numel()
     with torch.cuda.device(dev):
         stream = torch.cuda.current_stream(dev).cuda_stream
-        _check(library().msda_backward(B, S, M, D, Lq, L, K, MSDA_F32, _ptr(value), _ptr(ss),
+        _check(library().msda_backward(B, S, M, D, Lq, L, K, code, _ptr(value), _ptr(ss),
                                        _ptr(st), _ptr(sampling_locations),
                                        _ptr(attention_weights), _ptr(grad_output), _ptr(gv),
                                        _ptr(gl), _ptr(ga), _ptr(ws), ws_bytes,
@@ -246,13 +249,15 @@ class MSDeformAttnFunction(torch.autograd.Function):
     def backward(ctx, grad_output):
         value, loc, attn = ctx.saved_tensors
         ss, st = ctx.meta
-        gv, gl, ga = backward(value, ss, st, loc, attn, grad_output.contiguous())
-        return gv, None, None, gl, ga, None
+        gv, gl, ga = backward(value, ss, st, loc, attn,
+                              grad_output.to(value.dtype).contiguous())
+        # The op returns float32 gradients; autograd wants value's dtype.
+        return gv.to(value.dtype), None, None, gl, ga, None
 
 
 def ms_deform_attn(value, spatial_shapes, level_start_index, sampling_locations,
                    attention_weights, im2col_step=None):
-    """Differentiable MSDeformAttn core (value float32 for the backward)."""
+    """Differentiable MSDeformAttn core (value float32 or bfloat16)."""
     return MSDeformAttnFunction.apply(value, spatial_shapes, level_start_index,
                                       sampling_locations, attention_weights, im2col_step)
 

@@ -131,13 +131,16 @@ msda_status msda_backward(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq
                           int64_t K, msda_dtype value_dtype, const void* value,
                           const int64_t* spatial_shapes, const int64_t* level_start_index,
                           const float* sampling_locations, const float* attention_weights,
-                          const float* grad_output, float* grad_value,
+                          const void* grad_output, float* grad_value,
                           float* grad_sampling_locations, float* grad_attention_weights,
                           void* workspace, size_t workspace_bytes, void* stream) {
   Common c;
   msda_status st = check_common(B, S, M, D, Lq, L, K, &c);
   if (st != MSDA_OK) return st;
-  if (value_dtype != MSDA_F32) return MSDA_ERR_UNSUPPORTED;
+  // bfloat16 value / grad_output: scratch-free path only.
+  if (value_dtype != MSDA_F32 && !(value_dtype == MSDA_BF16 && workspace == nullptr))
+    return MSDA_ERR_UNSUPPORTED;
+  const uintptr_t in_align = value_dtype == MSDA_F32 ? 16 : 8;
   if (D % 4 != 0 || D > 128 || M > INT32_MAX) return MSDA_ERR_UNSUPPORTED;
   if (workspace != nullptr) {
     size_t need = 0;
@@ -155,7 +158,7 @@ msda_status msda_backward(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq
                grad_output == nullptr || grad_sampling_locations == nullptr ||
                grad_attention_weights == nullptr))
     return MSDA_ERR_NULL_POINTER;
-  if (work && (!aligned(value, 16) || !aligned(grad_output, 16) ||
+  if (work && (!aligned(value, in_align) || !aligned(grad_output, in_align) ||
                !aligned(sampling_locations, 8) || !aligned(grad_sampling_locations, 8) ||
                !aligned(attention_weights, 4) || !aligned(grad_attention_weights, 4) ||
                !aligned(spatial_shapes, 8) || !aligned(level_start_index, 8)))
@@ -165,7 +168,8 @@ msda_status msda_backward(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq
     if (st != MSDA_OK) return st;
   }
   msda::BackwardArgs a;
-  a.value = static_cast<const float*>(value);
+  a.value = value;
+  a.bf16 = value_dtype == MSDA_BF16;
   a.spatial_shapes = spatial_shapes;
   a.level_start_index = level_start_index;
   a.sampling_locations = sampling_locations;

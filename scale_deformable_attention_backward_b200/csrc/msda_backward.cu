@@ -26,18 +26,20 @@
 
 namespace msda {
 
-template <int LANES>
+// T: dtype of value and grad_output (float32, or bfloat16 read 8 bytes per lane);
+// arithmetic and grad_value are float32 for both.
+template <typename T, int LANES>
 __global__ void __launch_bounds__(256)
-backward_kernel(const float* __restrict__ value, const int64_t* __restrict__ spatial_shapes,
+backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial_shapes,
                 const int64_t* __restrict__ level_start_index,
                 const float* __restrict__ sampling_locations,
                 const float* __restrict__ attention_weights,
-                const float* __restrict__ grad_output, float* __restrict__ grad_value,
+                const T* __restrict__ grad_output, float* __restrict__ grad_value,
                 float* __restrict__ grad_sampling_locations,
                 float* __restrict__ grad_attention_weights, long long S, int M, int D,
                 long long Lq, int L, int K, long long groups) {
-  using V = Vec<float>;
-  constexpr int E = V::N;
+  using V = Vec4<T>;
+  constexpr int E = 4;
   __shared__ Levels lv;
   stage_levels(lv, spatial_shapes, level_start_index, L, S);
 
@@ -54,7 +56,7 @@ backward_kernel(const float* __restrict__ value, const int64_t* __restrict__ spa
     const int ch = lane * E;
     const bool lane_on = active && ch < D;  // clamped tail groups touch no memory
     const long long vofs = (grp.b * S * M + grp.m) * static_cast<long long>(D) + ch;
-    const float* vbase = value + vofs;
+    const T* vbase = value + vofs;
     float* gvbase = grad_value + vofs;
     const float* gloc = sampling_locations + grp.bqm * LK * 2;
     const float* gatt = attention_weights + grp.bqm * LK;
@@ -161,31 +163,37 @@ cudaError_t launch_zero(float* p, long long n, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-template <int LANES>
+template <typename T, int LANES>
 static cudaError_t launch_backward_t(const BackwardArgs& a, cudaStream_t stream) {
   constexpr int kThreads = 256;
   const long long per_block = kThreads / LANES;
   long long blocks = (a.groups + per_block - 1) / per_block;
   if (blocks > (1ll << 30)) blocks = 1ll << 30;
-  backward_kernel<LANES><<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(
-      a.value, a.spatial_shapes, a.level_start_index, a.sampling_locations,
-      a.attention_weights, a.grad_output, a.grad_value, a.grad_sampling_locations,
-      a.grad_attention_weights, a.S, a.M, a.D, a.Lq, a.L, a.K, a.groups);
+  backward_kernel<T, LANES><<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(
+      static_cast<const T*>(a.value), a.spatial_shapes, a.level_start_index,
+      a.sampling_locations, a.attention_weights, static_cast<const T*>(a.grad_output),
+      a.grad_value, a.grad_sampling_locations, a.grad_attention_weights, a.S, a.M, a.D, a.Lq,
+      a.L, a.K, a.groups);
   return cudaGetLastError();
+}
+
+template <typename T>
+static cudaError_t backward_lanes(const BackwardArgs& a, cudaStream_t stream) {
+  switch (a.lanes) {
+    case 1: return launch_backward_t<T, 1>(a, stream);
+    case 2: return launch_backward_t<T, 2>(a, stream);
+    case 4: return launch_backward_t<T, 4>(a, stream);
+    case 8: return launch_backward_t<T, 8>(a, stream);
+    case 16: return launch_backward_t<T, 16>(a, stream);
+    case 32: return launch_backward_t<T, 32>(a, stream);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t stream) {
   cudaError_t err = launch_zero(a.grad_value, a.value_elements, stream);
   if (err != cudaSuccess || a.groups == 0) return err;
-  switch (a.lanes) {
-    case 1: return launch_backward_t<1>(a, stream);
-    case 2: return launch_backward_t<2>(a, stream);
-    case 4: return launch_backward_t<4>(a, stream);
-    case 8: return launch_backward_t<8>(a, stream);
-    case 16: return launch_backward_t<16>(a, stream);
-    case 32: return launch_backward_t<32>(a, stream);
-    default: return cudaErrorInvalidValue;
-  }
+  return a.bf16 ? backward_lanes<__nv_bfloat16>(a, stream) : backward_lanes<float>(a, stream);
 }
 
 }  // namespace msda

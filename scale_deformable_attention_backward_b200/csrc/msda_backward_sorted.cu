@@ -713,7 +713,8 @@ cudaError_t launch_cells(const BackwardArgs& a, const SortedLayout& w, const int
   kd.per_m = make_fastdiv(a.M);
   kd.cells_per_bm = static_cast<int>(w.cells_per_bm);
   cell_kernel<LANES, CPL><<<grid_for(runs * LANES, kThreads), kThreads, 0, stream>>>(
-      a.value, a.spatial_shapes, a.level_start_index, a.grad_output, total, records, record_keys,
+      static_cast<const float*>(a.value), a.spatial_shapes, a.level_start_index,
+      static_cast<const float*>(a.grad_output), total, records, record_keys,
       a.grad_value, a.grad_sampling_locations, a.grad_attention_weights, a.S, a.M, a.D, a.L,
       w.cells_per_bm, kd, per_bq);
   return cudaGetLastError();

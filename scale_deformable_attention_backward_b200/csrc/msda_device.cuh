@@ -147,6 +147,30 @@ struct Vec<__nv_bfloat16> {
   }
 };
 
+// 4 channels per lane, widened to float32: 16 bytes of float32 or 8 bytes of
+// bfloat16 (the backward's lane width for both dtypes).
+template <typename T>
+struct Vec4;
+
+template <>
+struct Vec4<float> {
+  __device__ __forceinline__ static void load(const float* p, float (&v)[4]) {
+    const float4 r = __ldg(reinterpret_cast<const float4*>(p));
+    v[0] = r.x; v[1] = r.y; v[2] = r.z; v[3] = r.w;
+  }
+};
+
+template <>
+struct Vec4<__nv_bfloat16> {
+  __device__ __forceinline__ static void load(const __nv_bfloat16* p, float (&v)[4]) {
+    const uint2 r = __ldg(reinterpret_cast<const uint2*>(p));
+    v[0] = __uint_as_float(r.x << 16);
+    v[1] = __uint_as_float(r.x & 0xffff0000u);
+    v[2] = __uint_as_float(r.y << 16);
+    v[3] = __uint_as_float(r.y & 0xffff0000u);
+  }
+};
+
 // Decomposition of a flat work-group index g = ((b * Lq + q) * M + m) * chunks + c.
 struct Group {
   long long bq;    // b * Lq + q

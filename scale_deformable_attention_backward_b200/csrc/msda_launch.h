@@ -27,17 +27,18 @@ struct ForwardArgs {
 };
 
 struct BackwardArgs {
-  const float* value;
+  const void* value;               // float32, or bfloat16 (scratch-free path only)
   const int64_t* spatial_shapes;
   const int64_t* level_start_index;
   const float* sampling_locations;
   const float* attention_weights;
-  const float* grad_output;
+  const void* grad_output;         // value's dtype
   float* grad_value;
   float* grad_sampling_locations;
   float* grad_attention_weights;
   long long B, S, Lq;
   int M, D, L, K;
+  bool bf16;         // value / grad_output dtype
   int lanes;         // lanes per (b, q, m) group; D <= 4 * lanes
   long long groups;  // B * Lq * M
   long long value_elements;  // B * S * M * D (grad_value is zeroed first)

@@ -27,7 +27,8 @@ Geometry and input recipes follow the pages:
 Every draw comes from one ``numpy.random.default_rng(seed)`` in a fixed order:
 value, reference points, offsets, logits, grad_output.  Generation runs in
 float64 and casts at the end (value to bfloat16 with round-to-nearest-even for
-the bf16 workload; locations and weights always float32).
+the bf16 workloads, and grad_output too when they include the backward; locations
+and weights always float32).
 """
 from __future__ import annotations
 
@@ -104,7 +105,13 @@ CONFIGS: Dict[str, Config] = {
         recipe="decoder_box", dtype="f32", backward=True, Lq=300,
         description="decoder cross-attention with box reference points fp32 fwd+bwd: B=2 "
                     "Lq=300 M=8 D=32 K=4 L=4 over the 800x1200 encoder levels; box centre "
-                    "U[0.05,0.95]^2, size U[0.05,0.5]^2, offsets N(0,1)*K/2 box units")
+                    "U[0.05,0.95]^2, size U[0.05,0.5]^2, offsets N(0,1)*K/2 box units"),
+    "encoder_train_bf16": Config(
+        "encoder_train_bf16", B=8, M=8, D=32, K=4, shapes=tuple(ENCODER_608x848),
+        recipe="encoder_valid_ratio", dtype="bf16", backward=True,
+        description="encoder training bf16 fwd+bwd (fp32 arithmetic and gradients): B=8 M=8 "
+                    "D=32 K=4 L=4, levels (76,106),(38,53),(19,27),(8,13), S=Lq=10687, "
+                    "valid ratios U[0.7,1]")
 }
 
 
@@ -120,6 +127,7 @@ class Inputs:
     sampling_locations: np.ndarray     # [B,Lq,M,L,K,2] float32
     attention_weights: np.ndarray      # [B,Lq,M,L,K] float32
     grad_output: Optional[np.ndarray]  # [B,Lq,M*D] float32, backward workloads only
+    grad_output_bf16_bits: Optional[np.ndarray] = None  # raw bf16 of grad_output (bf16 only)
 
     @property
     def dims(self) -> Dict[str, int]:
@@ -235,6 +243,10 @@ def make_inputs(cfg: Config, seed: int = 0, with_grad: Optional[bool] = None) ->
 
     want_grad = cfg.backward if with_grad is None else with_grad
     grad = rng.standard_normal((B, Lq, M * D)).astype(np.float32) if want_grad else None
+    grad_bits = None
+    if grad is not None and cfg.dtype == "bf16":
+        grad_bits = bf16_round_bits(grad)
+        grad = bf16_to_f32_exact(grad_bits)
 
     return Inputs(
         config=cfg,
@@ -245,6 +257,7 @@ def make_inputs(cfg: Config, seed: int = 0, with_grad: Optional[bool] = None) ->
         sampling_locations=np.ascontiguousarray(loc.astype(np.float32)),
         attention_weights=np.ascontiguousarray(attn.astype(np.float32)),
         grad_output=grad,
+        grad_output_bf16_bits=grad_bits,
     )
 
 
@@ -334,4 +347,6 @@ def select_queries(inp: Inputs, queries: np.ndarray) -> Inputs:
         sampling_locations=np.ascontiguousarray(inp.sampling_locations[:, q]),
         attention_weights=np.ascontiguousarray(inp.attention_weights[:, q]),
         grad_output=None if inp.grad_output is None else np.ascontiguousarray(inp.grad_output[:, q]),
+        grad_output_bf16_bits=None if inp.grad_output_bf16_bits is None
+        else np.ascontiguousarray(inp.grad_output_bf16_bits[:, q]),
     )

@@ -32,7 +32,10 @@ def device_inputs(inp, device="cuda"):
     d["level_start_index"] = torch.from_numpy(inp.level_start_index).to(device)
     d["sampling_locations"] = torch.from_numpy(inp.sampling_locations).to(device)
     d["attention_weights"] = torch.from_numpy(inp.attention_weights).to(device)
-    if inp.grad_output is not None:
+    if inp.grad_output_bf16_bits is not None:
+        d["grad_output"] = torch.from_numpy(inp.grad_output_bf16_bits.view(np.int16)).view(
+            torch.bfloat16).to(device)
+    elif inp.grad_output is not None:
         d["grad_output"] = torch.from_numpy(inp.grad_output).to(device)
     return d
 
@@ -45,6 +48,11 @@ def gpu_forward(d):
 
 
 BACKWARD_PATHS = ("sorted", "direct")
+
+
+def backward_paths(d):
+    """The paths a call supports: the cell-sorted path is float32 only."""
+    return BACKWARD_PATHS if d["value"].dtype == torch.float32 else ("direct",)
 
 
 def gpu_backward(d, path="sorted"):
@@ -61,7 +69,7 @@ def gpu_backward(d, path="sorted"):
 def check_backward_paths(d, inp, what=""):
     """Both backward paths against one oracle backward."""
     rv, rl, ra = oracle_backward(inp)
-    for path in BACKWARD_PATHS:
+    for path in backward_paths(d):
         gv, gl, ga = gpu_backward(d, path)
         tag = f" {what} ({path})"
         assert_backward_f32(gv, rv, "grad_value" + tag)

@@ -110,7 +110,15 @@ def test_forward_empty_work_is_ok_without_launch(lib):
 
 
 def test_backward_argument_errors(lib):
-    assert _bwd(lib, dtype=1) == UNSUP             # backward is float32 only
+    # bfloat16 only on the scratch-free path; unknown dtype codes are refused.
+    assert _bwd(lib, dtype=1, ws=FAKE, ws_bytes=1 << 40) == UNSUP
+    assert _bwd(lib, dtype=2) == UNSUP
+    p = [FAKE] * 9
+    p[0] = FAKE + 4                                # bfloat16 value: 8-byte alignment
+    assert _bwd(lib, dtype=1, ptrs=p) == MISAL
+    p = [FAKE] * 9
+    p[5] = FAKE + 2                                # bfloat16 grad_output
+    assert _bwd(lib, dtype=1, ptrs=p) == MISAL
     assert _bwd(lib, D=132) == UNSUP               # at most 128 channels per head
     assert _bwd(lib, D=6) == UNSUP
     assert _bwd(lib, S=-3) == BAD

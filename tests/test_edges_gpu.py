@@ -30,8 +30,12 @@ def random_inputs(seed, B, M, D, K, shapes, Lq, lo=-0.3, hi=1.3, dtype="f32", gr
     attn = rng.uniform(0, 1, size=(B, Lq, M, L, K))
     attn = (attn / attn.sum(axis=(3, 4), keepdims=True)).astype(np.float32)
     go = rng.standard_normal((B, Lq, M * D)).astype(np.float32) if grad else None
+    go_bits = None
+    if go is not None and dtype == "bf16":
+        go_bits = W.bf16_round_bits(go)
+        go = W.bf16_bits_to_f32(go_bits)
     cfg = W.Config("random", B, M, D, K, tuple(shapes), "uniform", dtype, grad, Lq)
-    return W.Inputs(cfg, np.ascontiguousarray(value), bits, ss, start, loc, attn, go)
+    return W.Inputs(cfg, np.ascontiguousarray(value), bits, ss, start, loc, attn, go, go_bits)
 
 
 SHAPES = [[(5, 7)], [(1, 9), (6, 1), (3, 4)], [(16, 3), (8, 2), (4, 1), (2, 1)],
@@ -60,6 +64,35 @@ def test_random_shapes_bf16(D):
     inp = random_inputs(200 + D, B=2, M=2, D=D, K=4, shapes=SHAPES[2], Lq=29, dtype="bf16",
                         grad=False)
     G.assert_forward_bf16(G.gpu_forward(G.device_inputs(inp)), G.oracle_forward(inp))
+
+
+@pytest.mark.parametrize("D", [4, 8, 12, 20, 32, 64, 128])
+@pytest.mark.parametrize("shapes_id", [1, 2])
+def test_random_shapes_bf16_backward(D, shapes_id):
+    """bfloat16 value and grad_output through the scratch-free backward (float32
+    arithmetic and gradients): the oracle sees the same bfloat16 values widened,
+    so the float32 backward tolerances apply."""
+    inp = random_inputs(400 + D + shapes_id, B=2, M=3, D=D, K=3, shapes=SHAPES[shapes_id],
+                        Lq=41, dtype="bf16")
+    G.check_backward_paths(G.device_inputs(inp), inp, f"bf16 D={D}")
+
+
+def test_bf16_autograd():
+    """ms_deform_attn with a bfloat16 value: autograd gets grad_value in bfloat16
+    (rounded from the float32 result) and the location / weight gradients."""
+    inp = random_inputs(77, B=1, M=2, D=16, K=2, shapes=SHAPES[1], Lq=17, dtype="bf16")
+    d = G.device_inputs(inp)
+    v = d["value"].clone().requires_grad_(True)
+    loc = d["sampling_locations"].clone().requires_grad_(True)
+    att = d["attention_weights"].clone().requires_grad_(True)
+    out = binding.ms_deform_attn(v, d["spatial_shapes"], d["level_start_index"], loc, att)
+    out.backward(d["grad_output"])
+    torch.cuda.synchronize()
+    rv, rl, ra = G.oracle_backward(inp)
+    assert v.grad.dtype == torch.bfloat16
+    G.assert_forward_bf16(v.grad.float().cpu().numpy().astype(np.float64), rv, "bf16 grad_value")
+    G.assert_backward_f32(loc.grad.cpu().numpy().astype(np.float64), rl, "bf16 grad_loc")
+    G.assert_backward_f32(att.grad.cpu().numpy().astype(np.float64), ra, "bf16 grad_attn")
 
 
 @pytest.mark.parametrize("L,K", [(1, 1), (3, 5), (16, 1), (1, 64), (16, 4)])

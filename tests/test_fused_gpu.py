@@ -81,7 +81,8 @@ def test_fused_forward_matches_oracle_full_size(name):
         G.assert_forward_f32(got, ref, f"{name} fused forward")
 
 
-@pytest.mark.parametrize("name", [n for n, c in W.CONFIGS.items() if c.backward])
+@pytest.mark.parametrize("name", [n for n, c in W.CONFIGS.items()
+                                  if c.backward and c.dtype == "f32"])
 def test_fused_backward_matches_oracle_full_size(name):
     inp = W.make_fused_inputs(W.CONFIGS[name], seed=0)
     check_fused_backward(inp, fused_device(inp), f"{name} fused")

@@ -7,7 +7,7 @@ import numpy as np
 import pytest
 
 import gpu_support as G
-from scale_deformable_attention_backward_b200 import workloads as W
+from scale_deformable_attention_backward_b200 import binding, workloads as W
 
 pytestmark = pytest.mark.gpu
 
@@ -30,7 +30,7 @@ def test_backward_matches_oracle_full_size(name):
     inp = W.make_inputs(cfg, seed=0)
     d = G.device_inputs(inp)
     rv, rl, ra = G.oracle_backward(inp)
-    for path in G.BACKWARD_PATHS:
+    for path in G.backward_paths(d):
         gv, gl, ga = G.gpu_backward(d, path)
         G.assert_backward_f32(gv, rv, f"{name} grad_value ({path})")
         G.assert_backward_f32(gl, rl, f"{name} grad_sampling_locations ({path})")
@@ -66,3 +66,14 @@ def test_forward_is_deterministic():
     d = G.device_inputs(inp)
     a, b = G.gpu_forward(d), G.gpu_forward(d)
     assert np.array_equal(a, b)
+
+
+def test_bf16_backward_refuses_a_workspace():
+    """The cell-sorted path is float32 only: a bfloat16 call with a workspace is
+    refused before any launch."""
+    inp = W.make_inputs(W.CONFIGS["encoder_train_bf16"].with_batch(1), seed=4)
+    d = G.device_inputs(inp)
+    with pytest.raises(binding.MSDAError, match="UNSUPPORTED"):
+        binding.backward(d["value"], d["spatial_shapes"], d["level_start_index"],
+                         d["sampling_locations"], d["attention_weights"], d["grad_output"],
+                         workspace="auto")
