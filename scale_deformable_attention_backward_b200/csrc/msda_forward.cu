@@ -31,6 +31,8 @@
 // after them, so their HBM latency hides behind the gathers and one barrier
 // per unit suffices.  (Head-major tiles and contiguous per-block tile ranges,
 // which favour L1 reuse, measured slower on the encoder workload.)
+#include <type_traits>
+
 #include "msda_device.cuh"
 #include "msda_gather.cuh"
 #include "msda_launch.h"
@@ -42,6 +44,14 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kChunkPoints = 512;
 
+// Tuning per value dtype (measured on the encoder workloads): for float32 the
+// gathers of up to 8 points are issued back to back (predicated corner loads,
+// Corner::accumulate4) and the kernel is held to 5 blocks per SM (48
+// registers); bfloat16 keeps one branch per corner, a 4-point unroll and the
+// compiler's own register choice (64), which measured faster for it.  The two
+// dtypes therefore get their own __global__ entry (forward_kernel below) around
+// one body.
+
 }  // namespace
 
 // FUSED: the inputs are the step before the core (msda_fused.cu): the
@@ -51,13 +61,13 @@ constexpr int kChunkPoints = 512;
 // needs a group's L*K points in one unit (L*K <= PC <= 32), so the softmax is a
 // shuffle reduction over the PC consecutive threads that set the group up.
 template <typename T, int LANES, bool FUSED>
-__global__ void __launch_bounds__(kThreads)
-forward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial_shapes,
-               const int64_t* __restrict__ level_start_index,
-               const float* __restrict__ sampling_locations,
-               const float* __restrict__ attention_weights, T* __restrict__ output,
-               long long S, int M, int D, long long Lq, int L, int K, int chunks,
-               long long groups, const float* __restrict__ reference_points, int R) {
+__device__ __forceinline__ void
+forward_body(const T* __restrict__ value, const int64_t* __restrict__ spatial_shapes,
+             const int64_t* __restrict__ level_start_index,
+             const float* __restrict__ sampling_locations,
+             const float* __restrict__ attention_weights, T* __restrict__ output,
+             long long S, int M, int D, long long Lq, int L, int K, int chunks,
+             long long groups, const float* __restrict__ reference_points, int R) {
   using C = Corner<T>;
   constexpr int E = C::N;
   constexpr int G = kThreads / LANES;
@@ -159,15 +169,25 @@ forward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial_
     const T* vbase = value + (grp.b * S * M + grp.m) * static_cast<long long>(D) + ch;
     const int pc = min(PC, LK - p0);
     if (lane_on) {
+      if constexpr (std::is_same<T, float>::value) {
+#pragma unroll 8
+        for (int j = 0; j < pc; ++j) {
+          const int slot = j * G + (gi ^ (j & 7));
+          const int4 o = s_off[buf][slot];
+          const float4 w = s_w[buf][slot];
+          C::accumulate4(vbase, o, w, acc);
+        }
+      } else {
 #pragma unroll 4
-      for (int j = 0; j < pc; ++j) {
-        const int slot = j * G + (gi ^ (j & 7));
-        const int4 o = s_off[buf][slot];
-        const float4 w = s_w[buf][slot];
-        if (o.x >= 0) C::accumulate(vbase + o.x, w.x, acc);
-        if (o.y >= 0) C::accumulate(vbase + o.y, w.y, acc);
-        if (o.z >= 0) C::accumulate(vbase + o.z, w.z, acc);
-        if (o.w >= 0) C::accumulate(vbase + o.w, w.w, acc);
+        for (int j = 0; j < pc; ++j) {
+          const int slot = j * G + (gi ^ (j & 7));
+          const int4 o = s_off[buf][slot];
+          const float4 w = s_w[buf][slot];
+          if (o.x >= 0) C::accumulate(vbase + o.x, w.x, acc);
+          if (o.y >= 0) C::accumulate(vbase + o.y, w.y, acc);
+          if (o.z >= 0) C::accumulate(vbase + o.z, w.z, acc);
+          if (o.w >= 0) C::accumulate(vbase + o.w, w.w, acc);
+        }
       }
     }
     if (p0 + PC >= LK) {
@@ -184,6 +204,43 @@ forward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial_
   }
 }
 
+#define MSDA_FORWARD_PARAMS(T)                                                           \
+  const T *__restrict__ value, const int64_t *__restrict__ spatial_shapes,               \
+      const int64_t *__restrict__ level_start_index,                                     \
+      const float *__restrict__ sampling_locations,                                      \
+      const float *__restrict__ attention_weights, T *__restrict__ output, long long S,   \
+      int M, int D, long long Lq, int L, int K, int chunks, long long groups,            \
+      const float *__restrict__ reference_points, int R
+#define MSDA_FORWARD_ARGS                                                                \
+  value, spatial_shapes, level_start_index, sampling_locations, attention_weights, output, \
+      S, M, D, Lq, L, K, chunks, groups, reference_points, R
+
+template <int LANES, bool FUSED>
+__global__ void __launch_bounds__(kThreads, 5) forward_kernel_f32(MSDA_FORWARD_PARAMS(float)) {
+  forward_body<float, LANES, FUSED>(MSDA_FORWARD_ARGS);
+}
+
+template <int LANES, bool FUSED>
+__global__ void __launch_bounds__(kThreads)
+    forward_kernel_bf16(MSDA_FORWARD_PARAMS(__nv_bfloat16)) {
+  forward_body<__nv_bfloat16, LANES, FUSED>(MSDA_FORWARD_ARGS);
+}
+
+#undef MSDA_FORWARD_PARAMS
+#undef MSDA_FORWARD_ARGS
+
+// The entry of each value dtype.
+template <typename T, int LANES, bool FUSED>
+struct ForwardKernel;
+template <int LANES, bool FUSED>
+struct ForwardKernel<float, LANES, FUSED> {
+  static constexpr auto fn = forward_kernel_f32<LANES, FUSED>;
+};
+template <int LANES, bool FUSED>
+struct ForwardKernel<__nv_bfloat16, LANES, FUSED> {
+  static constexpr auto fn = forward_kernel_bf16<LANES, FUSED>;
+};
+
 // Blocks of this kernel that are resident on the current device at once
 // (SM count x blocks per SM), cached per device.
 template <typename T, int LANES, bool FUSED>
@@ -193,7 +250,7 @@ static long long resident_blocks() {
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
   if (dev >= 0 && dev < 64 && cached[dev] > 0) return cached[dev];
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, forward_kernel<T, LANES, FUSED>,
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ForwardKernel<T, LANES, FUSED>::fn,
                                                     kThreads, 0) != cudaSuccess ||
       sms <= 0 || per_sm <= 0)
     return 148;
@@ -208,7 +265,7 @@ static cudaError_t launch_forward_t(const ForwardArgs& a, cudaStream_t stream) {
   const long long tiles = (a.groups + G - 1) / G;
   long long blocks = resident_blocks<T, LANES, false>();
   if (blocks > tiles) blocks = tiles;
-  forward_kernel<T, LANES, false><<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(
+  ForwardKernel<T, LANES, false>::fn<<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(
       static_cast<const T*>(a.value), a.spatial_shapes, a.level_start_index,
       a.sampling_locations, a.attention_weights, static_cast<T*>(a.output), a.S, a.M, a.D,
       a.Lq, a.L, a.K, a.chunks, a.groups, nullptr, 0);
@@ -223,7 +280,7 @@ static cudaError_t launch_fused_pipelined_t(const FusedArgs& a, cudaStream_t str
   const long long tiles = (a.groups + G - 1) / G;
   long long blocks = resident_blocks<T, LANES, true>();
   if (blocks > tiles) blocks = tiles;
-  forward_kernel<T, LANES, true><<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(
+  ForwardKernel<T, LANES, true>::fn<<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(
       static_cast<const T*>(a.value), a.spatial_shapes, a.level_start_index,
       a.sampling_offsets, a.attention_logits, static_cast<T*>(a.output), a.S, a.M, a.D, a.Lq,
       a.L, a.K, a.chunks, a.groups, a.reference_points, a.R);

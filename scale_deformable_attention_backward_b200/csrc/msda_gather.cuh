@@ -57,6 +57,28 @@ struct Corner<float> {
     acc[0] = fma2(ww, make_float2(v.x, v.y), acc[0]);
     acc[1] = fma2(ww, make_float2(v.z, v.w), acc[1]);
   }
+  // All four corners of one point: the loads are predicated (a corner outside the
+  // map reads as zero without being loaded), then the accumulation runs in the
+  // corners' order.
+  __device__ __forceinline__ static void accumulate4(const float* vbase, const int4& o,
+                                                     const float4& w, float2 (&acc)[2]) {
+    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 v0 = z, v1 = z, v2 = z, v3 = z;
+    if (o.x >= 0) v0 = __ldg(reinterpret_cast<const float4*>(vbase + o.x));
+    if (o.y >= 0) v1 = __ldg(reinterpret_cast<const float4*>(vbase + o.y));
+    if (o.z >= 0) v2 = __ldg(reinterpret_cast<const float4*>(vbase + o.z));
+    if (o.w >= 0) v3 = __ldg(reinterpret_cast<const float4*>(vbase + o.w));
+    const float4 vs[4] = {v0, v1, v2, v3};
+    const float ws[4] = {w.x, w.y, w.z, w.w};
+    const int os[4] = {o.x, o.y, o.z, o.w};
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      if (os[c] < 0) continue;
+      const float2 ww = make_float2(ws[c], ws[c]);
+      acc[0] = fma2(ww, make_float2(vs[c].x, vs[c].y), acc[0]);
+      acc[1] = fma2(ww, make_float2(vs[c].z, vs[c].w), acc[1]);
+    }
+  }
   __device__ __forceinline__ static void store(float* p, const float2 (&acc)[2]) {
     *reinterpret_cast<float4*>(p) = make_float4(acc[0].x, acc[0].y, acc[1].x, acc[1].y);
   }
