@@ -217,6 +217,12 @@ def max_over_ranks(x: float, world: int, device=None) -> float:
     return float(t.item())
 
 
+def replica_throughput(world: int, units_per_rank: int, steps: int, total_ms_max: float) -> float:
+    """Whole-job units/s of `world` independent replicas (weak scaling): every rank
+    processes `units_per_rank` per step, and the job takes the slowest rank's time."""
+    return world * units_per_rank * steps / (total_ms_max / 1e3)
+
+
 def barrier(world: int):
     if world > 1:
         import torch.distributed as dist
@@ -307,7 +313,7 @@ def run_b200(args, world, rank, local):
     total_ms_max = max_over_ranks(total_ms, world, device)
     ms_per_step = total_ms_max / args.steps
     queries = B * Lq
-    value = world * queries * args.steps / (total_ms_max / 1e3)
+    value = replica_throughput(world, queries, args.steps, total_ms_max)
 
     peak, peak_kind = measured_peak()
     algo = algorithmic_bytes(cfg, inp)
