@@ -420,6 +420,23 @@ def run_b200(args, world, rank, local):
         "steps": n_fused,
     }
 
+    # The deterministic backward (exact integer accumulation of grad_value) on the
+    # step's workload, with its workspace allocated once.
+    dws = torch.empty(binding.deterministic_workspace_size(B, S, M, D, Lq, L, K),
+                      dtype=torch.uint8, device=device)
+
+    def det_bwd():
+        binding.backward(d["value"], d["spatial_shapes"], d["level_start_index"],
+                         d["sampling_locations"], d["attention_weights"], d["grad_output"],
+                         grad_value=gv, grad_sampling_locations=gl, grad_attention_weights=ga,
+                         workspace=dws, deterministic=True)
+
+    det_ms = max_over_ranks(time_steps(det_bwd, n_fused), world, device)
+    roofline["other"]["backward_deterministic"] = {
+        "mean_ms": round(det_ms, 4),
+        "achieved_gbs": round(algo["backward"] / (det_ms * 1e-3) / 1e9, 1),
+        "note": "msda_backward_deterministic (bit-identical grad_value), not the timed step"}
+
     # The bfloat16 training step (value and grad_output bf16; float32 arithmetic and
     # gradients) on the bf16 encoder geometry.
     bcfg = W.CONFIGS["encoder_train_bf16"]

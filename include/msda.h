@@ -145,6 +145,48 @@ msda_status msda_backward(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq
                           size_t workspace_bytes, void *stream);
 
 /*
+ * Deterministic training backward: the same gradients as msda_backward, and
+ * bit-identical from run to run, whatever the order in which the GPU
+ * schedules the points (the float atomics of msda_backward land in an order
+ * that varies, and so do the last bits of grad_value).  The pages have no
+ * counterpart; it is the scratch-free path with every
+ * grad_value contribution A w_ij gO[d] (the same float32 product) scaled by
+ * 2^e, rounded to an integer and summed exactly with 64-bit integer atomics,
+ * then converted to float32 once.  e comes from a deterministic pass over
+ * the inputs (sum |A| times max |grad_output| bounds every element), so no sum
+ * overflows; the result is closer to the exact sum than float atomics give.
+ * grad_sampling_locations and grad_attention_weights are deterministic in the
+ * scratch-free path already.  If an input (A or grad_output) is not finite,
+ * the call falls back to float atomics, so that NaN and Inf propagate as in
+ * msda_backward; the finite elements are then no longer guaranteed
+ * bit-identical across runs.
+ *
+ *   arguments as msda_backward (value_dtype MSDA_F32 or MSDA_BF16, D <= 128),
+ *   workspace, workspace_bytes
+ *       device scratch owned by the caller, 256-byte aligned, at least
+ *       msda_backward_deterministic_workspace_size() bytes (8 bytes per
+ *       grad_value element plus 8 KB); required (NULL returns
+ *       MSDA_ERR_NULL_POINTER, too small MSDA_ERR_WORKSPACE).  Overlapping
+ *       calls must not share it.
+ */
+msda_status msda_backward_deterministic(int64_t B, int64_t S, int64_t M, int64_t D,
+                                        int64_t Lq, int64_t L, int64_t K,
+                                        msda_dtype value_dtype, const void *value,
+                                        const int64_t *spatial_shapes,
+                                        const int64_t *level_start_index,
+                                        const float *sampling_locations,
+                                        const float *attention_weights,
+                                        const void *grad_output, float *grad_value,
+                                        float *grad_sampling_locations,
+                                        float *grad_attention_weights, void *workspace,
+                                        size_t workspace_bytes, void *stream);
+
+/* Bytes of workspace msda_backward_deterministic needs (host only). */
+msda_status msda_backward_deterministic_workspace_size(int64_t B, int64_t S, int64_t M,
+                                                       int64_t D, int64_t Lq, int64_t L,
+                                                       int64_t K, size_t *bytes);
+
+/*
  * The op fused with the step before it: the sampling locations and attention
  * weights are formed inside the kernels from the raw reference points,
  * sampling offsets and attention logits, so neither is written to or read

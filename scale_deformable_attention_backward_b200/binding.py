@@ -35,6 +35,8 @@ SIGNATURES = {
     "msda_backward": (_I32, [_I64] * 7 + [_I32] + [_VP] * 10 + [_SZ, _VP]),
     "msda_backward_workspace_size": (_I32, [_I64] * 7 + [ctypes.POINTER(_SZ)]),
     "msda_backward_noalloc": (_I32, [_I64] * 7 + [_I32] + [_VP] * 10),
+    "msda_backward_deterministic": (_I32, [_I64] * 7 + [_I32] + [_VP] * 10 + [_SZ, _VP]),
+    "msda_backward_deterministic_workspace_size": (_I32, [_I64] * 7 + [ctypes.POINTER(_SZ)]),
     "msda_fused_forward": (_I32, [_I64] * 8 + [_I32] + [_VP] * 8),
     "msda_fused_backward": (_I32, [_I64] * 8 + [_I32] + [_VP] * 12),
     "msda_check_metadata": (_I32, [_I64, _I64, _VP, _VP]),
@@ -168,7 +170,7 @@ def backward(value: torch.Tensor, spatial_shapes, level_start_index,
              grad_value: Optional[torch.Tensor] = None,
              grad_sampling_locations: Optional[torch.Tensor] = None,
              grad_attention_weights: Optional[torch.Tensor] = None,
-             workspace=None,
+             workspace=None, deterministic: bool = False,
              ) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
     """MSDeformAttn backward: (grad_value, grad_sampling_locations,
     grad_attention_weights), all float32.
@@ -178,7 +180,11 @@ def backward(value: torch.Tensor, spatial_shapes, level_start_index,
     ``workspace``: ``None`` (default) selects the scratch-free path (one vector
     atomic per point corner), the faster one on the encoder workloads;
     ``"auto"`` takes scratch for the cell-sorted path from torch's caching
-    allocator, and a uint8 CUDA tensor supplies that scratch."""
+    allocator, and a uint8 CUDA tensor supplies that scratch.
+
+    ``deterministic=True`` selects ``msda_backward_deterministic`` (bit-identical
+    results run to run); its scratch is ``workspace`` if that is a uint8 CUDA
+    tensor, else taken from torch's caching allocator."""
     dev = value.device
     B, S, M, D, Lq, L, K = _dims(value, sampling_locations, attention_weights)
     _require(value, "value", None, dev)
@@ -205,6 +211,21 @@ def backward(value: torch.Tensor, spatial_shapes, level_start_index,
         out.append(t)
     gv, gl, ga = out
     ws, ws_bytes = None, 0
+    if deterministic:
+        if isinstance(workspace, torch.Tensor):
+            _require(workspace, "workspace", torch.uint8, dev)
+            ws = workspace
+        else:
+            ws = torch.empty(deterministic_workspace_size(B, S, M, D, Lq, L, K),
+                             dtype=torch.uint8, device=dev)
+        with torch.cuda.device(dev):
+            stream = torch.cuda.current_stream(dev).cuda_stream
+            _check(library().msda_backward_deterministic(
+                B, S, M, D, Lq, L, K, code, _ptr(value), _ptr(ss), _ptr(st),
+                _ptr(sampling_locations), _ptr(attention_weights), _ptr(grad_output), _ptr(gv),
+                _ptr(gl), _ptr(ga), _ptr(ws), ws.numel(), ctypes.c_void_p(stream)),
+                "msda_backward_deterministic")
+        return gv, gl, ga
     if isinstance(workspace, str):
         if workspace != "auto":
             raise ValueError("workspace must be 'auto', None or a uint8 CUDA tensor")
@@ -223,6 +244,15 @@ def backward(value: torch.Tensor, spatial_shapes, level_start_index,
                                        ctypes.c_void_p(stream)),
                "msda_backward")
     return gv, gl, ga
+
+
+def deterministic_workspace_size(B, S, M, D, Lq, L, K) -> int:
+    """Bytes of scratch the deterministic backward needs (host computation)."""
+    n = ctypes.c_size_t(0)
+    _check(library().msda_backward_deterministic_workspace_size(B, S, M, D, Lq, L, K,
+                                                                ctypes.byref(n)),
+           "msda_backward_deterministic_workspace_size")
+    return int(n.value)
 
 
 def workspace_size(B, S, M, D, Lq, L, K) -> int:

@@ -194,6 +194,87 @@ msda_status msda_backward(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq
   return err == cudaSuccess ? MSDA_OK : MSDA_ERR_CUDA;
 }
 
+msda_status msda_backward_deterministic_workspace_size(int64_t B, int64_t S, int64_t M,
+                                                       int64_t D, int64_t Lq, int64_t L,
+                                                       int64_t K, size_t* bytes) {
+  if (bytes == nullptr) return MSDA_ERR_NULL_POINTER;
+  *bytes = 0;
+  Common c;
+  const msda_status st = check_common(B, S, M, D, Lq, L, K, &c);
+  if (st != MSDA_OK) return st;
+  if (c.value_elems > (kLimit - msda::kFixedHeaderBytes) / 8) return MSDA_ERR_UNSUPPORTED;
+  *bytes = static_cast<size_t>(msda::kFixedHeaderBytes + 8 * c.value_elems);
+  return MSDA_OK;
+}
+
+msda_status msda_backward_deterministic(int64_t B, int64_t S, int64_t M, int64_t D,
+                                        int64_t Lq, int64_t L, int64_t K,
+                                        msda_dtype value_dtype, const void* value,
+                                        const int64_t* spatial_shapes,
+                                        const int64_t* level_start_index,
+                                        const float* sampling_locations,
+                                        const float* attention_weights,
+                                        const void* grad_output, float* grad_value,
+                                        float* grad_sampling_locations,
+                                        float* grad_attention_weights, void* workspace,
+                                        size_t workspace_bytes, void* stream) {
+  Common c;
+  msda_status st = check_common(B, S, M, D, Lq, L, K, &c);
+  if (st != MSDA_OK) return st;
+  if (value_dtype != MSDA_F32 && value_dtype != MSDA_BF16) return MSDA_ERR_UNSUPPORTED;
+  if (D % 4 != 0 || D > 128 || M > INT32_MAX) return MSDA_ERR_UNSUPPORTED;
+  size_t need = 0;
+  st = msda_backward_deterministic_workspace_size(B, S, M, D, Lq, L, K, &need);
+  if (st != MSDA_OK) return st;
+  if (c.value_elems == 0 && c.out_elems == 0) return MSDA_OK;
+  if (workspace == nullptr) return MSDA_ERR_NULL_POINTER;
+  if (workspace_bytes < need) return MSDA_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return MSDA_ERR_MISALIGNED;
+  const uintptr_t in_align = value_dtype == MSDA_F32 ? 16 : 8;
+  if (c.value_elems > 0 && grad_value == nullptr) return MSDA_ERR_NULL_POINTER;
+  if (!aligned(grad_value, 16)) return MSDA_ERR_MISALIGNED;
+  const bool work = c.out_elems > 0;
+  if (work && (value == nullptr || spatial_shapes == nullptr || level_start_index == nullptr ||
+               sampling_locations == nullptr || attention_weights == nullptr ||
+               grad_output == nullptr || grad_sampling_locations == nullptr ||
+               grad_attention_weights == nullptr))
+    return MSDA_ERR_NULL_POINTER;
+  if (work && (!aligned(value, in_align) || !aligned(grad_output, in_align) ||
+               !aligned(sampling_locations, 8) || !aligned(grad_sampling_locations, 8) ||
+               !aligned(attention_weights, 4) || !aligned(grad_attention_weights, 4) ||
+               !aligned(spatial_shapes, 8) || !aligned(level_start_index, 8)))
+    return MSDA_ERR_MISALIGNED;
+  if (work && validate_env()) {
+    st = check_device_metadata(S, L, spatial_shapes, level_start_index);
+    if (st != MSDA_OK) return st;
+  }
+  msda::BackwardArgs a;
+  a.value = value;
+  a.bf16 = value_dtype == MSDA_BF16;
+  a.spatial_shapes = spatial_shapes;
+  a.level_start_index = level_start_index;
+  a.sampling_locations = sampling_locations;
+  a.attention_weights = attention_weights;
+  a.grad_output = grad_output;
+  a.grad_value = grad_value;
+  a.grad_sampling_locations = grad_sampling_locations;
+  a.grad_attention_weights = grad_attention_weights;
+  a.B = B;
+  a.S = S;
+  a.Lq = Lq;
+  a.M = static_cast<int>(M);
+  a.D = static_cast<int>(D);
+  a.L = static_cast<int>(L);
+  a.K = static_cast<int>(K);
+  a.lanes = pow2_at_least(D / 4);
+  a.groups = work ? B * Lq * M : 0;
+  a.value_elements = c.value_elems;
+  return msda::launch_backward_deterministic(a, workspace, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? MSDA_OK
+             : MSDA_ERR_CUDA;
+}
+
 msda_status msda_fused_forward(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq,
                                int64_t L, int64_t K, int64_t R, msda_dtype value_dtype,
                                const void* value, const int64_t* spatial_shapes,

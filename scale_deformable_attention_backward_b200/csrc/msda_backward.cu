@@ -26,9 +26,31 @@
 
 namespace msda {
 
+// Header of the deterministic backward's workspace: the scale pass's per-block
+// partials, then its result.
+struct FixedHeader {
+  float sum_abs_weights[kScaleBlocks];
+  float max_abs_grad[kScaleBlocks];
+  int fixed;         // 1: all inputs finite, integer accumulation; 0: float atomics
+  float scale;       // 2^e
+  float inv_scale;   // 2^-e
+};
+static_assert(sizeof(FixedHeader) <= kFixedHeaderBytes, "header must fit its slot");
+
 // T: dtype of value and grad_output (float32, or bfloat16 read 8 bytes per lane);
 // arithmetic and grad_value are float32 for both.
-template <typename T, int LANES>
+//
+// FIXED (the deterministic backward): each grad_value contribution A w_ij gO[d]
+// (the same float32 product as the default path) is multiplied by 2^e, rounded
+// to an integer and added with a 64-bit integer atomic.  Integer addition is
+// associative, so the sums -- and after fixed_to_float_kernel, grad_value -- do
+// not depend on the order in which the atomics land.  e is chosen so that no
+// partial sum can reach 2^62 (see scale_final_kernel).  The accumulator row of a
+// (b, pixel, m) keeps channel 4i + c of lane i at c * D/4 + i, so each 64-bit
+// atomic instruction of a sub-warp covers one contiguous span.  If an input is
+// not finite (header->fixed == 0) the kernel falls back to float atomics into
+// grad_value: the NaN / Inf pattern does not depend on the order either.
+template <typename T, int LANES, bool FIXED>
 __global__ void __launch_bounds__(256)
 backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial_shapes,
                 const int64_t* __restrict__ level_start_index,
@@ -37,11 +59,20 @@ backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial
                 const T* __restrict__ grad_output, float* __restrict__ grad_value,
                 float* __restrict__ grad_sampling_locations,
                 float* __restrict__ grad_attention_weights, long long S, int M, int D,
-                long long Lq, int L, int K, long long groups) {
+                long long Lq, int L, int K, long long groups,
+                unsigned long long* __restrict__ fixed_acc,
+                const FixedHeader* __restrict__ header) {
   using V = Vec4<T>;
   constexpr int E = 4;
   __shared__ Levels lv;
   stage_levels(lv, spatial_shapes, level_start_index, L, S);
+  bool use_fixed = false;
+  float scale = 1.0f;
+  if constexpr (FIXED) {
+    use_fixed = header->fixed != 0;
+    scale = header->scale;
+  }
+  const int dq = D / 4;
 
   const int lane = threadIdx.x % LANES;
   const int groups_per_block = blockDim.x / LANES;
@@ -58,6 +89,22 @@ backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial
     const long long vofs = (grp.b * S * M + grp.m) * static_cast<long long>(D) + ch;
     const T* vbase = value + vofs;
     float* gvbase = grad_value + vofs;
+    unsigned long long* abase =
+        FIXED ? fixed_acc + (grp.b * S * M + grp.m) * static_cast<long long>(D) + lane : nullptr;
+    // grad_value corner at element offset o (relative to the (b, m, lane) base) += w gO.
+    auto scatter = [&](long long o, float w, const float (&g)[E]) {
+      if constexpr (FIXED) {
+        if (use_fixed) {
+#pragma unroll
+          for (int c = 0; c < E; ++c)
+            atomicAdd(abase + o + c * dq, static_cast<unsigned long long>(
+                                              __float2ll_rn(__fmul_rn(w * g[c], scale))));
+          return;
+        }
+      }
+      atomicAdd(reinterpret_cast<float4*>(gvbase + o),
+                make_float4(w * g[0], w * g[1], w * g[2], w * g[3]));
+    };
     const float* gloc = sampling_locations + grp.bqm * LK * 2;
     const float* gatt = attention_weights + grp.bqm * LK;
 
@@ -109,14 +156,10 @@ backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial
           }
           const float w00 = a * hx * hy, w10 = a * c.fx * hy;
           const float w01 = a * hx * c.fy, w11 = a * c.fx * c.fy;
-          if (v00) atomicAdd(reinterpret_cast<float4*>(gvbase + off),
-                             make_float4(w00 * go[0], w00 * go[1], w00 * go[2], w00 * go[3]));
-          if (v10) atomicAdd(reinterpret_cast<float4*>(gvbase + off + MD),
-                             make_float4(w10 * go[0], w10 * go[1], w10 * go[2], w10 * go[3]));
-          if (v01) atomicAdd(reinterpret_cast<float4*>(gvbase + off + row),
-                             make_float4(w01 * go[0], w01 * go[1], w01 * go[2], w01 * go[3]));
-          if (v11) atomicAdd(reinterpret_cast<float4*>(gvbase + off + row + MD),
-                             make_float4(w11 * go[0], w11 * go[1], w11 * go[2], w11 * go[3]));
+          if (v00) scatter(off, w00, go);
+          if (v10) scatter(off + MD, w10, go);
+          if (v01) scatter(off + row, w01, go);
+          if (v11) scatter(off + row + MD, w11, go);
         }
 #pragma unroll
         for (int o = LANES / 2; o > 0; o >>= 1) {
@@ -163,29 +206,125 @@ cudaError_t launch_zero(float* p, long long n, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-template <typename T, int LANES>
-static cudaError_t launch_backward_t(const BackwardArgs& a, cudaStream_t stream) {
+// The deterministic backward's scale, pass 1: a fixed grid of kScaleBlocks
+// blocks, each summing |A| and taking max |gO| over a fixed strided share in a
+// fixed order (so the result is the same on every run and every device).
+// A NaN anywhere makes the block's sum or max NaN; an Inf makes it Inf.
+__device__ __forceinline__ float to_float(float x) { return x; }
+__device__ __forceinline__ float to_float(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T>
+__global__ void __launch_bounds__(256)
+scale_partials_kernel(const float* __restrict__ attention_weights, long long n_weights,
+                      const T* __restrict__ grad_output, long long n_grad,
+                      FixedHeader* __restrict__ header) {
+  __shared__ float s_sum[8], s_max[8];
+  const long long stride = static_cast<long long>(kScaleBlocks) * 256;
+  float sum = 0.0f, mx = 0.0f;
+  for (long long i = blockIdx.x * 256ll + threadIdx.x; i < n_weights; i += stride)
+    sum += fabsf(attention_weights[i]);
+  for (long long i = blockIdx.x * 256ll + threadIdx.x; i < n_grad; i += stride) {
+    const float g = fabsf(to_float(grad_output[i]));
+    mx = (g > mx || g != g) ? g : mx;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    sum += __shfl_xor_sync(kFullMask, sum, o);
+    const float y = __shfl_xor_sync(kFullMask, mx, o);
+    mx = (y > mx || y != y) ? y : mx;
+  }
+  if ((threadIdx.x & 31) == 0) {
+    s_sum[threadIdx.x >> 5] = sum;
+    s_max[threadIdx.x >> 5] = mx;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float t = 0.0f, m = 0.0f;
+    for (int w = 0; w < 8; ++w) {
+      t += s_sum[w];
+      m = (s_max[w] > m || s_max[w] != s_max[w]) ? s_max[w] : m;
+    }
+    header->sum_abs_weights[blockIdx.x] = t;
+    header->max_abs_grad[blockIdx.x] = m;
+  }
+}
+
+// Pass 2 (one warp): bound = sum |A| * max |gO| bounds every grad_value element
+// (a point adds A w_ij gO to a corner, and the w_ij of a point sum to 1), so
+// with e = 60 - ceil(log2(bound)) no sum of scaled contributions reaches 2^60.
+__global__ void scale_final_kernel(FixedHeader* __restrict__ header) {
+  const int lane = threadIdx.x;
+  float sum = 0.0f, mx = 0.0f;
+  for (int i = lane; i < kScaleBlocks; i += 32) {
+    sum += header->sum_abs_weights[i];
+    const float m = header->max_abs_grad[i];
+    mx = (m > mx || m != m) ? m : mx;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    sum += __shfl_xor_sync(kFullMask, sum, o);
+    const float y = __shfl_xor_sync(kFullMask, mx, o);
+    mx = (y > mx || y != y) ? y : mx;
+  }
+  if (lane == 0) {
+    const float bound = sum * mx;
+    const bool finite = isfinite(bound);
+    int e = 60;
+    if (finite && bound > 0.0f) {
+      int ex = 0;
+      frexpf(bound, &ex);  // bound < 2^ex
+      e = 60 - ex;
+    }
+    e = max(-60, min(100, e));
+    header->fixed = finite ? 1 : 0;
+    header->scale = ldexpf(1.0f, e);
+    header->inv_scale = ldexpf(1.0f, -e);
+  }
+}
+
+// grad_value = accumulator * 2^-e (one rounding of the exact integer sum), with
+// the accumulator row's channel order undone.  Nothing to do on the float
+// fallback, whose atomics wrote grad_value directly.
+__global__ void fixed_to_float_kernel(const unsigned long long* __restrict__ acc,
+                                      const FixedHeader* __restrict__ header,
+                                      float* __restrict__ grad_value, long long n, int D) {
+  if (header->fixed == 0) return;
+  const float inv = header->inv_scale;
+  const int dq = D / 4;
+  for (long long j = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; j < n;
+       j += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long row = j / D;
+    const int d = static_cast<int>(j - row * D);
+    const long long v = static_cast<long long>(acc[row * D + (d & 3) * dq + (d >> 2)]);
+    grad_value[j] = __fmul_rn(__ll2float_rn(v), inv);
+  }
+}
+
+template <typename T, int LANES, bool FIXED>
+static cudaError_t launch_backward_t(const BackwardArgs& a, unsigned long long* acc,
+                                     const FixedHeader* header, cudaStream_t stream) {
   constexpr int kThreads = 256;
   const long long per_block = kThreads / LANES;
   long long blocks = (a.groups + per_block - 1) / per_block;
   if (blocks > (1ll << 30)) blocks = 1ll << 30;
-  backward_kernel<T, LANES><<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(
+  backward_kernel<T, LANES, FIXED><<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(
       static_cast<const T*>(a.value), a.spatial_shapes, a.level_start_index,
       a.sampling_locations, a.attention_weights, static_cast<const T*>(a.grad_output),
       a.grad_value, a.grad_sampling_locations, a.grad_attention_weights, a.S, a.M, a.D, a.Lq,
-      a.L, a.K, a.groups);
+      a.L, a.K, a.groups, acc, header);
   return cudaGetLastError();
 }
 
-template <typename T>
-static cudaError_t backward_lanes(const BackwardArgs& a, cudaStream_t stream) {
+template <typename T, bool FIXED>
+static cudaError_t backward_lanes(const BackwardArgs& a, unsigned long long* acc,
+                                  const FixedHeader* header, cudaStream_t stream) {
   switch (a.lanes) {
-    case 1: return launch_backward_t<T, 1>(a, stream);
-    case 2: return launch_backward_t<T, 2>(a, stream);
-    case 4: return launch_backward_t<T, 4>(a, stream);
-    case 8: return launch_backward_t<T, 8>(a, stream);
-    case 16: return launch_backward_t<T, 16>(a, stream);
-    case 32: return launch_backward_t<T, 32>(a, stream);
+    case 1: return launch_backward_t<T, 1, FIXED>(a, acc, header, stream);
+    case 2: return launch_backward_t<T, 2, FIXED>(a, acc, header, stream);
+    case 4: return launch_backward_t<T, 4, FIXED>(a, acc, header, stream);
+    case 8: return launch_backward_t<T, 8, FIXED>(a, acc, header, stream);
+    case 16: return launch_backward_t<T, 16, FIXED>(a, acc, header, stream);
+    case 32: return launch_backward_t<T, 32, FIXED>(a, acc, header, stream);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -193,7 +332,43 @@ static cudaError_t backward_lanes(const BackwardArgs& a, cudaStream_t stream) {
 cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t stream) {
   cudaError_t err = launch_zero(a.grad_value, a.value_elements, stream);
   if (err != cudaSuccess || a.groups == 0) return err;
-  return a.bf16 ? backward_lanes<__nv_bfloat16>(a, stream) : backward_lanes<float>(a, stream);
+  return a.bf16 ? backward_lanes<__nv_bfloat16, false>(a, nullptr, nullptr, stream)
+                : backward_lanes<float, false>(a, nullptr, nullptr, stream);
+}
+
+cudaError_t launch_backward_deterministic(const BackwardArgs& a, void* workspace,
+                                          cudaStream_t stream) {
+  auto* header = static_cast<FixedHeader*>(workspace);
+  auto* acc = reinterpret_cast<unsigned long long*>(static_cast<char*>(workspace) +
+                                                    kFixedHeaderBytes);
+  cudaError_t err = launch_zero(a.grad_value, a.value_elements, stream);
+  if (err != cudaSuccess || a.groups == 0) return err;
+  // The accumulators (8 bytes per element) are zeroed as twice as many floats.
+  if ((err = launch_zero(reinterpret_cast<float*>(acc), 2 * a.value_elements, stream)) !=
+      cudaSuccess)
+    return err;
+  const long long n_weights = a.groups * a.L * a.K;
+  const long long n_grad = a.groups * a.D;
+  if (a.bf16)
+    scale_partials_kernel<__nv_bfloat16><<<kScaleBlocks, 256, 0, stream>>>(
+        a.attention_weights, n_weights, static_cast<const __nv_bfloat16*>(a.grad_output),
+        n_grad, header);
+  else
+    scale_partials_kernel<float><<<kScaleBlocks, 256, 0, stream>>>(
+        a.attention_weights, n_weights, static_cast<const float*>(a.grad_output), n_grad,
+        header);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  scale_final_kernel<<<1, 32, 0, stream>>>(header);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  err = a.bf16 ? backward_lanes<__nv_bfloat16, true>(a, acc, header, stream)
+               : backward_lanes<float, true>(a, acc, header, stream);
+  if (err != cudaSuccess) return err;
+  long long blocks = (a.value_elements + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  if (blocks > 0)
+    fixed_to_float_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+        acc, header, a.grad_value, a.value_elements, a.D);
+  return cudaGetLastError();
 }
 
 }  // namespace msda

@@ -96,4 +96,12 @@ cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t stream);
 cudaError_t launch_backward_sorted(const BackwardArgs& a, void* workspace, cudaStream_t stream);
 cudaError_t launch_zero(float* p, long long n, cudaStream_t stream);
 
+// Deterministic backward (msda_backward.cu): the scratch-free kernel with the
+// grad_value contributions accumulated exactly as scaled 64-bit integers.  The
+// workspace holds a kFixedHeaderBytes header, then 8 bytes per grad_value element.
+constexpr int kScaleBlocks = 512;
+constexpr long long kFixedHeaderBytes = 8192;
+cudaError_t launch_backward_deterministic(const BackwardArgs& a, void* workspace,
+                                          cudaStream_t stream);
+
 }  // namespace msda

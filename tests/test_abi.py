@@ -205,3 +205,40 @@ def test_fused_argument_errors(lib):
     # Empty problems launch nothing.
     assert _ffwd(lib, Lq=0) == OK
     assert _fbwd(lib, B=0) == OK
+
+
+def _dbwd(lib, B=1, S=80, M=2, D=8, Lq=80, L=2, K=2, dtype=0, ptrs=None, ws=FAKE,
+          ws_bytes=1 << 40):
+    p = [FAKE] * 9 if ptrs is None else ptrs
+    v = lambda x: None if x is None else ctypes.c_void_p(x)
+    return lib.msda_backward_deterministic(B, S, M, D, Lq, L, K, dtype, *[v(x) for x in p],
+                                           v(ws), ws_bytes, None)
+
+
+def test_deterministic_backward_arguments(lib):
+    n = ctypes.c_size_t(0)
+    assert lib.msda_backward_deterministic_workspace_size(4, 19947, 8, 32, 19947, 4, 4,
+                                                          ctypes.byref(n)) == OK
+    # 8 bytes per grad_value element plus an 8 KB header.
+    assert n.value == 8192 + 8 * 4 * 19947 * 8 * 32
+    assert lib.msda_backward_deterministic_workspace_size(-1, 1, 1, 4, 1, 1, 1,
+                                                          ctypes.byref(n)) == BAD
+    assert lib.msda_backward_deterministic_workspace_size(1, 1, 1, 4, 1, 1, 1, None) == NULLP
+    # Every call below fails validation before any launch.
+    assert _dbwd(lib, ws=None) == NULLP                 # the workspace is required
+    need = 8192 + 8 * 80 * 2 * 8
+    assert _dbwd(lib, ws_bytes=need - 1) == WORKSPACE
+    assert _dbwd(lib, ws=FAKE + 16) == MISAL
+    assert _dbwd(lib, dtype=2) == UNSUP
+    assert _dbwd(lib, D=132) == UNSUP
+    assert _dbwd(lib, D=6) == UNSUP
+    p = [FAKE] * 9
+    p[6] = None                                         # grad_value
+    assert _dbwd(lib, ptrs=p) == NULLP
+    p = [FAKE] * 9
+    p[5] = FAKE + 4                                     # float32 grad_output: 16-byte
+    assert _dbwd(lib, ptrs=p) == MISAL
+    p = [FAKE] * 9
+    p[0] = FAKE + 4                                     # bfloat16 value: 8-byte
+    assert _dbwd(lib, dtype=1, ptrs=p) == MISAL
+    assert _dbwd(lib, B=0, ptrs=[None] * 9, ws=None) == OK
