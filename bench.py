@@ -78,6 +78,25 @@ def algorithmic_bytes(cfg: W.Config, inp: W.Inputs) -> dict:
     return {"forward": fwd, "backward": bwd}
 
 
+def grad_value_adds(inp: W.Inputs) -> int:
+    """Float adds the backward's grad_value scatter performs: D per corner inside
+    the map, i.e. one vector atomic per lane and corner (host count from the
+    inputs, float64 pixel mapping)."""
+    B, S, M, D = inp.value.shape
+    ss = inp.spatial_shapes.astype(np.float64)
+    loc = inp.sampling_locations.astype(np.float64)            # [B,Lq,M,L,K,2]
+    W_ = ss[:, 1][None, None, None, :, None]
+    H_ = ss[:, 0][None, None, None, :, None]
+    x0 = np.floor(loc[..., 0] * W_ - 0.5)
+    y0 = np.floor(loc[..., 1] * H_ - 0.5)
+    vx = (x0 >= 0) & (x0 <= W_ - 1)
+    vx1 = (x0 + 1 >= 0) & (x0 + 1 <= W_ - 1)
+    vy = (y0 >= 0) & (y0 <= H_ - 1)
+    vy1 = (y0 + 1 >= 0) & (y0 + 1 <= H_ - 1)
+    corners = (vx & vy).sum() + (vx1 & vy).sum() + (vx & vy1).sum() + (vx1 & vy1).sum()
+    return int(corners) * D
+
+
 def source_digest(files) -> str:
     """Digest of the kernel sources a recorded measurement depends on."""
     h = hashlib.sha256()
@@ -339,6 +358,15 @@ def run_b200(args, world, rank, local):
                          "traffic": recorded_traffic(f"{STEP_WORKLOAD}.backward")},
         },
     }
+
+    # The backward's real ceiling: L2 float atomics (a probe on this pool measured
+    # about 1.5e12 float adds/s for 16-byte vector reductions).
+    adds = grad_value_adds(inp)
+    roofline["other"]["backward"]["atomic_adds"] = adds
+    roofline["other"]["backward"]["atomic_adds_per_s"] = round(adds / (b_ms * 1e-3), 1)
+    roofline["other"]["backward"]["atomic_note"] = (
+        "bound by L2 float atomics; a throughput probe on this pool measured about 1.5e12 "
+        "float adds/s for 16-byte vector reductions")
 
     # The cell-sorted backward (with a workspace), timed alone for reference.
     for _ in range(args.warmup):

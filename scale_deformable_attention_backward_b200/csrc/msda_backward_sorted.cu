@@ -53,6 +53,8 @@
 // Scratch (caller-provided workspace, see msda_backward_workspace_size): counts
 // per (chunk, cell), per-cell totals, scan tile sums, the slot of every point,
 // and the sorted records (16 bytes) and keys (4 bytes).
+#include <mutex>
+
 #include "msda_device.cuh"
 #include "msda_launch.h"
 
@@ -762,16 +764,20 @@ cudaError_t launch_backward_sorted(const BackwardArgs& a, void* workspace,
   // The hist and place kernels' per-cell tables exceed the default 48 KB of
   // dynamic shared memory; the opt-in is set once per device.
   const size_t cell_smem = sizeof(int) * static_cast<size_t>(kHistCells);
+  static std::mutex smem_mu;
   static bool smem_set[64] = {};
   int dev = 0;
   if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
-  if (dev < 0 || dev >= 64 || !smem_set[dev]) {
-    if ((err = cudaFuncSetAttribute(hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    static_cast<int>(cell_smem))) != cudaSuccess ||
-        (err = cudaFuncSetAttribute(place_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    static_cast<int>(cell_smem))) != cudaSuccess)
-      return err;
-    if (dev >= 0 && dev < 64) smem_set[dev] = true;
+  {
+    std::lock_guard<std::mutex> lock(smem_mu);
+    if (dev < 0 || dev >= 64 || !smem_set[dev]) {
+      if ((err = cudaFuncSetAttribute(hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      static_cast<int>(cell_smem))) != cudaSuccess ||
+          (err = cudaFuncSetAttribute(place_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      static_cast<int>(cell_smem))) != cudaSuccess)
+        return err;
+      if (dev >= 0 && dev < 64) smem_set[dev] = true;
+    }
   }
   const unsigned blocks = static_cast<unsigned>(w.segments * w.chunks);
   const int chunks = static_cast<int>(w.chunks);

@@ -31,6 +31,7 @@
 // after them, so their HBM latency hides behind the gathers and one barrier
 // per unit suffices.  (Head-major tiles and contiguous per-block tile ranges,
 // which favour L1 reuse, measured slower on the encoder workload.)
+#include <atomic>
 #include <type_traits>
 
 #include "msda_device.cuh"
@@ -245,17 +246,17 @@ struct ForwardKernel<__nv_bfloat16, LANES, FUSED> {
 // (SM count x blocks per SM), cached per device.
 template <typename T, int LANES, bool FUSED>
 static long long resident_blocks() {
-  static long long cached[64] = {};
+  static std::atomic<long long> cached[64];  // 0 until known; benign concurrent fills
   int dev = 0, sms = 0, per_sm = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-  if (dev >= 0 && dev < 64 && cached[dev] > 0) return cached[dev];
+  if (dev >= 0 && dev < 64 && cached[dev].load() > 0) return cached[dev].load();
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
       cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ForwardKernel<T, LANES, FUSED>::fn,
                                                     kThreads, 0) != cudaSuccess ||
       sms <= 0 || per_sm <= 0)
     return 148;
   const long long n = static_cast<long long>(sms) * per_sm;
-  if (dev >= 0 && dev < 64) cached[dev] = n;
+  if (dev >= 0 && dev < 64) cached[dev].store(n);
   return n;
 }
 

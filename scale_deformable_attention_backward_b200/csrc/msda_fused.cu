@@ -22,6 +22,7 @@
 //   d z_i   = A_i (dA_i - sum_j A_j dA_j)             over the (b, q, m) group
 // where d loc and dA are the core's grad_sampling_locations and
 // grad_attention_weights.
+#include <atomic>
 #include <cmath>
 
 #include "msda_device.cuh"
@@ -301,17 +302,17 @@ fused_backward_kernel(const float* __restrict__ value, const int64_t* __restrict
 
 template <typename T, int LANES>
 long long resident_forward_blocks() {
-  static long long cached[64] = {};
+  static std::atomic<long long> cached[64];  // 0 until known; benign concurrent fills
   int dev = 0, sms = 0, per_sm = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-  if (dev >= 0 && dev < 64 && cached[dev] > 0) return cached[dev];
+  if (dev >= 0 && dev < 64 && cached[dev].load() > 0) return cached[dev].load();
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
       cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fused_forward_kernel<T, LANES>,
                                                     kThreads, 0) != cudaSuccess ||
       sms <= 0 || per_sm <= 0)
     return 148;
   const long long n = static_cast<long long>(sms) * per_sm;
-  if (dev >= 0 && dev < 64) cached[dev] = n;
+  if (dev >= 0 && dev < 64) cached[dev].store(n);
   return n;
 }
 
