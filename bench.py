@@ -465,6 +465,39 @@ def run_b200(args, world, rank, local):
         "achieved_gbs": round(algo["backward"] / (det_ms * 1e-3) / 1e9, 1),
         "note": "msda_backward_deterministic (bit-identical grad_value), not the timed step"}
 
+    # The output projection after the op (Linear 256 -> 256 on the tensor cores,
+    # tcgen05 kind::tf32) on the step's forward output.
+    prng = np.random.default_rng(1)
+    pw = torch.from_numpy((prng.standard_normal((M * D, M * D)) /
+                           np.sqrt(M * D)).astype(np.float32)).to(device)
+    pb = torch.from_numpy(prng.standard_normal(M * D).astype(np.float32)).to(device)
+    px = out.reshape(-1, M * D)
+    py = torch.empty_like(px)
+
+    def proj_step():
+        binding.output_projection(px, pw, pb, out=py)
+
+    proj_ms = max_over_ranks(time_steps(proj_step, n_fused), world, device)
+    proj_rows = B * Lq
+    proj_bytes = proj_rows * M * D * 4 * 2 + M * D * M * D * 4 + M * D * 4
+    proj_flops = 2.0 * proj_rows * (M * D) * (M * D)
+    with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+        bf16_peak = float(json.load(f).get("bf16_tflops", 0.0)) or None
+    tf32_peak = None if bf16_peak is None else bf16_peak * 1.1 / 2.25
+    proj_gbs = proj_bytes / (proj_ms * 1e-3) / 1e9
+    projection = {
+        "workload": f"output_proj Linear {M * D}->{M * D} on the step's forward output "
+                    f"({proj_rows} rows)",
+        "kernel": "proj_kernel: tcgen05.mma kind::tf32, accumulator in tensor memory",
+        "mean_ms": round(proj_ms, 4),
+        "roofline": {"bound": "hbm", "achieved": round(proj_gbs, 1), "peak": peak,
+                     "unit": "GB/s", "frac": round(proj_gbs / peak, 4),
+                     "algorithmic_bytes": proj_bytes},
+        "tensor": {"achieved_tflops": round(proj_flops / (proj_ms * 1e-3) / 1e12, 1),
+                   "tf32_peak_tflops": None if tf32_peak is None else round(tf32_peak, 1),
+                   "peak_source": "measured bf16 burst x nominal tf32/bf16 ratio 1.1/2.25"},
+    }
+
     # The bfloat16 training step (value and grad_output bf16; float32 arithmetic and
     # gradients) on the bf16 encoder geometry.
     bcfg = W.CONFIGS["encoder_train_bf16"]
@@ -580,6 +613,7 @@ def run_b200(args, world, rank, local):
         "forward_encoder": forward_encoder,
         "fused": fused,
         "bf16_train": bf16_train,
+        "projection": projection,
         "e2e": {"value": round(world * queries / (e2e_ms * 1e-3), 1), "unit": "queries/s",
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h)},

@@ -187,6 +187,35 @@ msda_status msda_backward_deterministic_workspace_size(int64_t B, int64_t S, int
                                                        int64_t K, size_t *bytes);
 
 /*
+ * The output projection after the op, on the tensor cores: a Linear layer,
+ *   y[r, n] = sum_k x[r, k] * weight[n, k] + bias[n]
+ * ("Deformable DETR模型解读（附源码+论文）", MultiScaleDeformableAttention.forward,
+ * output_proj applied to the op's [N, Lq, M*D] output, rows = N * Lq).
+ * tcgen05.mma kind::tf32: the operands are read as TF32 (the float32 top 19
+ * bits), products are summed in float32, so |error| stays within about
+ * 2^-9 * sum_k |x[r,k] * weight[n,k]|; bias is added in float32.
+ *
+ *   x       [rows, c_in]     float32, 16-byte aligned (c_in % 8 == 0, 8 <= c_in <= 4096)
+ *   weight  [c_out, c_in]    float32, 16-byte aligned (nn.Linear's layout;
+ *                            c_out % 16 == 0, 16 <= c_out <= 256)
+ *   bias    [c_out]          float32, or NULL
+ *   y       [rows, c_out]    float32, 16-byte aligned, written
+ * rows == 0 launches nothing.  The kernel's waits for its MMAs are bounded;
+ * if one ever runs out, its rows are left unwritten and
+ * msda_output_projection_check reports it.
+ */
+msda_status msda_output_projection(int64_t rows, int64_t c_in, int64_t c_out, const float *x,
+                                   const float *weight, const float *bias, float *y,
+                                   void *stream);
+
+/*
+ * *failed = 1 if a projection since the last check gave up waiting for its
+ * MMAs, else 0; clears the flag.  Synchronises with the device (it copies the
+ * flag to the host).
+ */
+msda_status msda_output_projection_check(int *failed);
+
+/*
  * The op fused with the step before it: the sampling locations and attention
  * weights are formed inside the kernels from the raw reference points,
  * sampling offsets and attention logits, so neither is written to or read

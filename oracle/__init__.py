@@ -163,6 +163,19 @@ class Oracle:
         return gv, goff, gz, gref
 
 
+def project(x, weight, bias=None):
+    """The output projection after the op, a Linear layer ("Deformable DETR模型解读",
+    MultiScaleDeformableAttention.forward, output_proj): y = x @ weight.T + bias in
+    float64 (numpy's matmul serves as the step).  x [rows, c_in], weight
+    [c_out, c_in], bias [c_out] or None."""
+    x64 = np.asarray(x, dtype=np.float64)
+    w64 = np.asarray(weight, dtype=np.float64)
+    y = x64 @ w64.T
+    if bias is not None:
+        y = y + np.asarray(bias, dtype=np.float64)[None, :]
+    return y
+
+
 _DEFAULT = None
 
 
@@ -190,4 +203,5 @@ def fused_backward(*args, **kwargs):
     return default().fused_backward(*args, **kwargs)
 
 
-__all__ = ["Oracle", "default", "forward", "backward", "fused_forward", "fused_backward"]
+__all__ = ["Oracle", "default", "forward", "backward", "fused_forward", "fused_backward",
+           "project"]

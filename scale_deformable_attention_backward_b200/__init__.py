@@ -11,7 +11,7 @@ call, which raises if it is missing.
 """
 _BINDING_NAMES = ("forward", "backward", "ms_deform_attn", "MSDeformAttnFunction",
                   "fused_forward", "fused_backward", "ms_deform_attn_fused",
-                  "MSDeformAttnFusedFunction", "MSDAError", "library")
+                  "MSDeformAttnFusedFunction", "output_projection", "MSDAError", "library")
 
 __all__ = list(_BINDING_NAMES)
 

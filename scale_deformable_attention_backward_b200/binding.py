@@ -39,6 +39,8 @@ SIGNATURES = {
     "msda_backward_deterministic_workspace_size": (_I32, [_I64] * 7 + [ctypes.POINTER(_SZ)]),
     "msda_fused_forward": (_I32, [_I64] * 8 + [_I32] + [_VP] * 8),
     "msda_fused_backward": (_I32, [_I64] * 8 + [_I32] + [_VP] * 12),
+    "msda_output_projection": (_I32, [_I64] * 3 + [_VP] * 5),
+    "msda_output_projection_check": (_I32, [ctypes.POINTER(_I32)]),
     "msda_check_metadata": (_I32, [_I64, _I64, _VP, _VP]),
     "msda_status_string": (ctypes.c_char_p, [_I32]),
     "msda_version": (_I32, []),
@@ -405,3 +407,42 @@ def ms_deform_attn_fused(value, spatial_shapes, level_start_index, reference_poi
     return MSDeformAttnFusedFunction.apply(value, spatial_shapes, level_start_index,
                                            reference_points, sampling_offsets,
                                            attention_logits)
+
+
+def output_projection(x: torch.Tensor, weight: torch.Tensor, bias: Optional[torch.Tensor] = None,
+                      out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """The Linear layer after the op on the tensor cores (``msda_output_projection``):
+    ``x [..., c_in] @ weight[c_out, c_in].T + bias``, float32 in and out (TF32
+    products, float32 sums)."""
+    dev = x.device
+    c_in = x.shape[-1]
+    c_out = weight.shape[0]
+    if tuple(weight.shape) != (c_out, c_in):
+        raise ValueError("weight must be [c_out, c_in]")
+    _require(x, "x", torch.float32, dev)
+    _require(weight, "weight", torch.float32, dev)
+    if bias is not None:
+        _require(bias, "bias", torch.float32, dev)
+        if tuple(bias.shape) != (c_out,):
+            raise ValueError("bias must be [c_out]")
+    rows = x.numel() // c_in if c_in else 0
+    if out is None:
+        out = torch.empty(tuple(x.shape[:-1]) + (c_out,), dtype=torch.float32, device=dev)
+    else:
+        _require(out, "out", torch.float32, dev)
+        if tuple(out.shape) != tuple(x.shape[:-1]) + (c_out,):
+            raise ValueError("out must be [..., c_out]")
+    with torch.cuda.device(dev):
+        stream = torch.cuda.current_stream(dev).cuda_stream
+        _check(library().msda_output_projection(rows, c_in, c_out, _ptr(x), _ptr(weight),
+                                                _ptr(bias), _ptr(out), ctypes.c_void_p(stream)),
+               "msda_output_projection")
+    return out
+
+
+def output_projection_failed() -> bool:
+    """Whether a projection since the last call gave up waiting for its MMAs
+    (synchronises with the device)."""
+    f = ctypes.c_int(0)
+    _check(library().msda_output_projection_check(ctypes.byref(f)), "msda_output_projection_check")
+    return bool(f.value)

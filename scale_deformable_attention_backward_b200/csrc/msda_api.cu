@@ -275,6 +275,38 @@ msda_status msda_backward_deterministic(int64_t B, int64_t S, int64_t M, int64_t
              : MSDA_ERR_CUDA;
 }
 
+msda_status msda_output_projection(int64_t rows, int64_t c_in, int64_t c_out, const float* x,
+                                   const float* weight, const float* bias, float* y,
+                                   void* stream) {
+  if (rows < 0 || c_in < 0 || c_out < 0) return MSDA_ERR_BAD_SHAPE;
+  if (c_in % 8 != 0 || c_in < 8 || c_in > 4096 || c_out % 16 != 0 || c_out < 16 ||
+      c_out > 256)
+    return MSDA_ERR_UNSUPPORTED;
+  int64_t xe = 0, ye = 0;
+  if (!product_ok({rows, c_in}, &xe) || !product_ok({rows, c_out}, &ye))
+    return MSDA_ERR_BAD_SHAPE;
+  if (rows == 0) return MSDA_OK;
+  if (x == nullptr || weight == nullptr || y == nullptr) return MSDA_ERR_NULL_POINTER;
+  if (!aligned(x, 16) || !aligned(weight, 16) || !aligned(y, 16) || !aligned(bias, 4))
+    return MSDA_ERR_MISALIGNED;
+  return msda::launch_projection(x, weight, bias, y, rows, static_cast<int>(c_in),
+                                 static_cast<int>(c_out), static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? MSDA_OK
+             : MSDA_ERR_CUDA;
+}
+
+msda_status msda_output_projection_check(int* failed) {
+  if (failed == nullptr) return MSDA_ERR_NULL_POINTER;
+  int* flag = nullptr;
+  if (msda::projection_failed_flag(&flag) != cudaSuccess) return MSDA_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpy(failed, flag, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess ||
+      cudaMemcpy(flag, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+    return MSDA_ERR_CUDA;
+  return MSDA_OK;
+}
+
 msda_status msda_fused_forward(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq,
                                int64_t L, int64_t K, int64_t R, msda_dtype value_dtype,
                                const void* value, const int64_t* spatial_shapes,

@@ -242,3 +242,20 @@ def test_deterministic_backward_arguments(lib):
     p[0] = FAKE + 4                                     # bfloat16 value: 8-byte
     assert _dbwd(lib, dtype=1, ptrs=p) == MISAL
     assert _dbwd(lib, B=0, ptrs=[None] * 9, ws=None) == OK
+
+
+def test_output_projection_arguments(lib):
+    v = lambda p: None if p is None else ctypes.c_void_p(p)
+
+    def proj(rows=128, c_in=256, c_out=256, x=FAKE, w=FAKE, b=FAKE, y=FAKE):
+        return lib.msda_output_projection(rows, c_in, c_out, v(x), v(w), v(b), v(y), None)
+
+    # Every call below fails validation before any launch.
+    assert proj(rows=-1) == BAD
+    assert proj(c_in=12) == UNSUP and proj(c_in=0) == UNSUP and proj(c_in=4104) == UNSUP
+    assert proj(c_out=8) == UNSUP and proj(c_out=24) == UNSUP and proj(c_out=272) == UNSUP
+    assert proj(x=None) == NULLP and proj(w=None) == NULLP and proj(y=None) == NULLP
+    assert proj(x=FAKE + 8) == MISAL and proj(w=FAKE + 4) == MISAL and proj(y=FAKE + 8) == MISAL
+    assert proj(b=FAKE + 2) == MISAL
+    assert proj(rows=0, x=None, w=None, b=None, y=None) == OK
+    assert lib.msda_output_projection_check(None) == NULLP
