@@ -8,15 +8,17 @@
 // This is a dense contraction, so it runs on the tensor cores: kind::tf32
 // (float32 operands read as TF32, float32 accumulation).
 //
-// One CTA of 128 threads owns 128 rows of X at a time (a persistent loop over
-// row tiles).  Per K chunk of 32 it stages the X chunk [128 x 32] and the Wt
-// chunk [C_out x 32] in shared memory as K-major core matrices without swizzle
-// (a core matrix is 8 rows x 16 bytes; K-neighbouring core matrices are LBO
-// bytes apart, 8-row groups SBO bytes apart), then thread 0 issues four
-// M=128 x N=C_out x K=8 MMAs into a C_out-column float32 accumulator in tensor
-// memory and commits them to an mbarrier.  After the last chunk every warp
-// reads its 32 rows of the accumulator (tcgen05.ld 32x32b), adds the bias and
-// writes them.  Every wait on the mbarrier is bounded: past the limit the CTA
+// One CTA of 256 threads owns 128 rows of X at a time (a persistent loop over
+// row tiles).  Per K chunk of 32 it copies (cp.async, 16 bytes per copy) the X
+// chunk [128 x 32] and the Wt chunk [C_out x 32] into shared memory as K-major
+// core matrices without swizzle (a core matrix is 8 rows x 16 bytes;
+// K-neighbouring core matrices are LBO bytes apart, 8-row groups SBO bytes
+// apart); the chunks are double-buffered, so the copies of chunk c + 1 run
+// while the tensor core works on chunk c.  Thread 0 issues four
+// M=128 x N=C_out x K=8 MMAs per chunk into a C_out-column float32 accumulator
+// in tensor memory and commits them to the buffer's mbarrier.  After the last
+// chunk the 8 warps read the accumulator (tcgen05.ld 32x32b; warp w takes rows
+// 32 (w % 4) .. + 31 and every other 16-column block), add the bias and write.  Every wait on the mbarrier is bounded: past the limit the CTA
 // sets a device flag (read by msda_output_projection_check) and stops,
 // releasing its tensor memory.
 #include <cstdint>
@@ -28,17 +30,19 @@ namespace msda {
 
 namespace {
 
-constexpr int kProjThreads = 128;
+constexpr int kProjThreads = 256;
 constexpr int kProjRows = 128;        // MMA M
 constexpr int kProjChunk = 32;        // K per staged chunk (4 MMAs of K = 8)
 constexpr int kProjMaxOut = 256;      // MMA N limit (one accumulator)
-// Shared memory: X chunk 128 x 32 floats (16 KB) + Wt chunk up to 256 x 32
-// floats (32 KB), plus padding that limits residency to 2 CTAs per SM, so two
-// 256-column accumulators always fit the SM's 512 tensor-memory columns.
+// Shared memory: two stages of an X chunk 128 x 32 floats (16 KB) and a Wt
+// chunk up to 256 x 32 floats (32 KB).  96 KB per CTA keeps residency at 2 CTAs
+// per SM, so two 256-column accumulators always fit the SM's 512 tensor-memory
+// columns.
 constexpr int kProjXBytes = kProjRows * kProjChunk * 4;
 constexpr int kProjWBytes = kProjMaxOut * kProjChunk * 4;
-constexpr int kProjSmemBytes = 80 * 1024;
-constexpr long long kProjWaitLimit = 1ll << 26;  // polls of the mbarrier before giving up
+constexpr int kProjStageBytes = kProjXBytes + kProjWBytes;
+constexpr int kProjSmemBytes = 2 * kProjStageBytes;
+constexpr long long kProjWaitLimit = 1ll << 26;  // polls of an mbarrier before giving up
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -83,14 +87,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t phase) {
   return done != 0;
 }
 
+// 16-byte asynchronous copy global -> shared; src_bytes = 0 writes zeros.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+
 __global__ void __launch_bounds__(kProjThreads)
 proj_kernel(const float* __restrict__ x, const float* __restrict__ wt,
             const float* __restrict__ bias, float* __restrict__ y, long long rows, int c_in,
             int c_out, int* __restrict__ status) {
   extern __shared__ __align__(1024) unsigned char smem[];
-  unsigned char* xs = smem;
-  unsigned char* ws = smem + kProjXBytes;
-  __shared__ __align__(8) uint64_t mma_done;
+  __shared__ __align__(8) uint64_t mma_done[2];  // one per staging buffer
   __shared__ uint32_t tmem_base;
   __shared__ int failed;
 
@@ -107,7 +116,8 @@ proj_kernel(const float* __restrict__ x, const float* __restrict__ wt,
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   if (tid == 0) {
-    mbar_init(&mma_done, 1);
+    mbar_init(&mma_done[0], 1);
+    mbar_init(&mma_done[1], 1);
     failed = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -117,39 +127,73 @@ proj_kernel(const float* __restrict__ x, const float* __restrict__ wt,
   const uint32_t tmem = tmem_base;
   const uint32_t idesc = tf32_idesc(c_out);
   const int n_pad = (c_out + 7) & ~7;  // rows of the Wt chunk (multiple of 8)
-  uint32_t phase = 0;
+  const int nch = (c_in + kProjChunk - 1) / kProjChunk;
+  uint32_t phase0 = 0u, phase1 = 0u;  // parity of each buffer's next completion
+
+  // Waits for the MMAs committed to buffer b's barrier (every thread), bounded.
+  auto wait_mma = [&](int b) {
+    const uint32_t ph = b ? phase1 : phase0;
+    long long polls = 0;
+    while (!mbar_try_wait(&mma_done[b], ph)) {
+      if (++polls > kProjWaitLimit) {
+        failed = 1;
+        break;
+      }
+    }
+    if (b)
+      phase1 ^= 1u;
+    else
+      phase0 ^= 1u;
+  };
+  // Issues the copies of K chunk c of row tile r0 into buffer b.
+  auto stage = [&](long long r0, int c, int b) {
+    const int k0 = c * kProjChunk;
+    const int kc = min(kProjChunk, c_in - k0);
+    const uint32_t xs = smem_u32(smem + b * kProjStageBytes);
+    const uint32_t ws = xs + kProjXBytes;
+    for (int i = tid; i < kProjRows * (kProjChunk / 4); i += kProjThreads) {
+      const int row = i / (kProjChunk / 4), kq = (i % (kProjChunk / 4)) * 4;
+      const bool in = r0 + row < rows && kq < kc;
+      const float* src = in ? x + (r0 + row) * c_in + k0 + kq : x;
+      cp_async16(xs + core_offset(row, kq, kProjRows), src, in ? 16 : 0);
+    }
+    for (int i = tid; i < n_pad * (kProjChunk / 4); i += kProjThreads) {
+      const int n = i / (kProjChunk / 4), kq = (i % (kProjChunk / 4)) * 4;
+      const bool in = n < c_out && kq < kc;
+      const float* src = in ? wt + static_cast<long long>(n) * c_in + k0 + kq : wt;
+      cp_async16(ws + core_offset(n, kq, n_pad), src, in ? 16 : 0);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
 
   const long long tiles = (rows + kProjRows - 1) / kProjRows;
-  for (long long tile = blockIdx.x; tile < tiles && !failed; tile += gridDim.x) {
+  if (blockIdx.x < tiles) stage(static_cast<long long>(blockIdx.x) * kProjRows, 0, 0);
+  for (long long tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
     const long long r0 = tile * kProjRows;
-    for (int k0 = 0; k0 < c_in; k0 += kProjChunk) {
-      const int kc = min(kProjChunk, c_in - k0);  // a multiple of 8
-      // Stage the chunks: X rows past the end and K past c_in read as zero.
-      for (int i = tid; i < kProjRows * (kProjChunk / 4); i += kProjThreads) {
-        const int row = i / (kProjChunk / 4), kq = (i % (kProjChunk / 4)) * 4;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (r0 + row < rows && kq < kc)
-          v = __ldg(reinterpret_cast<const float4*>(x + (r0 + row) * c_in + k0 + kq));
-        *reinterpret_cast<float4*>(xs + core_offset(row, kq, kProjRows)) = v;
+    // Chunk 0 of this tile was issued before the previous tile's epilogue.
+    for (int c = 0; c < nch; ++c) {
+      if (c + 1 < nch) {
+        // Buffer (c + 1) & 1 was read by chunk c - 1's MMAs.
+        if (c >= 1) wait_mma((c - 1) & 1);
+        stage(r0, c + 1, (c + 1) & 1);
+        asm volatile("cp.async.wait_group 1;" ::: "memory");  // chunk c has landed
+      } else {
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
       }
-      for (int i = tid; i < n_pad * (kProjChunk / 4); i += kProjThreads) {
-        const int n = i / (kProjChunk / 4), kq = (i % (kProjChunk / 4)) * 4;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (n < c_out && kq < kc)
-          v = __ldg(reinterpret_cast<const float4*>(wt + static_cast<long long>(n) * c_in + k0 + kq));
-        *reinterpret_cast<float4*>(ws + core_offset(n, kq, n_pad)) = v;
-      }
-      // The generic-proxy stores must be visible to the tensor core's reads.
+      // The copies must be visible to the tensor core's (async proxy) reads.
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       __syncthreads();
+      if (failed) break;
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
       if (tid == 0) {
-        const uint32_t xa = smem_u32(xs), wa = smem_u32(ws);
+        const int b = c & 1;
+        const int kc = min(kProjChunk, c_in - c * kProjChunk);
+        const uint32_t xa = smem_u32(smem + b * kProjStageBytes), wa = xa + kProjXBytes;
         for (int s = 0; s < kc / 8; ++s) {
           // K step s covers k groups 2s, 2s + 1.
           const uint64_t da = smem_desc(xa + 2 * s * kProjRows * 16, kProjRows * 16, 128);
           const uint64_t db = smem_desc(wa + 2 * s * n_pad * 16, n_pad * 16, 128);
-          const uint32_t accumulate = (k0 > 0 || s > 0) ? 1u : 0u;
+          const uint32_t accumulate = (c > 0 || s > 0) ? 1u : 0u;
           asm volatile(
               "{\n\t.reg .pred p;\n\t"
               "setp.ne.b32 p, %4, 0;\n\t"
@@ -160,26 +204,26 @@ proj_kernel(const float* __restrict__ x, const float* __restrict__ wt,
         }
         asm volatile(
             "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                smem_u32(&mma_done))
+                smem_u32(&mma_done[b]))
             : "memory");
       }
-      // Bounded wait for the MMAs (they also release the staged chunks).
-      long long polls = 0;
-      while (!mbar_try_wait(&mma_done, phase)) {
-        if (++polls > kProjWaitLimit) {
-          failed = 1;
-          break;
-        }
-      }
-      phase ^= 1u;
-      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      __syncthreads();
-      if (failed) break;
     }
+    // The commits not waited for inside the loop: chunks nch - 2 and nch - 1.
+    if (!failed) {
+      if (nch >= 2) wait_mma((nch - 2) & 1);
+      wait_mma((nch - 1) & 1);
+    }
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    __syncthreads();
     if (failed) break;
-    // Epilogue: warp w holds accumulator lanes (rows) 32w .. 32w + 31.
-    const long long r = r0 + warp * 32 + lane;
-    for (int c0 = 0; c0 < c_out; c0 += 16) {
+    // Both buffers are free again: the next tile's first chunk loads during
+    // this tile's epilogue.
+    if (tile + gridDim.x < tiles) stage((tile + gridDim.x) * kProjRows, 0, 0);
+    // Epilogue: warp w reads accumulator lanes (rows) 32 (w % 4) .. + 31 and
+    // every other 16-column block, starting at 16 (w / 4).
+    const int quarter = warp & 3;
+    const long long r = r0 + quarter * 32 + lane;
+    for (int c0 = (warp >> 2) * 16; c0 < c_out; c0 += 32) {
       uint32_t v[16];
       asm volatile(
           "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, "
@@ -187,23 +231,21 @@ proj_kernel(const float* __restrict__ x, const float* __restrict__ wt,
           : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
             "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
             "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
-          : "r"(tmem + (static_cast<uint32_t>(warp * 32) << 16) + static_cast<uint32_t>(c0)));
+          : "r"(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(c0)));
       asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
       if (r < rows) {
         float* dst = y + r * c_out + c0;
 #pragma unroll
         for (int j = 0; j < 16; j += 4) {
-          if (c0 + j < c_out) {
-            float4 o = make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
-                                   __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
-            if (bias != nullptr) {
-              o.x += __ldg(bias + c0 + j);
-              o.y += __ldg(bias + c0 + j + 1);
-              o.z += __ldg(bias + c0 + j + 2);
-              o.w += __ldg(bias + c0 + j + 3);
-            }
-            *reinterpret_cast<float4*>(dst + j) = o;
+          float4 o = make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
+                                 __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+          if (bias != nullptr) {
+            o.x += __ldg(bias + c0 + j);
+            o.y += __ldg(bias + c0 + j + 1);
+            o.z += __ldg(bias + c0 + j + 2);
+            o.w += __ldg(bias + c0 + j + 3);
           }
+          *reinterpret_cast<float4*>(dst + j) = o;
         }
       }
     }
@@ -212,6 +254,7 @@ proj_kernel(const float* __restrict__ x, const float* __restrict__ wt,
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   }
+  asm volatile("cp.async.wait_all;" ::: "memory");
   if (failed && tid == 0) atomicExch(status, 1);
   __syncthreads();
   if (warp == 0)
@@ -233,7 +276,7 @@ cudaError_t launch_projection(const float* x, const float* weight, const float* 
   int* status = nullptr;
   cudaError_t err0 = projection_failed_flag(&status);
   if (err0 != cudaSuccess) return err0;
-  static_assert(kProjXBytes + kProjWBytes <= kProjSmemBytes, "staging must fit");
+  static_assert(kProjSmemBytes <= 113 * 1024, "two CTAs per SM must fit");
   int dev = 0, sms = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
