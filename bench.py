@@ -488,7 +488,7 @@ def run_b200(args, world, rank, local):
     projection = {
         "workload": f"output_proj Linear {M * D}->{M * D} on the step's forward output "
                     f"({proj_rows} rows)",
-        "kernel": "proj_kernel: tcgen05.mma kind::tf32, accumulator in tensor memory",
+        "kernel": "proj_kernel: TMA loads/stores, tcgen05.mma kind::tf32, accumulators in tensor memory",
         "mean_ms": round(proj_ms, 4),
         "roofline": {"bound": "hbm", "achieved": round(proj_gbs, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(proj_gbs / peak, 4),
@@ -648,11 +648,24 @@ def run_case(args, local):
         inp = W.make_inputs(cfg, seed=0, with_grad=args.case.startswith("backward"))
         d = _device_inputs(inp, device)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    if args.case == "projection":
+        # output_proj on the op's output, with the weights the full bench uses.
+        px = binding.forward(d["value"], d["spatial_shapes"], d["level_start_index"],
+                             d["sampling_locations"], d["attention_weights"])
+        C = px.shape[-1]
+        px = px.reshape(-1, C)
+        prng = np.random.default_rng(1)
+        pw = torch.from_numpy((prng.standard_normal((C, C)) / np.sqrt(C)).astype(
+            np.float32)).to(device)
+        pb = torch.from_numpy(prng.standard_normal(C).astype(np.float32)).to(device)
+        py = torch.empty_like(px)
     fused_args = ("value", "spatial_shapes", "level_start_index", "reference_points",
                   "sampling_offsets", "attention_logits")
 
     def launch():
-        if args.case == "fused_forward":
+        if args.case == "projection":
+            binding.output_projection(px, pw, pb, out=py)
+        elif args.case == "fused_forward":
             binding.fused_forward(*[d[k] for k in fused_args])
         elif args.case == "fused_backward":
             binding.fused_backward(*[d[k] for k in fused_args], d["grad_output"],
@@ -730,7 +743,8 @@ def parse_args(argv=None):
     p.add_argument("--no-cpu-baseline", action="store_true",
                    help="skip the CPU oracle timing (it takes ~10-20 s)")
     p.add_argument("--case", choices=["step", "forward", "forward_encoder", "backward",
-                                      "backward_sorted", "fused_forward", "fused_backward"],
+                                      "backward_sorted", "fused_forward", "fused_backward",
+                                      "projection"],
                    default="step",
                    help="time one launch type alone (for profiler captures) instead of "
                         "the full benchmark")

@@ -200,17 +200,18 @@ msda_status msda_backward_deterministic_workspace_size(int64_t B, int64_t S, int
  *                            c_out % 16 == 0, 16 <= c_out <= 256)
  *   bias    [c_out]          float32, or NULL
  *   y       [rows, c_out]    float32, 16-byte aligned, written
- * rows == 0 launches nothing.  The kernel's waits for its MMAs are bounded;
- * if one ever runs out, its rows are left unwritten and
- * msda_output_projection_check reports it.
+ * rows == 0 launches nothing; rows above 2^31 - 129 give MSDA_ERR_UNSUPPORTED
+ * (TMA tile coordinates are 32-bit).  The kernel's waits (for its
+ * TMA copies, its MMAs and its epilogue) are bounded; if one ever runs out,
+ * some rows are left unwritten and msda_output_projection_check reports it.
  */
 msda_status msda_output_projection(int64_t rows, int64_t c_in, int64_t c_out, const float *x,
                                    const float *weight, const float *bias, float *y,
                                    void *stream);
 
 /*
- * *failed = 1 if a projection since the last check gave up waiting for its
- * MMAs, else 0; clears the flag.  Synchronises with the device (it copies the
+ * *failed = 1 if a projection since the last check gave up waiting (for a
+ * copy, an MMA or its epilogue), else 0; clears the flag.  Synchronises with the device (it copies the
  * flag to the host).
  */
 msda_status msda_output_projection_check(int *failed);

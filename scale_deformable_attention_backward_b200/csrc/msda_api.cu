@@ -280,7 +280,7 @@ msda_status msda_output_projection(int64_t rows, int64_t c_in, int64_t c_out, co
                                    void* stream) {
   if (rows < 0 || c_in < 0 || c_out < 0) return MSDA_ERR_BAD_SHAPE;
   if (c_in % 8 != 0 || c_in < 8 || c_in > 4096 || c_out % 16 != 0 || c_out < 16 ||
-      c_out > 256)
+      c_out > 256 || rows > static_cast<int64_t>(INT32_MAX) - 128)
     return MSDA_ERR_UNSUPPORTED;
   int64_t xe = 0, ye = 0;
   if (!product_ok({rows, c_in}, &xe) || !product_ok({rows, c_out}, &ye))

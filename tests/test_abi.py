@@ -254,6 +254,7 @@ def test_output_projection_arguments(lib):
     assert proj(rows=-1) == BAD
     assert proj(c_in=12) == UNSUP and proj(c_in=0) == UNSUP and proj(c_in=4104) == UNSUP
     assert proj(c_out=8) == UNSUP and proj(c_out=24) == UNSUP and proj(c_out=272) == UNSUP
+    assert proj(rows=2**31 - 128) == UNSUP  # past the TMA's 32-bit row coordinates
     assert proj(x=None) == NULLP and proj(w=None) == NULLP and proj(y=None) == NULLP
     assert proj(x=FAKE + 8) == MISAL and proj(w=FAKE + 4) == MISAL and proj(y=FAKE + 8) == MISAL
     assert proj(b=FAKE + 2) == MISAL

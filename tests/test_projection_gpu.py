@@ -36,7 +36,9 @@ def check(x, w, b, what):
 
 @pytest.mark.parametrize("rows,c_in,c_out", [
     (1, 8, 16), (127, 32, 16), (128, 256, 256), (129, 256, 256), (300, 40, 48),
-    (1000, 256, 128), (4096, 264, 256), (333, 4096, 32)])
+    (1000, 256, 128), (4096, 264, 256), (333, 4096, 32),
+    # several row tiles per CTA (both accumulators reused), ragged last tile
+    (40000, 96, 80), (80000, 256, 256)])
 def test_projection_random(rows, c_in, c_out):
     rng = np.random.default_rng(rows + c_in + c_out)
     x = rng.standard_normal((rows, c_in)).astype(np.float32)
