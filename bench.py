@@ -23,7 +23,8 @@ Printed (rank 0, one JSON line): the contract keys, plus
                  alone the same way, with its own roofline;
   e2e            the same metric through the public API with host buffers: the
                  H2D copy of every input and the D2H copy of every result are
-                 inside the timed region;
+                 inside the timed region; consecutive steps are pipelined over
+                 upload / compute / download streams;
   cpu_baseline   the float64 CPU oracle on a bounded sample (rank 0, N=1);
   clocks         SM clocks and throttle reasons sampled during the timed region.
 
@@ -562,43 +563,85 @@ def run_b200(args, world, rank, local):
                      "algorithmic_bytes": fbytes},
     }
 
-    # End to end through the public API with host buffers.
+    # End to end through the public API with host buffers.  Every step uploads
+    # its inputs from pinned host memory, runs forward + backward and downloads
+    # the output and the three gradients.  Steps are independent, so they are
+    # pipelined over three streams (upload, compute, download) with two device
+    # buffer sets: step i's upload overlaps step i-1's compute and step i-2's
+    # download.  PCIe carries host->device and device->host at once.
     pin = {k: torch.from_numpy(getattr(inp, k)).pin_memory() for k in
            ("value", "sampling_locations", "attention_weights", "grad_output")}
-    host_out = {k: torch.empty(t.shape, dtype=t.dtype).pin_memory() for k, t in
-                (("out", out), ("gv", gv), ("gl", gl), ("ga", ga))}
-    h2d = sum(t.numel() * t.element_size() for t in pin.values()) + \
-        inp.spatial_shapes.nbytes + inp.level_start_index.nbytes
-    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
-    ss_host = torch.from_numpy(inp.spatial_shapes)
-    st_host = torch.from_numpy(inp.level_start_index)
+    pin["spatial_shapes"] = torch.from_numpy(inp.spatial_shapes).pin_memory()
+    pin["level_start_index"] = torch.from_numpy(inp.level_start_index).pin_memory()
+    n_buf = 2
+    dev_in = [{k: torch.empty(t.shape, dtype=t.dtype, device=device) for k, t in pin.items()}
+              for _ in range(n_buf)]
+    out_shapes = (("out", out), ("gv", gv), ("gl", gl), ("ga", ga))
+    dev_out = [{k: torch.empty(t.shape, dtype=t.dtype, device=device) for k, t in out_shapes}
+               for _ in range(n_buf)]
+    host_out = [{k: torch.empty(t.shape, dtype=t.dtype).pin_memory() for k, t in out_shapes}
+                for _ in range(n_buf)]
+    h2d = sum(t.numel() * t.element_size() for t in pin.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out[0].values())
+    s_up, s_run, s_down = (torch.cuda.Stream(device) for _ in range(3))
+    ev_up = [torch.cuda.Event() for _ in range(n_buf)]
+    ev_run = [torch.cuda.Event() for _ in range(n_buf)]
+    ev_down = [torch.cuda.Event() for _ in range(n_buf)]
     e2e_steps = max(3, min(args.steps, 20))
 
-    def e2e_step():
-        dv = pin["value"].to(device, non_blocking=True)
-        dl = pin["sampling_locations"].to(device, non_blocking=True)
-        da = pin["attention_weights"].to(device, non_blocking=True)
-        dg = pin["grad_output"].to(device, non_blocking=True)
-        dss = ss_host.to(device, non_blocking=True)
-        dst = st_host.to(device, non_blocking=True)
-        o = binding.forward(dv, dss, dst, dl, da)
-        g = binding.backward(dv, dss, dst, dl, da, dg)
-        for (k, src) in zip(("out", "gv", "gl", "ga"), (o,) + tuple(g)):
-            host_out[k].copy_(src, non_blocking=True)
+    def e2e_step(i):
+        b = i % n_buf
+        di, do, ho = dev_in[b], dev_out[b], host_out[b]
+        with torch.cuda.stream(s_up):
+            if i >= n_buf:
+                s_up.wait_event(ev_run[b])      # step i - 2 no longer reads di
+            for k, t in pin.items():
+                di[k].copy_(t, non_blocking=True)
+            ev_up[b].record(s_up)
+        with torch.cuda.stream(s_run):
+            s_run.wait_event(ev_up[b])
+            if i >= n_buf:
+                s_run.wait_event(ev_down[b])    # step i - 2's results have left do
+            binding.forward(di["value"], di["spatial_shapes"], di["level_start_index"],
+                            di["sampling_locations"], di["attention_weights"],
+                            output=do["out"])
+            binding.backward(di["value"], di["spatial_shapes"], di["level_start_index"],
+                             di["sampling_locations"], di["attention_weights"],
+                             di["grad_output"], grad_value=do["gv"],
+                             grad_sampling_locations=do["gl"], grad_attention_weights=do["ga"])
+            ev_run[b].record(s_run)
+        with torch.cuda.stream(s_down):
+            s_down.wait_event(ev_run[b])
+            for k in ho:
+                ho[k].copy_(do[k], non_blocking=True)
+            ev_down[b].record(s_down)
 
-    for _ in range(2):
-        e2e_step()
+    for i in range(2 * n_buf):
+        e2e_step(i)
     torch.cuda.synchronize()
     barrier(world)
     ee0 = torch.cuda.Event(enable_timing=True)
     ee1 = torch.cuda.Event(enable_timing=True)
-    ee0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    ee1.record(stream)
+    ee0.record(s_up)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    # The last download is ordered after every earlier upload, launch and download.
+    ee1.record(s_down)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(ee0.elapsed_time(ee1), world, device) / e2e_steps
     barrier(world)
+    # The pipeline returns what one plain call on the device-resident inputs
+    # returns (the output and grad_sampling_locations do not depend on the order
+    # of atomics, so they must match bit for bit).
+    ref_out = binding.forward(d["value"], d["spatial_shapes"], d["level_start_index"],
+                              d["sampling_locations"], d["attention_weights"])
+    _, ref_gl, _ = binding.backward(d["value"], d["spatial_shapes"], d["level_start_index"],
+                                    d["sampling_locations"], d["attention_weights"],
+                                    d["grad_output"])
+    last = host_out[(e2e_steps - 1) % n_buf]
+    if not (torch.equal(last["out"], ref_out.cpu()) and torch.equal(last["gl"], ref_gl.cpu())):
+        raise RuntimeError("end-to-end pipeline results differ from a plain call's")
+    del ref_out, ref_gl
 
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": "queries/s", "n_gpus": world,
@@ -616,7 +659,8 @@ def run_b200(args, world, rank, local):
         "projection": projection,
         "e2e": {"value": round(world * queries / (e2e_ms * 1e-3), 1), "unit": "queries/s",
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": int(h2d),
-                "d2h_bytes_per_step": int(d2h)},
+                "d2h_bytes_per_step": int(d2h),
+                "pipeline": "upload / compute / download on three streams, two buffer sets"},
         "gpu_launches": (1 + BACKWARD_LAUNCHES) * args.steps,
         "clocks": clocks.summary(),
         "wall_s_timed_region": round(wall, 3),
