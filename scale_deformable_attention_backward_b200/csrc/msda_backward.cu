@@ -15,12 +15,9 @@
 //
 // (dx/dloc_x = W_l because x = loc_x * W_l - 0.5.)
 //
-// Decomposition as in the forward: a sub-warp of LANES lanes owns one (b, q, m);
-// each lane owns 4 channels.  Per point the lanes gather the four corners,
-// form their partial channel sums, reduce them with a butterfly of shuffles and
-// scatter the grad_value contributions with 16-byte vector atomics
-// (red.global.add.v4.f32).  Lane j keeps the reduced sums of point j of the
-// current round and writes them coalesced at the end of the round.
+// The grad_value contributions are scattered with 16-byte vector atomics
+// (red.global.add.v4.f32); the work decomposition is described at
+// backward_kernel.
 #include "msda_device.cuh"
 #include "msda_launch.h"
 
@@ -37,8 +34,30 @@ struct FixedHeader {
 };
 static_assert(sizeof(FixedHeader) <= kFixedHeaderBytes, "header must fit its slot");
 
+constexpr int kBwdThreads = 256;
+constexpr int kBwdPoints = 512;  // points set up per unit (two per thread)
+
 // T: dtype of value and grad_output (float32, or bfloat16 read 8 bytes per lane);
 // arithmetic and grad_value are float32 for both.
+//
+// Work decomposition.  A sub-warp of LANES lanes owns one (b, q, m) group and
+// each lane 4 of the head's channels, so a point corner is one 128-byte line of
+// grad_value for D = 32.  A block owns G = 256 / LANES consecutive groups and
+// walks their points in units of PC = 512 / G points per group:
+//   phase 1  each thread maps two of the unit's points once -- exact floor,
+//            corner validity, 32-bit corner offsets, the four weights
+//            A * bilinear and (fx, fy, A * W_l, A * H_l) -- into a swizzled
+//            shared table;
+//   phase 2  per point, each sub-warp reads the setup (broadcast), gathers its
+//            slice of the four corners, forms the four corner dot products
+//            G_ij = sum_d gO[d] V_ij[d] over its channels, scatters the
+//            grad_value contributions, and reduces G_00..G_11 over the lanes.
+//            Lane j keeps point j's sums; after each batch of LANES points every
+//            lane turns its point's G_ij into grad_attn and grad_loc:
+//              grad_attn = hy (hx G00 + fx G10) + fy (hx G01 + fx G11)
+//              grad_x    = A W_l (hy (G10 - G00) + fy (G11 - G01))
+//              grad_y    = A H_l (hx (G01 - G00) + fx (G11 - G10))
+// These are the derivatives above with the channel sum taken first.
 //
 // FIXED (the deterministic backward): each grad_value contribution A w_ij gO[d]
 // (the same float32 product as the default path) is multiplied by 2^e, rounded
@@ -51,7 +70,7 @@ static_assert(sizeof(FixedHeader) <= kFixedHeaderBytes, "header must fit its slo
 // not finite (header->fixed == 0) the kernel falls back to float atomics into
 // grad_value: the NaN / Inf pattern does not depend on the order either.
 template <typename T, int LANES, bool FIXED>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(kBwdThreads)
 backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial_shapes,
                 const int64_t* __restrict__ level_start_index,
                 const float* __restrict__ sampling_locations,
@@ -64,7 +83,14 @@ backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial
                 const FixedHeader* __restrict__ header) {
   using V = Vec4<T>;
   constexpr int E = 4;
+  constexpr int G = kBwdThreads / LANES;
+  constexpr int PC = kBwdPoints / G;
+  constexpr int PER = kBwdPoints / kBwdThreads;
+  static_assert(G >= 8, "the shared-memory swizzle needs at least 8 groups per block");
   __shared__ Levels lv;
+  __shared__ int4 s_off[kBwdPoints];
+  __shared__ float4 s_w[kBwdPoints];
+  __shared__ float4 s_g[kBwdPoints];
   stage_levels(lv, spatial_shapes, level_start_index, L, S);
   bool use_fixed = false;
   float scale = 1.0f;
@@ -75,13 +101,13 @@ backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial
   const int dq = D / 4;
 
   const int lane = threadIdx.x % LANES;
-  const int groups_per_block = blockDim.x / LANES;
+  const int gi = threadIdx.x / LANES;
   const int LK = L * K;
-  const long long MD = static_cast<long long>(M) * D;
+  const int MD = M * D;  // < 2^31: one image's value block is (checked by the C ABI)
+  const long long tiles = (groups + G - 1) / G;
 
-  for (long long g0 = static_cast<long long>(blockIdx.x) * groups_per_block; g0 < groups;
-       g0 += static_cast<long long>(gridDim.x) * groups_per_block) {
-    const long long g_raw = g0 + threadIdx.x / LANES;
+  for (long long tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+    const long long g_raw = tile * G + gi;
     const bool active = g_raw < groups;
     const Group grp = decompose(active ? g_raw : groups - 1, 1, M, Lq);
     const int ch = lane * E;
@@ -92,7 +118,7 @@ backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial
     unsigned long long* abase =
         FIXED ? fixed_acc + (grp.b * S * M + grp.m) * static_cast<long long>(D) + lane : nullptr;
     // grad_value corner at element offset o (relative to the (b, m, lane) base) += w gO.
-    auto scatter = [&](long long o, float w, const float (&g)[E]) {
+    auto scatter = [&](int o, float w, const float (&g)[E]) {
       if constexpr (FIXED) {
         if (use_fixed) {
 #pragma unroll
@@ -105,87 +131,99 @@ backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial
       atomicAdd(reinterpret_cast<float4*>(gvbase + o),
                 make_float4(w * g[0], w * g[1], w * g[2], w * g[3]));
     };
-    const float* gloc = sampling_locations + grp.bqm * LK * 2;
-    const float* gatt = attention_weights + grp.bqm * LK;
 
     float go[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) go[e] = 0.0f;
-    if (lane_on) V::load(grad_output + grp.bq * MD + static_cast<long long>(grp.m) * D + ch, go);
+    if (lane_on)
+      V::load(grad_output + grp.bq * static_cast<long long>(MD) + static_cast<long long>(grp.m) * D +
+                  ch,
+              go);
 
-    int l = 0, k = 0;
-    int H = lv.H[0], W = lv.W[0];
-    long long start = lv.start[0];
-    for (int p0 = 0; p0 < LK; p0 += LANES) {
-      const int pj = p0 + lane;
-      float2 xy = make_float2(0.0f, 0.0f);
-      float aj = 0.0f;
-      if (pj < LK) {
-        xy = __ldg(reinterpret_cast<const float2*>(gloc) + pj);
-        aj = __ldg(gatt + pj);
+    for (int q0 = 0; q0 < LK; q0 += PC) {
+      const int pc = min(PC, LK - q0);
+      // Phase 1: the unit's points, two per thread.
+#pragma unroll
+      for (int r = 0; r < PER; ++r) {
+        const int t = threadIdx.x + r * kBwdThreads;
+        const int tg = t / PC, tj = t % PC;
+        const long long g = tile * G + tg;
+        if (tj < pc && g < groups) {
+          const long long pidx = g * LK + q0 + tj;
+          const float2 xy = __ldg(reinterpret_cast<const float2*>(sampling_locations) + pidx);
+          const float a = __ldg(attention_weights + pidx);
+          const int l = (q0 + tj) / K;
+          const int H = lv.H[l], W = lv.W[l];
+          const Cell c = locate(xy.x, xy.y, H, W);
+          const float hx = 1.0f - c.fx, hy = 1.0f - c.fy;
+          // Offsets only for corners inside the map (0 <= pixel < S).
+          const int base = static_cast<int>(lv.start[l] + static_cast<long long>(c.y0) * W + c.x0);
+          int4 off;
+          off.x = (c.vx0 && c.vy0) ? base * MD : -1;
+          off.y = (c.vx1 && c.vy0) ? (base + 1) * MD : -1;
+          off.z = (c.vx0 && c.vy1) ? (base + W) * MD : -1;
+          off.w = (c.vx1 && c.vy1) ? (base + W + 1) * MD : -1;
+          const int slot = tj * G + (tg ^ (tj & 7));
+          s_off[slot] = off;
+          s_w[slot] = make_float4(a * hx * hy, a * c.fx * hy, a * hx * c.fy, a * c.fx * c.fy);
+          s_g[slot] = make_float4(c.fx, c.fy, a * static_cast<float>(W), a * static_cast<float>(H));
+        }
       }
-      float keep_attn = 0.0f, keep_x = 0.0f, keep_y = 0.0f;
-      const int n = min(LANES, LK - p0);
-      for (int j = 0; j < n; ++j) {
-        const float lx = __shfl_sync(kFullMask, xy.x, j, LANES);
-        const float ly = __shfl_sync(kFullMask, xy.y, j, LANES);
-        const float a = __shfl_sync(kFullMask, aj, j, LANES);
-        const Cell c = locate(lx, ly, H, W);
-        const float hx = 1.0f - c.fx, hy = 1.0f - c.fy;
-        const long long row = static_cast<long long>(W) * MD;
-        const long long off = (start + static_cast<long long>(c.y0) * W + c.x0) * MD;
-        const bool v00 = c.vx0 && c.vy0, v10 = c.vx1 && c.vy0;
-        const bool v01 = c.vx0 && c.vy1, v11 = c.vx1 && c.vy1;
-        float s_attn = 0.0f, s_x = 0.0f, s_y = 0.0f;
-        if (lane_on) {
-          // Corner naming: q<i><j> = V(x0 + i, y0 + j).
-          float q00[E], q10[E], q01[E], q11[E];
+      __syncthreads();
+
+      // Phase 2: gathers, scatters and the corner dot products.
+      for (int j0 = 0; j0 < pc; j0 += LANES) {
+        const int nb = min(LANES, pc - j0);
+        float keep[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        for (int jj = 0; jj < nb; ++jj) {
+          const int j = j0 + jj;
+          const int slot = j * G + (gi ^ (j & 7));
+          const int4 o = s_off[slot];
+          float dot[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+          if (lane_on) {
+            const float4 w = s_w[slot];
+            const int os[4] = {o.x, o.y, o.z, o.w};
+            const float ws[4] = {w.x, w.y, w.z, w.w};
+            float q[4][E];
 #pragma unroll
-          for (int e = 0; e < E; ++e) q00[e] = q10[e] = q01[e] = q11[e] = 0.0f;
-          if (v00) V::load(vbase + off, q00);
-          if (v10) V::load(vbase + off + MD, q10);
-          if (v01) V::load(vbase + off + row, q01);
-          if (v11) V::load(vbase + off + row + MD, q11);
+            for (int i = 0; i < 4; ++i) {
 #pragma unroll
-          for (int e = 0; e < E; ++e) {
-            const float top = fmaf(c.fx, q10[e], hx * q00[e]);
-            const float bot = fmaf(c.fx, q11[e], hx * q01[e]);
-            s_attn = fmaf(go[e], fmaf(c.fy, bot, hy * top), s_attn);
-            s_x = fmaf(go[e], fmaf(c.fy, q11[e] - q01[e], hy * (q10[e] - q00[e])), s_x);
-            s_y = fmaf(go[e], fmaf(c.fx, q11[e] - q10[e], hx * (q01[e] - q00[e])), s_y);
+              for (int e = 0; e < E; ++e) q[i][e] = 0.0f;
+              if (os[i] >= 0) V::load(vbase + os[i], q[i]);
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+#pragma unroll
+              for (int e = 0; e < E; ++e) dot[i] = fmaf(go[e], q[i][e], dot[i]);
+              if (os[i] >= 0) scatter(os[i], ws[i], go);
+            }
           }
-          const float w00 = a * hx * hy, w10 = a * c.fx * hy;
-          const float w01 = a * hx * c.fy, w11 = a * c.fx * c.fy;
-          if (v00) scatter(off, w00, go);
-          if (v10) scatter(off + MD, w10, go);
-          if (v01) scatter(off + row, w01, go);
-          if (v11) scatter(off + row + MD, w11, go);
-        }
 #pragma unroll
-        for (int o = LANES / 2; o > 0; o >>= 1) {
-          s_attn += __shfl_xor_sync(kFullMask, s_attn, o, LANES);
-          s_x += __shfl_xor_sync(kFullMask, s_x, o, LANES);
-          s_y += __shfl_xor_sync(kFullMask, s_y, o, LANES);
-        }
-        if (lane == j) {
-          keep_attn = s_attn;
-          keep_x = a * static_cast<float>(W) * s_x;
-          keep_y = a * static_cast<float>(H) * s_y;
-        }
-        if (++k == K) {
-          k = 0;
-          if (++l < L) {
-            H = lv.H[l];
-            W = lv.W[l];
-            start = lv.start[l];
+          for (int sh = LANES / 2; sh > 0; sh >>= 1) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dot[i] += __shfl_xor_sync(kFullMask, dot[i], sh, LANES);
+          }
+          if (lane == jj) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) keep[i] = dot[i];
           }
         }
+        if (active && lane < nb) {
+          const int j = j0 + lane;
+          const float4 gg = s_g[j * G + (gi ^ (j & 7))];
+          const float fx = gg.x, fy = gg.y, hx = 1.0f - fx, hy = 1.0f - fy;
+          const float s_attn = fmaf(hy, fmaf(fx, keep[1], hx * keep[0]),
+                                    fy * fmaf(fx, keep[3], hx * keep[2]));
+          const float s_x = fmaf(hy, keep[1] - keep[0], fy * (keep[3] - keep[2]));
+          const float s_y = fmaf(hx, keep[2] - keep[0], fx * (keep[3] - keep[1]));
+          const long long pidx = grp.bqm * LK + q0 + j;
+          grad_attention_weights[pidx] = s_attn;
+          reinterpret_cast<float2*>(grad_sampling_locations)[pidx] =
+              make_float2(gg.z * s_x, gg.w * s_y);
+        }
       }
-      if (active && pj < LK) {
-        grad_attention_weights[grp.bqm * LK + pj] = keep_attn;
-        reinterpret_cast<float2*>(grad_sampling_locations + grp.bqm * LK * 2)[pj] =
-            make_float2(keep_x, keep_y);
-      }
+      // The next unit's setup overwrites the table.
+      __syncthreads();
     }
   }
 }
@@ -303,11 +341,10 @@ __global__ void fixed_to_float_kernel(const unsigned long long* __restrict__ acc
 template <typename T, int LANES, bool FIXED>
 static cudaError_t launch_backward_t(const BackwardArgs& a, unsigned long long* acc,
                                      const FixedHeader* header, cudaStream_t stream) {
-  constexpr int kThreads = 256;
-  const long long per_block = kThreads / LANES;
+  const long long per_block = kBwdThreads / LANES;
   long long blocks = (a.groups + per_block - 1) / per_block;
   if (blocks > (1ll << 30)) blocks = 1ll << 30;
-  backward_kernel<T, LANES, FIXED><<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(
+  backward_kernel<T, LANES, FIXED><<<static_cast<unsigned>(blocks), kBwdThreads, 0, stream>>>(
       static_cast<const T*>(a.value), a.spatial_shapes, a.level_start_index,
       a.sampling_locations, a.attention_weights, static_cast<const T*>(a.grad_output),
       a.grad_value, a.grad_sampling_locations, a.grad_attention_weights, a.S, a.M, a.D, a.Lq,
