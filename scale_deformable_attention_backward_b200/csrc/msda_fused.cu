@@ -141,13 +141,16 @@ fused_forward_kernel(const T* __restrict__ value, const int64_t* __restrict__ sp
   }
 }
 
-// Backward: the scratch-free backward of msda_backward.cu (a sub-warp per
-// (b, q, m), four corner gathers and one 16-byte vector atomic per lane and
-// corner for each point) with the locations and weights formed from the raw
-// inputs, and the chain rule through them applied per point.  grad_logits
-// holds dA until the group's sum_j A_j dA_j is known, then d z.
+// Backward: the two phases of msda_backward.cu's backward_kernel with the
+// locations and weights formed from the raw inputs in phase 1, and the chain
+// rule through them applied per point when its corner dot products are
+// complete.  Per tile, each group's lanes first compute its softmax normaliser
+// (max and 1 / sum) into shared memory, so that any thread can form any of the
+// tile's weights.  grad_logits holds dA until the group's sum_j A_j dA_j is
+// known, then d z.  Lane i of a group combines (and later revisits) the points
+// p with p % LANES == i.
 template <int LANES>
-__global__ void __launch_bounds__(kThreads, 3)  // 3 blocks per SM, as the core backward
+__global__ void __launch_bounds__(kThreads)
 fused_backward_kernel(const float* __restrict__ value, const int64_t* __restrict__ spatial_shapes,
                       const int64_t* __restrict__ level_start_index,
                       const float* __restrict__ reference_points,
@@ -159,18 +162,27 @@ fused_backward_kernel(const float* __restrict__ value, const int64_t* __restrict
                       long long Lq, int L, int K, int R, long long groups) {
   using V = Vec<float>;
   constexpr int E = V::N;
+  constexpr int G = kThreads / LANES;
+  constexpr int PC = kChunkPoints / G;
+  constexpr int PER = kChunkPoints / kThreads;
+  static_assert(G >= 8, "the shared-memory swizzle needs at least 8 groups per block");
+  static_assert(PC % LANES == 0, "a lane must own the same points in every unit");
   __shared__ Levels lv;
+  __shared__ int4 s_off[kChunkPoints];
+  __shared__ float4 s_w[kChunkPoints];
+  __shared__ float4 s_g[kChunkPoints];  // fx, fy, A, 0
+  __shared__ float2 s_norm[G];
   stage_levels(lv, spatial_shapes, level_start_index, L, S);
 
   const int lane = threadIdx.x % LANES;
-  const int groups_per_block = blockDim.x / LANES;
+  const int gi = threadIdx.x / LANES;
   const int LK = L * K;
-  const long long MD = static_cast<long long>(M) * D;
+  const int MD = M * D;  // < 2^31: one image's value block is (checked by the C ABI)
   const float half_over_k = 0.5f / static_cast<float>(K);
+  const long long tiles = (groups + G - 1) / G;
 
-  for (long long g0 = static_cast<long long>(blockIdx.x) * groups_per_block; g0 < groups;
-       g0 += static_cast<long long>(gridDim.x) * groups_per_block) {
-    const long long g_raw = g0 + threadIdx.x / LANES;
+  for (long long tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+    const long long g_raw = tile * G + gi;
     const bool active = g_raw < groups;
     const Group grp = decompose(active ? g_raw : groups - 1, 1, M, Lq);
     const int ch = lane * E;
@@ -180,111 +192,126 @@ fused_backward_kernel(const float* __restrict__ value, const int64_t* __restrict
     float* gvbase = grad_value + vofs;
     const float* zg = attention_logits + grp.bqm * LK;
     const float2 nz = softmax_norm<LANES>(zg, LK, lane);
+    if (lane == 0) s_norm[gi] = nz;
 
     float go[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) go[e] = 0.0f;
-    if (lane_on) V::load(grad_output + grp.bq * MD + static_cast<long long>(grp.m) * D + ch, go);
-
+    if (lane_on)
+      V::load(grad_output + grp.bq * static_cast<long long>(MD) + static_cast<long long>(grp.m) * D +
+                  ch,
+              go);
     float sum_adA = 0.0f;  // this lane's share of sum_j A_j dA_j
-    int l = 0, k = 0;
-    int H = lv.H[0], W = lv.W[0];
-    long long start = lv.start[0];
-    for (int p0 = 0; p0 < LK; p0 += LANES) {
-      const int pj = p0 + lane;
-      const int lj = pj / K;
-      float2 xy = make_float2(0.0f, 0.0f), offj = make_float2(0.0f, 0.0f);
-      float aj = 0.0f;
-      if (pj < LK) {
-        offj = __ldg(reinterpret_cast<const float2*>(sampling_offsets) + grp.bqm * LK + pj);
-        xy = fused_location(reference_points + (grp.bq * L + lj) * R, offj, R, lv.W[lj],
-                            lv.H[lj], K);
-        aj = expf(__ldg(zg + pj) - nz.x) * nz.y;
-      }
-      float keep_attn = 0.0f, keep_x = 0.0f, keep_y = 0.0f;
-      const int n = min(LANES, LK - p0);
-      for (int j = 0; j < n; ++j) {
-        const float lx = __shfl_sync(kFullMask, xy.x, j, LANES);
-        const float ly = __shfl_sync(kFullMask, xy.y, j, LANES);
-        const float a = __shfl_sync(kFullMask, aj, j, LANES);
-        const Cell c = locate(lx, ly, H, W);
-        const float hx = 1.0f - c.fx, hy = 1.0f - c.fy;
-        const long long row = static_cast<long long>(W) * MD;
-        const long long off = (start + static_cast<long long>(c.y0) * W + c.x0) * MD;
-        const bool v00 = c.vx0 && c.vy0, v10 = c.vx1 && c.vy0;
-        const bool v01 = c.vx0 && c.vy1, v11 = c.vx1 && c.vy1;
-        float s_attn = 0.0f, s_x = 0.0f, s_y = 0.0f;
-        if (lane_on) {
-          float q00[E], q10[E], q01[E], q11[E];
+    __syncthreads();       // s_norm is complete
+
+    for (int q0 = 0; q0 < LK; q0 += PC) {
+      const int pc = min(PC, LK - q0);
+      // Phase 1: locations, weights and cells of the unit's points.
 #pragma unroll
-          for (int e = 0; e < E; ++e) q00[e] = q10[e] = q01[e] = q11[e] = 0.0f;
-          if (v00) V::load(vbase + off, q00);
-          if (v10) V::load(vbase + off + MD, q10);
-          if (v01) V::load(vbase + off + row, q01);
-          if (v11) V::load(vbase + off + row + MD, q11);
-#pragma unroll
-          for (int e = 0; e < E; ++e) {
-            const float top = fmaf(c.fx, q10[e], hx * q00[e]);
-            const float bot = fmaf(c.fx, q11[e], hx * q01[e]);
-            s_attn = fmaf(go[e], fmaf(c.fy, bot, hy * top), s_attn);
-            s_x = fmaf(go[e], fmaf(c.fy, q11[e] - q01[e], hy * (q10[e] - q00[e])), s_x);
-            s_y = fmaf(go[e], fmaf(c.fx, q11[e] - q10[e], hx * (q01[e] - q00[e])), s_y);
-          }
-          const float w00 = a * hx * hy, w10 = a * c.fx * hy;
-          const float w01 = a * hx * c.fy, w11 = a * c.fx * c.fy;
-          if (v00) atomicAdd(reinterpret_cast<float4*>(gvbase + off),
-                             make_float4(w00 * go[0], w00 * go[1], w00 * go[2], w00 * go[3]));
-          if (v10) atomicAdd(reinterpret_cast<float4*>(gvbase + off + MD),
-                             make_float4(w10 * go[0], w10 * go[1], w10 * go[2], w10 * go[3]));
-          if (v01) atomicAdd(reinterpret_cast<float4*>(gvbase + off + row),
-                             make_float4(w01 * go[0], w01 * go[1], w01 * go[2], w01 * go[3]));
-          if (v11) atomicAdd(reinterpret_cast<float4*>(gvbase + off + row + MD),
-                             make_float4(w11 * go[0], w11 * go[1], w11 * go[2], w11 * go[3]));
-        }
-#pragma unroll
-        for (int o = LANES / 2; o > 0; o >>= 1) {
-          s_attn += __shfl_xor_sync(kFullMask, s_attn, o, LANES);
-          s_x += __shfl_xor_sync(kFullMask, s_x, o, LANES);
-          s_y += __shfl_xor_sync(kFullMask, s_y, o, LANES);
-        }
-        if (lane == j) {
-          keep_attn = s_attn;
-          keep_x = a * s_x;  // grad_loc.x / W of this point
-          keep_y = a * s_y;  // grad_loc.y / H
-        }
-        if (++k == K) {
-          k = 0;
-          if (++l < L) {
-            H = lv.H[l];
-            W = lv.W[l];
-            start = lv.start[l];
-          }
+      for (int r = 0; r < PER; ++r) {
+        const int t = threadIdx.x + r * kThreads;
+        const int tg = t / PC, tj = t % PC;
+        const long long g = tile * G + tg;
+        if (tj < pc && g < groups) {
+          const long long pidx = g * LK + q0 + tj;
+          const int l = (q0 + tj) / K;
+          const int H = lv.H[l], W = lv.W[l];
+          const float2 offj = __ldg(reinterpret_cast<const float2*>(sampling_offsets) + pidx);
+          const long long bq = g / M;
+          const float2 xy = fused_location(reference_points + (bq * L + l) * R, offj, R, W, H, K);
+          const float2 n = s_norm[tg];
+          const float a = expf(__ldg(attention_logits + pidx) - n.x) * n.y;
+          const Cell c = locate(xy.x, xy.y, H, W);
+          const float hx = 1.0f - c.fx, hy = 1.0f - c.fy;
+          // Offsets only for corners inside the map (0 <= pixel < S).
+          const int base = static_cast<int>(lv.start[l] + static_cast<long long>(c.y0) * W + c.x0);
+          int4 off;
+          off.x = (c.vx0 && c.vy0) ? base * MD : -1;
+          off.y = (c.vx1 && c.vy0) ? (base + 1) * MD : -1;
+          off.z = (c.vx0 && c.vy1) ? (base + W) * MD : -1;
+          off.w = (c.vx1 && c.vy1) ? (base + W + 1) * MD : -1;
+          const int slot = tj * G + (tg ^ (tj & 7));
+          s_off[slot] = off;
+          s_w[slot] = make_float4(a * hx * hy, a * c.fx * hy, a * hx * c.fy, a * c.fx * c.fy);
+          s_g[slot] = make_float4(c.fx, c.fy, a, 0.0f);
         }
       }
-      if (active && pj < LK) {
-        const long long p = grp.bqm * LK + pj;
-        sum_adA = fmaf(aj, keep_attn, sum_adA);
-        grad_logits[p] = keep_attn;  // dA for now
-        const float Wj = static_cast<float>(lv.W[lj]), Hj = static_cast<float>(lv.H[lj]);
-        const float gx = keep_x * Wj, gy = keep_y * Hj;  // grad_loc
-        float2 goff;
-        if (R == 2) {
-          goff = make_float2(keep_x, keep_y);
-        } else {
+      __syncthreads();
+
+      // Phase 2: gathers, scatters, corner dot products, and the chain rule.
+      for (int j0 = 0; j0 < pc; j0 += LANES) {
+        const int nb = min(LANES, pc - j0);
+        float keep[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        for (int jj = 0; jj < nb; ++jj) {
+          const int j = j0 + jj;
+          const int slot = j * G + (gi ^ (j & 7));
+          const int4 o = s_off[slot];
+          float dot[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+          if (lane_on) {
+            const float4 w = s_w[slot];
+            const int os[4] = {o.x, o.y, o.z, o.w};
+            const float ws[4] = {w.x, w.y, w.z, w.w};
+            float q[4][E];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+#pragma unroll
+              for (int e = 0; e < E; ++e) q[i][e] = 0.0f;
+              if (os[i] >= 0) V::load(vbase + os[i], q[i]);
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+#pragma unroll
+              for (int e = 0; e < E; ++e) dot[i] = fmaf(go[e], q[i][e], dot[i]);
+              if (os[i] >= 0)
+                atomicAdd(reinterpret_cast<float4*>(gvbase + os[i]),
+                          make_float4(ws[i] * go[0], ws[i] * go[1], ws[i] * go[2], ws[i] * go[3]));
+            }
+          }
+#pragma unroll
+          for (int sh = LANES / 2; sh > 0; sh >>= 1) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dot[i] += __shfl_xor_sync(kFullMask, dot[i], sh, LANES);
+          }
+          if (lane == jj) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) keep[i] = dot[i];
+          }
+        }
+        if (active && lane < nb) {
+          const int pj = q0 + j0 + lane;
+          const long long p = grp.bqm * LK + pj;
+          const int lj = pj / K;
+          const float4 gg = s_g[(j0 + lane) * G + (gi ^ ((j0 + lane) & 7))];
+          const float fx = gg.x, fy = gg.y, hx = 1.0f - fx, hy = 1.0f - fy, a = gg.z;
+          const float dA = fmaf(hy, fmaf(fx, keep[1], hx * keep[0]),
+                                fy * fmaf(fx, keep[3], hx * keep[2]));
+          const float s_x = fmaf(hy, keep[1] - keep[0], fy * (keep[3] - keep[2]));
+          const float s_y = fmaf(hx, keep[2] - keep[0], fx * (keep[3] - keep[1]));
+          sum_adA = fmaf(a, dA, sum_adA);
+          grad_logits[p] = dA;  // dA for now
+          const float kx = a * s_x, ky = a * s_y;  // grad_loc / (W, H)
+          const float gx = kx * static_cast<float>(lv.W[lj]);
+          const float gy = ky * static_cast<float>(lv.H[lj]);
           const float* rp = reference_points + (grp.bq * L + lj) * R;
-          goff = make_float2(gx * __ldg(rp + 2) * half_over_k, gy * __ldg(rp + 3) * half_over_k);
-        }
-        reinterpret_cast<float2*>(grad_offsets)[p] = goff;
-        if (grad_reference != nullptr) {
-          float* gr = grad_reference + (grp.bq * L + lj) * R;
-          atomicAdd(gr + 0, gx);
-          atomicAdd(gr + 1, gy);
-          if (R == 4) {
-            atomicAdd(gr + 2, gx * offj.x * half_over_k);
-            atomicAdd(gr + 3, gy * offj.y * half_over_k);
+          float2 goff;
+          if (R == 2)
+            goff = make_float2(kx, ky);
+          else
+            goff = make_float2(gx * __ldg(rp + 2) * half_over_k, gy * __ldg(rp + 3) * half_over_k);
+          reinterpret_cast<float2*>(grad_offsets)[p] = goff;
+          if (grad_reference != nullptr) {
+            float* gr = grad_reference + (grp.bq * L + lj) * R;
+            atomicAdd(gr + 0, gx);
+            atomicAdd(gr + 1, gy);
+            if (R == 4) {
+              const float2 offj = __ldg(reinterpret_cast<const float2*>(sampling_offsets) + p);
+              atomicAdd(gr + 2, gx * offj.x * half_over_k);
+              atomicAdd(gr + 3, gy * offj.y * half_over_k);
+            }
           }
         }
       }
+      __syncthreads();  // the table and s_norm are rewritten next
     }
     // Softmax Jacobian: d z_j = A_j (dA_j - sum_i A_i dA_i).  Each lane revisits
     // the points it wrote.
