@@ -49,15 +49,18 @@ constexpr int kBwdPoints = 512;  // points set up per unit (two per thread)
 //            A * bilinear and (fx, fy, A * W_l, A * H_l) -- into a swizzled
 //            shared table;
 //   phase 2  per point, each sub-warp reads the setup (broadcast), gathers its
-//            slice of the four corners, forms the four corner dot products
-//            G_ij = sum_d gO[d] V_ij[d] over its channels, scatters the
-//            grad_value contributions, and reduces G_00..G_11 over the lanes.
-//            Lane j keeps point j's sums; after each batch of LANES points every
-//            lane turns its point's G_ij into grad_attn and grad_loc:
-//              grad_attn = hy (hx G00 + fx G10) + fy (hx G01 + fx G11)
-//              grad_x    = A W_l (hy (G10 - G00) + fy (G11 - G01))
-//              grad_y    = A H_l (hx (G01 - G00) + fx (G11 - G10))
-// These are the derivatives above with the channel sum taken first.
+//            slice of the four corners, scatters the grad_value contributions,
+//            and forms over its channels the four dot products
+//              P  = sum_d gO V00,          Ex = sum_d gO (V10 - V00),
+//              Ey = sum_d gO (V01 - V00),  Exy = sum_d gO (V11 - V01 - V10 + V00)
+//            (differences taken per channel, so a common offset of the value
+//            field cancels exactly), then reduces them over the lanes.  Lane j
+//            keeps point j's sums; after each batch of LANES points every lane
+//            turns its point's sums into
+//              grad_attn = P + fx Ex + fy Ey + fx fy Exy
+//              grad_x    = A W_l (Ex + fy Exy)
+//              grad_y    = A H_l (Ey + fx Exy)
+// These are the derivatives above, regrouped with hx + fx = hy + fy = 1.
 //
 // FIXED (the deterministic backward): each grad_value contribution A w_ij gO[d]
 // (the same float32 product as the default path) is multiplied by 2^e, rounded
@@ -192,9 +195,19 @@ backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial
               if (os[i] >= 0) V::load(vbase + os[i], q[i]);
             }
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
+            for (int e = 0; e < E; ++e) {
+              // Corner differences per channel: a common offset of the value
+              // field cancels here exactly, not between large dot products.
+              const float dx = q[1][e] - q[0][e];            // V10 - V00
+              const float dy = q[2][e] - q[0][e];            // V01 - V00
+              const float dxy = (q[3][e] - q[2][e]) - dx;    // V11 - V01 - V10 + V00
+              dot[0] = fmaf(go[e], q[0][e], dot[0]);
+              dot[1] = fmaf(go[e], dx, dot[1]);
+              dot[2] = fmaf(go[e], dy, dot[2]);
+              dot[3] = fmaf(go[e], dxy, dot[3]);
+            }
 #pragma unroll
-              for (int e = 0; e < E; ++e) dot[i] = fmaf(go[e], q[i][e], dot[i]);
+            for (int i = 0; i < 4; ++i) {
               if (os[i] >= 0) scatter(os[i], ws[i], go);
             }
           }
@@ -211,11 +224,10 @@ backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial
         if (active && lane < nb) {
           const int j = j0 + lane;
           const float4 gg = s_g[j * G + (gi ^ (j & 7))];
-          const float fx = gg.x, fy = gg.y, hx = 1.0f - fx, hy = 1.0f - fy;
-          const float s_attn = fmaf(hy, fmaf(fx, keep[1], hx * keep[0]),
-                                    fy * fmaf(fx, keep[3], hx * keep[2]));
-          const float s_x = fmaf(hy, keep[1] - keep[0], fy * (keep[3] - keep[2]));
-          const float s_y = fmaf(hx, keep[2] - keep[0], fx * (keep[3] - keep[1]));
+          const float fx = gg.x, fy = gg.y;
+          const float s_attn = fmaf(fx, fmaf(fy, keep[3], keep[1]), fmaf(fy, keep[2], keep[0]));
+          const float s_x = fmaf(fy, keep[3], keep[1]);
+          const float s_y = fmaf(fx, keep[3], keep[2]);
           const long long pidx = grp.bqm * LK + q0 + j;
           grad_attention_weights[pidx] = s_attn;
           reinterpret_cast<float2*>(grad_sampling_locations)[pidx] =

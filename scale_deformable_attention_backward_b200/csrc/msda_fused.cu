@@ -143,8 +143,8 @@ fused_forward_kernel(const T* __restrict__ value, const int64_t* __restrict__ sp
 
 // Backward: the two phases of msda_backward.cu's backward_kernel with the
 // locations and weights formed from the raw inputs in phase 1, and the chain
-// rule through them applied per point when its corner dot products are
-// complete.  Per tile, each group's lanes first compute its softmax normaliser
+// rule through them applied per point when its four dot products (P, Ex, Ey,
+// Exy: the value and its corner differences against gO) are complete.  Per tile, each group's lanes first compute its softmax normaliser
 // (max and 1 / sum) into shared memory, so that any thread can form any of the
 // tile's weights.  grad_logits holds dA until the group's sum_j A_j dA_j is
 // known, then d z.  Lane i of a group combines (and later revisits) the points
@@ -259,9 +259,19 @@ fused_backward_kernel(const float* __restrict__ value, const int64_t* __restrict
               if (os[i] >= 0) V::load(vbase + os[i], q[i]);
             }
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
+            for (int e = 0; e < E; ++e) {
+              // Corner differences per channel: a common offset of the value
+              // field cancels here exactly, not between large dot products.
+              const float dx = q[1][e] - q[0][e];            // V10 - V00
+              const float dy = q[2][e] - q[0][e];            // V01 - V00
+              const float dxy = (q[3][e] - q[2][e]) - dx;    // V11 - V01 - V10 + V00
+              dot[0] = fmaf(go[e], q[0][e], dot[0]);
+              dot[1] = fmaf(go[e], dx, dot[1]);
+              dot[2] = fmaf(go[e], dy, dot[2]);
+              dot[3] = fmaf(go[e], dxy, dot[3]);
+            }
 #pragma unroll
-              for (int e = 0; e < E; ++e) dot[i] = fmaf(go[e], q[i][e], dot[i]);
+            for (int i = 0; i < 4; ++i) {
               if (os[i] >= 0)
                 atomicAdd(reinterpret_cast<float4*>(gvbase + os[i]),
                           make_float4(ws[i] * go[0], ws[i] * go[1], ws[i] * go[2], ws[i] * go[3]));
@@ -282,11 +292,10 @@ fused_backward_kernel(const float* __restrict__ value, const int64_t* __restrict
           const long long p = grp.bqm * LK + pj;
           const int lj = pj / K;
           const float4 gg = s_g[(j0 + lane) * G + (gi ^ ((j0 + lane) & 7))];
-          const float fx = gg.x, fy = gg.y, hx = 1.0f - fx, hy = 1.0f - fy, a = gg.z;
-          const float dA = fmaf(hy, fmaf(fx, keep[1], hx * keep[0]),
-                                fy * fmaf(fx, keep[3], hx * keep[2]));
-          const float s_x = fmaf(hy, keep[1] - keep[0], fy * (keep[3] - keep[2]));
-          const float s_y = fmaf(hx, keep[2] - keep[0], fx * (keep[3] - keep[1]));
+          const float fx = gg.x, fy = gg.y, a = gg.z;
+          const float dA = fmaf(fx, fmaf(fy, keep[3], keep[1]), fmaf(fy, keep[2], keep[0]));
+          const float s_x = fmaf(fy, keep[3], keep[1]);
+          const float s_y = fmaf(fx, keep[3], keep[2]);
           sum_adA = fmaf(a, dA, sum_adA);
           grad_logits[p] = dA;  // dA for now
           const float kx = a * s_x, ky = a * s_y;  // grad_loc / (W, H)

@@ -52,6 +52,19 @@ def test_random_shapes_f32(D, shapes_id):
     G.check_backward_paths(d, inp)
 
 
+@pytest.mark.parametrize("offset", [100.0, -1000.0])
+def test_value_with_large_common_offset(offset):
+    """value = offset + N(0, 1): the backward forms grad_loc from differences of
+    corner dot products (G10 - G00 ...), whose common part cancels.  The result
+    must still meet the float32 backward tolerance against the oracle, on every
+    backward path."""
+    inp = random_inputs(31, B=2, M=4, D=32, K=4, shapes=SHAPES[2], Lq=45)
+    inp = dataclasses.replace(inp, value=np.ascontiguousarray(inp.value + np.float32(offset)))
+    d = G.device_inputs(inp)
+    G.assert_forward_f32(G.gpu_forward(d), G.oracle_forward(inp), f"forward offset={offset}")
+    G.check_backward_paths(d, inp)
+
+
 @pytest.mark.parametrize("D", [256, 384])
 def test_forward_channel_chunks_f32(D):
     """More than 32 lanes' worth of channels: several chunks per head."""
