@@ -415,6 +415,8 @@ def output_projection(x: torch.Tensor, weight: torch.Tensor, bias: Optional[torc
     ``x [..., c_in] @ weight[c_out, c_in].T + bias``, float32 in and out (TF32
     products, float32 sums)."""
     dev = x.device
+    if x.dim() < 1 or weight.dim() != 2:
+        raise ValueError("x must be [..., c_in] and weight [c_out, c_in]")
     c_in = x.shape[-1]
     c_out = weight.shape[0]
     if tuple(weight.shape) != (c_out, c_in):
@@ -441,7 +443,8 @@ def output_projection(x: torch.Tensor, weight: torch.Tensor, bias: Optional[torc
 
 
 def output_projection_failed() -> bool:
-    """Whether a projection since the last call gave up waiting for its MMAs
+    """Whether a projection since the last call gave up waiting (for a TMA copy,
+    an MMA or its epilogue) and left rows unwritten; clears the flag
     (synchronises with the device)."""
     f = ctypes.c_int(0)
     _check(library().msda_output_projection_check(ctypes.byref(f)), "msda_output_projection_check")
