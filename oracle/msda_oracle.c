@@ -22,7 +22,7 @@
  *           zeros padding and align_corners=False; output laid out [N, Lq, M*D]
  *           with channel m*D + d).
  *
- * Readings taken where the pages are silent (each one is listed in the design doc):
+ * Readings taken where the pages are silent:
  *  - grid_sample with align_corners=False maps a grid value g in [-1, 1] to the
  *    pixel coordinate ((g + 1) * W - 1) / 2; with g = 2*loc - 1 that is
  *    loc * W - 0.5.  Pixel centres sit at integer coordinates.
@@ -209,7 +209,7 @@ int msda_oracle_backward(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq,
  *  - reference points with 2 components (x, y): loc = ref + off / (W_l, H_l);
  *  - reference points with 4 components (box centre x, y and size w, h):
  *    loc = ref[0:2] + off / K * ref[2:4] * 0.5.
- * Readings (listed in the design doc):
+ * Readings taken where the pages are silent:
  *  - with round_f32 = 1 the location is formed in float32, every operation
  *    rounded once in the pages' order (division by the normaliser, then the
  *    addition; for boxes the division by K, the product with the size, the
