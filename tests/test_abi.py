@@ -260,3 +260,23 @@ def test_output_projection_arguments(lib):
     assert proj(b=FAKE + 2) == MISAL
     assert proj(rows=0, x=None, w=None, b=None, y=None) == OK
     assert lib.msda_output_projection_check(None) == NULLP
+
+
+def test_binding_rejects_cpu_tensors_and_bad_ranks():
+    """The binding validates before any CUDA call: CPU tensors are refused (there
+    is no CPU path) and the projection's operands must have the right ranks."""
+    import torch
+    x = torch.zeros(4, 8)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        binding.output_projection(x, torch.zeros(16, 8))
+    with pytest.raises(ValueError):
+        binding.output_projection(torch.zeros(()), torch.zeros(16, 8))
+    with pytest.raises(ValueError):
+        binding.output_projection(x, torch.zeros(16))
+    with pytest.raises(ValueError, match="weight must be"):
+        binding.output_projection(x, torch.zeros(16, 4))
+    v = torch.zeros(1, 5, 2, 4)
+    loc = torch.zeros(1, 3, 2, 1, 1, 2)
+    a = torch.zeros(1, 3, 2, 1, 1)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        binding.forward(v, torch.tensor([[1, 5]]), torch.tensor([0]), loc, a)
