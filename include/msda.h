@@ -26,8 +26,12 @@
  *
  * Conventions for every entry point
  *  - All tensor arguments are DEVICE pointers to contiguous row-major arrays
- *    owned by the caller.  The library allocates nothing and keeps no state
- *    between calls.
+ *    owned by the caller.  The library allocates nothing at call time.  The
+ *    state it keeps between calls is small and fixed: the scratch array of
+ *    msda_backward_noalloc (reserved on each device with the library's device
+ *    code), two device flags that record a bounded wait that ran out
+ *    (msda_output_projection_check, msda_wait_check), and per-device caches of
+ *    the SM count and of kernel attributes.
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *    Work is enqueued asynchronously on it; results are ready once the stream
  *    has been synchronised.
@@ -315,12 +319,22 @@ msda_status msda_backward_workspace_size(int64_t B, int64_t S, int64_t M, int64_
  * msda_backward), taking the scratch from one array of
  * MSDA_NOALLOC_SCRATCH_BYTES that the library holds on each device.  It calls
  * no cudaMalloc, cudaFree or other allocating routine.
+ *   - value_dtype must be MSDA_F32 (grad_output is float32); MSDA_BF16 returns
+ *     MSDA_ERR_UNSUPPORTED.
  *   - Sizes whose msda_backward_workspace_size exceeds MSDA_NOALLOC_SCRATCH_BYTES
  *     are rejected with MSDA_ERR_WORKSPACE before anything is enqueued (for
  *     example B=1, S=19947, M=8, D=32, L=K=4 fits up to Lq = 9259 queries).
- *   - The first call on a device looks up the array's device address (set-up,
- *     once per device, with that device current); make that first call before
- *     any stream capture.
+ *   - First call on a device: CUDA loads device code lazily by default, so the
+ *     first call there loads this path's kernels and reserves the 32 MiB array
+ *     on that device -- device memory the CUDA driver takes at that moment, not
+ *     through any allocator of the caller's.  A caller whose framework is about
+ *     to take the whole memory pool should therefore make one warm-up call with
+ *     a small real problem on each device before the pool is taken (or set
+ *     CUDA_MODULE_LOADING=EAGER, which reserves everything when the library is
+ *     loaded).  That first call should also come before any stream capture.
+ *     Later calls reserve nothing.
+ *   - The array's device address is looked up on every call, with the calling
+ *     thread's current device and context.
  *   - Every call on a device uses the same array, and the array keeps the last
  *     call's contents; each call clears what it needs at zero.  Calls that
  *     overlap on the GPU (other streams, other host threads) race on it and must
@@ -335,6 +349,16 @@ msda_status msda_backward_noalloc(int64_t B, int64_t S, int64_t M, int64_t D, in
                                   const float *grad_output, float *grad_value,
                                   float *grad_sampling_locations,
                                   float *grad_attention_weights, void *stream);
+
+/*
+ * *failed = 1 if a kernel with bounded waits between its warps (the encoder
+ * kernels that stage value windows in shared memory) gave up a wait since the
+ * last check, else 0; clears the flag.  Such a kernel leaves some outputs
+ * unwritten.  The waits cannot run out unless the library has a bug; the bound
+ * exists so that a bug cannot hang the GPU.  Synchronises with the device (it
+ * copies the flag to the host).
+ */
+msda_status msda_wait_check(int *failed);
 
 /*
  * Host-side metadata check, for callers that hold host copies of the metadata

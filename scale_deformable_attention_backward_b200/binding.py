@@ -41,6 +41,7 @@ SIGNATURES = {
     "msda_fused_backward": (_I32, [_I64] * 8 + [_I32] + [_VP] * 12),
     "msda_output_projection": (_I32, [_I64] * 3 + [_VP] * 5),
     "msda_output_projection_check": (_I32, [ctypes.POINTER(_I32)]),
+    "msda_wait_check": (_I32, [ctypes.POINTER(_I32)]),
     "msda_check_metadata": (_I32, [_I64, _I64, _VP, _VP]),
     "msda_status_string": (ctypes.c_char_p, [_I32]),
     "msda_version": (_I32, []),
@@ -448,4 +449,14 @@ def output_projection_failed() -> bool:
     (synchronises with the device)."""
     f = ctypes.c_int(0)
     _check(library().msda_output_projection_check(ctypes.byref(f)), "msda_output_projection_check")
+    return bool(f.value)
+
+
+def wait_failed() -> bool:
+    """Whether a kernel with bounded waits between its warps (the encoder
+    kernels that stage value windows in shared memory) gave up a wait since the
+    last call and left outputs unwritten; clears the flag (synchronises with the
+    device)."""
+    f = ctypes.c_int(0)
+    _check(library().msda_wait_check(ctypes.byref(f)), "msda_wait_check")
     return bool(f.value)

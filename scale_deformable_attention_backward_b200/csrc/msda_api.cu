@@ -111,6 +111,7 @@ msda_status msda_forward(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq,
   a.sampling_locations = sampling_locations;
   a.attention_weights = attention_weights;
   a.output = output;
+  a.B = B;
   a.S = S;
   a.Lq = Lq;
   a.M = static_cast<int>(M);
@@ -300,6 +301,17 @@ msda_status msda_output_projection_check(int* failed) {
   if (failed == nullptr) return MSDA_ERR_NULL_POINTER;
   int* flag = nullptr;
   if (msda::projection_failed_flag(&flag) != cudaSuccess) return MSDA_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpy(failed, flag, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess ||
+      cudaMemcpy(flag, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+    return MSDA_ERR_CUDA;
+  return MSDA_OK;
+}
+
+msda_status msda_wait_check(int* failed) {
+  if (failed == nullptr) return MSDA_ERR_NULL_POINTER;
+  int* flag = nullptr;
+  if (msda::tiled_wait_flag(&flag) != cudaSuccess) return MSDA_ERR_CUDA;
   const int zero = 0;
   if (cudaMemcpy(failed, flag, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess ||
       cudaMemcpy(flag, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)

@@ -32,6 +32,8 @@
 // per unit suffices.  (Head-major tiles and contiguous per-block tile ranges,
 // which favour L1 reuse, measured slower on the encoder workload.)
 #include <atomic>
+#include <cstdlib>
+#include <cstring>
 #include <type_traits>
 
 #include "msda_device.cuh"
@@ -314,6 +316,14 @@ static cudaError_t dispatch_lanes(const ForwardArgs& a, cudaStream_t stream) {
 }
 
 cudaError_t launch_forward(const ForwardArgs& a, cudaStream_t stream) {
+  if (forward_tiles_apply(a)) {
+    // The encoder-form kernels (queries = value pixels): selected by
+    // MSDA_FORWARD_KERNEL=staged (shared-memory windows) or =l1 (L1 windows);
+    // the per-point gather below otherwise.
+    const char* v = std::getenv("MSDA_FORWARD_KERNEL");
+    if (v != nullptr && std::strcmp(v, "staged") == 0) return launch_forward_tiled(a, stream);
+    if (v != nullptr && std::strcmp(v, "l1") == 0) return launch_forward_l1(a, stream);
+  }
   return a.bf16 ? dispatch_lanes<__nv_bfloat16>(a, stream) : dispatch_lanes<float>(a, stream);
 }
 

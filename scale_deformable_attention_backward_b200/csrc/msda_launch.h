@@ -18,7 +18,7 @@ struct ForwardArgs {
   const float* sampling_locations;
   const float* attention_weights;
   void* output;
-  long long S, Lq;
+  long long B, S, Lq;
   int M, D, L, K;
   bool bf16;
   int lanes;         // lanes per work group: a power of two <= 32
@@ -90,6 +90,17 @@ struct SortedLayout {
 SortedLayout sorted_layout(long long B, long long S, long long M, long long Lq, int L, int K);
 
 cudaError_t launch_forward(const ForwardArgs& a, cudaStream_t stream);
+// Whether the encoder-form forward kernels apply: the queries are the value's
+// pixels (Lq == S), D * sizeof(T) is 64, 128 or 256 bytes, K <= 8,
+// B * Lq * M < 2^31 and S < 2^26.
+bool forward_tiles_apply(const ForwardArgs& a);
+// The encoder-form forward with shared-memory value windows (msda_forward_tiled.cu).
+cudaError_t launch_forward_tiled(const ForwardArgs& a, cudaStream_t stream);
+// The same tiles gathered through L1 (msda_forward_l1.cu).
+cudaError_t launch_forward_l1(const ForwardArgs& a, cudaStream_t stream);
+// Device address of the flag a tiled kernel sets when one of its bounded waits
+// runs out (msda_forward_tiled.cu).
+cudaError_t tiled_wait_flag(int** flag);
 // Backward with one vector atomic per point corner (no scratch).
 cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t stream);
 // Backward with the points grouped by cell; `workspace` holds sorted_layout().bytes.

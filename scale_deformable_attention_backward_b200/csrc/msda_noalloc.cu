@@ -9,7 +9,6 @@
 // bytes) comes from `noalloc_scratch` below, which every device that loads this
 // library holds until the process exits.
 #include <cstdint>
-#include <mutex>
 #include <cuda_runtime.h>
 
 #include "msda.h"
@@ -20,24 +19,16 @@ namespace {
 // there.
 static __device__ __align__(256) unsigned char noalloc_scratch[MSDA_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-
 // In host code `noalloc_scratch` names a host-side stand-in, not device memory,
-// so its device address is looked up once per device, with that device current.
+// so its device address is looked up with the device current.  The lookup runs
+// on every call: it allocates nothing once the module is loaded, and the
+// address it returns always belongs to the current context (a cached one would
+// not survive cudaDeviceReset or a switch to another context).
 msda_status scratch_address(void** out) {
-  static void* address[kMaxDevices] = {};
-  static std::mutex lock;
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, noalloc_scratch) != cudaSuccess || p == nullptr)
     return MSDA_ERR_CUDA;
-  std::lock_guard<std::mutex> guard(lock);
-  if (address[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, noalloc_scratch) != cudaSuccess || p == nullptr)
-      return MSDA_ERR_CUDA;
-    address[dev] = p;
-  }
-  *out = address[dev];
+  *out = p;
   return MSDA_OK;
 }
 
@@ -49,6 +40,8 @@ extern "C" msda_status msda_backward_noalloc(
     const int64_t* level_start_index, const float* sampling_locations,
     const float* attention_weights, const float* grad_output, float* grad_value,
     float* grad_sampling_locations, float* grad_attention_weights, void* stream) {
+  // The cell-sorted path behind this entry point is float32 only.
+  if (value_dtype != MSDA_F32) return MSDA_ERR_UNSUPPORTED;
   size_t need = 0;
   msda_status st = msda_backward_workspace_size(B, S, M, D, Lq, L, K, &need);
   if (st != MSDA_OK) return st;

@@ -280,3 +280,18 @@ def test_binding_rejects_cpu_tensors_and_bad_ranks():
     a = torch.zeros(1, 3, 2, 1, 1)
     with pytest.raises(ValueError, match="CUDA tensor"):
         binding.forward(v, torch.tensor([[1, 5]]), torch.tensor([0]), loc, a)
+
+
+def test_noalloc_argument_errors(lib):
+    """msda_backward_noalloc refuses, before any device call, a bfloat16 value
+    (its cell-sorted path is float32 only) and sizes whose scratch would not fit
+    the library's fixed array."""
+    ptrs = [ctypes.c_void_p(FAKE)] * 9
+    tiny = (1, 80, 2, 8, 80, 2, 2)
+    assert lib.msda_backward_noalloc(*tiny, 1, *ptrs, None) == UNSUP
+    assert lib.msda_backward_noalloc(*tiny, 2, *ptrs, None) == UNSUP
+    big = (4, 19947, 8, 32, 19947, 4, 4)
+    st, need = ctypes.c_int(0), ctypes.c_size_t(0)
+    assert lib.msda_backward_workspace_size(*big, ctypes.byref(need)) == OK
+    assert need.value > 32 << 20
+    assert lib.msda_backward_noalloc(*big, 0, *ptrs, None) == WORKSPACE

@@ -58,38 +58,56 @@ def _with_workspace(lib, d, outs):
                              _p(ga), _p(ws), need, stream)
 
 
-def _inputs(name):
+def _inputs(name, seed):
     if name == "tiny_fp32":
-        return W.make_inputs(W.CONFIGS["tiny_fp32"], seed=0)
-    enc = W.make_inputs(W.CONFIGS["encoder_train_fp32"].with_batch(1), seed=5)
+        return W.make_inputs(W.CONFIGS["tiny_fp32"], seed=seed)
+    enc = W.make_inputs(W.CONFIGS["encoder_train_fp32"].with_batch(1), seed=seed)
     return W.select_queries(enc, np.arange(0, enc.config.queries, 9))  # 2217 queries
 
 
-@pytest.mark.parametrize("name", ["tiny_fp32", "encoder_b1_subset"])
-def test_noalloc_matches_backward_with_workspace(name):
+NAMES = ("grad_value", "grad_sampling_locations", "grad_attention_weights")
+
+
+def test_noalloc_matches_backward_with_workspace_and_oracle():
+    """Calls with different layouts and inputs in a row -- the encoder subset,
+    the tiny workload, the encoder subset with another seed, and the first
+    input again -- each compared with msda_backward given a caller workspace
+    and with the float64 oracle.  The array keeps each call's contents, so a
+    leftover from the previous call would show up in the next one.  From the
+    second call on, the device's free memory must not change across a call:
+    the first call has loaded the kernels and reserved the array."""
     lib = binding.library()
-    inp = _inputs(name)
-    d = G.device_inputs(inp)
-    assert binding.workspace_size(*_dims(d)) <= SCRATCH_BYTES
-    ref = _outputs(d)
-    assert _with_workspace(lib, d, ref) == 0
-    torch.cuda.synchronize()
-    ref = [t.double().cpu().numpy() for t in ref]
-    names = ("grad_value", "grad_sampling_locations", "grad_attention_weights")
-    # Two calls in a row: the second must not see anything the first left behind.
-    for call in range(2):
+    sequence = [("encoder_b1_subset", 5), ("tiny_fp32", 0), ("encoder_b1_subset", 6),
+                ("encoder_b1_subset", 5)]
+    for call, (name, seed) in enumerate(sequence):
+        inp = _inputs(name, seed)
+        d = G.device_inputs(inp)
+        assert binding.workspace_size(*_dims(d)) <= SCRATCH_BYTES
+        ref = _outputs(d)
+        assert _with_workspace(lib, d, ref) == 0
         outs = _outputs(d)
+        torch.cuda.synchronize()
+        free_before = torch.cuda.mem_get_info()[0]
         assert _noalloc(lib, d, outs) == 0
         torch.cuda.synchronize()
-        for got, want, what in zip(outs, ref, names):
-            G.assert_backward_f32(got.double().cpu().numpy(), want,
-                                  f"{name} {what}, no-alloc call {call + 1}")
+        if call > 0:
+            assert torch.cuda.mem_get_info()[0] == free_before, \
+                f"call {call + 1} changed the free device memory"
+        want_oracle = G.oracle_backward(inp)
+        for got, want_ws, want_or, what in zip(outs, ref, want_oracle, NAMES):
+            got = got.double().cpu().numpy()
+            tag = f"{name} seed {seed} {what}, no-alloc call {call + 1}"
+            G.assert_backward_f32(got, want_ws.double().cpu().numpy(), tag + " vs workspace")
+            G.assert_backward_f32(got, want_or, tag + " vs oracle")
+    assert not binding.wait_failed()
 
 
-def test_noalloc_rejects_sizes_beyond_its_scratch():
+def test_noalloc_rejects_sizes_beyond_its_scratch_and_bf16():
     lib = binding.library()
     B, S, M, D, Lq, L, K = 4, 19947, 8, 32, 19947, 4, 4
     assert binding.workspace_size(B, S, M, D, Lq, L, K) > SCRATCH_BYTES
     fake = ctypes.c_void_p(0x10000)  # never dereferenced: the call is rejected first
     status = lib.msda_backward_noalloc(B, S, M, D, Lq, L, K, 0, *([fake] * 9), None)
     assert status == 6  # MSDA_ERR_WORKSPACE
+    status = lib.msda_backward_noalloc(1, 80, 2, 8, 80, 2, 2, 1, *([fake] * 9), None)
+    assert status == 3  # MSDA_ERR_UNSUPPORTED: the sorted path is float32 only
