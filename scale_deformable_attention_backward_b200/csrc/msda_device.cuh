@@ -182,6 +182,25 @@ struct Group {
 
 __device__ __forceinline__ Group decompose(long long g, int chunks, int M, long long Lq) {
   Group r;
+  if (g < (1ll << 31)) {
+    // 32-bit divisions: a 64-bit one costs several times the instructions, and
+    // this runs per thread per work unit.  g < 2^31 implies bq < 2^31.
+    const unsigned u = static_cast<unsigned>(g);
+    unsigned bqm = u;
+    r.chunk = 0;
+    if (chunks != 1) {
+      bqm = u / static_cast<unsigned>(chunks);
+      r.chunk = static_cast<int>(u - bqm * static_cast<unsigned>(chunks));
+    }
+    const unsigned bq = bqm / static_cast<unsigned>(M);
+    r.m = static_cast<int>(bqm - bq * static_cast<unsigned>(M));
+    r.bqm = bqm;
+    r.bq = bq;
+    // Lq > bq means b = 0 (this also covers Lq >= 2^31, which would not fit the
+    // 32-bit division).
+    r.b = Lq > static_cast<long long>(bq) ? 0 : bq / static_cast<unsigned>(Lq);
+    return r;
+  }
   r.chunk = static_cast<int>(g % chunks);
   r.bqm = g / chunks;
   r.m = static_cast<int>(r.bqm % M);

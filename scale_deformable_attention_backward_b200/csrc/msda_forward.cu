@@ -102,7 +102,7 @@ forward_body(const T* __restrict__ value, const int64_t* __restrict__ spatial_sh
       const int tg = t / PC, tj = t % PC;
       const long long g = t_ * G + tg;
       if (tj < pc && g < groups) {
-        const long long bqm = g / chunks;
+        const long long bqm = chunks == 1 ? g : g / chunks;
         pxy[r] = __ldg(reinterpret_cast<const float2*>(sampling_locations) + bqm * LK + q0 + tj);
         pa[r] = __ldg(attention_weights + bqm * LK + q0 + tj);
       }
@@ -132,7 +132,7 @@ forward_body(const T* __restrict__ value, const int64_t* __restrict__ spatial_sh
         pa[r] = e * (1.0f / sum);
         if (live) {
           const int l = (q0 + tj) / K;
-          const long long bq = g / chunks / M;
+          const long long bq = decompose(g, chunks, M, Lq).bq;
           pxy[r] = fused_location(reference_points + (bq * L + l) * R, pxy[r], R, lv.W[l],
                                   lv.H[l], K);
         }

@@ -162,6 +162,7 @@ forward_tiled_kernel(const T* __restrict__ value, const int64_t* __restrict__ sp
   constexpr int SETUP = (QPS * kMaxK + LANES - 1) / LANES;  // points a lane sets up, at most
   static_assert(CPR >= 1 && 32 % CPR == 0, "a warp copies whole pixels");
   static_assert(QPS >= 1 && QPS * NSW == kMaxTileQueries, "queries split evenly");
+  static_assert(NSW % 8 == 0, "the record swizzle needs a multiple of 8 sub-warps");
 
   // Dynamic shared memory: the consumers' record table; per slot the step's raw
   // points (x, y, A) and a window of `capacity` pixel rows plus one row of zeros
@@ -418,9 +419,12 @@ forward_tiled_kernel(const T* __restrict__ value, const int64_t* __restrict__ sp
             o.z = v01 ? ~((base + W) * MD) : INT_MIN;
             o.w = v11 ? ~((base + W + 1) * MD) : INT_MIN;
           }
+          // Entry t * NSW + (sw ^ (t & 7)): the sub-warps of a warp read one t
+          // at a time from different bank groups, and a sub-warp's lanes write
+          // different t to different bank groups.
           const int t = tj[i] * K + tk[i];
-          s_off[t * NSW + sw] = o;
-          s_w[t * NSW + sw] =
+          s_off[t * NSW + (sw ^ (t & 7))] = o;
+          s_w[t * NSW + (sw ^ (t & 7))] =
               make_float4(p.z * hx * hy, p.z * c.fx * hy, p.z * hx * c.fy, p.z * c.fx * c.fy);
         }
       }
@@ -433,7 +437,8 @@ forward_tiled_kernel(const T* __restrict__ value, const int64_t* __restrict__ sp
       if (j * NSW + sw < count) {
 #pragma unroll 4
         for (int k = 0; k < K; ++k) {
-          const int idx = (j * K + k) * NSW + sw;
+          const int t = j * K + k;
+          const int idx = t * NSW + (sw ^ (t & 7));
           const int4 o = s_off[idx];
           const float4 w = s_w[idx];
           float v0[E], v1[E], v2[E], v3[E];

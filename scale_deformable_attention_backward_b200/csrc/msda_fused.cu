@@ -106,7 +106,7 @@ fused_forward_kernel(const T* __restrict__ value, const int64_t* __restrict__ sp
         const int tg = t / PC, tj = t % PC;
         const long long g = tile * G + tg;
         if (tj < pc && g < groups) {
-          const long long bqm = g / chunks;
+          const long long bqm = chunks == 1 ? g : g / chunks;
           const long long bq = bqm / M;
           const int i = p0 + tj;
           const int l = i / K;

@@ -59,7 +59,10 @@ struct Corner<float> {
   }
   // All four corners of one point: the loads are predicated (a corner outside the
   // map reads as zero without being loaded), then the accumulation runs in the
-  // corners' order.
+  // corners' order.  A corner outside the map still takes its FMA with the zero
+  // it read: w * 0 leaves the sum unchanged (up to the sign of a zero sum), NaN
+  // weights still make it NaN, and issuing the FMAs unconditionally measured
+  // faster than branching around them.
   __device__ __forceinline__ static void accumulate4(const float* vbase, const int4& o,
                                                      const float4& w, float2 (&acc)[2]) {
     const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -70,10 +73,8 @@ struct Corner<float> {
     if (o.w >= 0) v3 = __ldg(reinterpret_cast<const float4*>(vbase + o.w));
     const float4 vs[4] = {v0, v1, v2, v3};
     const float ws[4] = {w.x, w.y, w.z, w.w};
-    const int os[4] = {o.x, o.y, o.z, o.w};
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-      if (os[c] < 0) continue;
       const float2 ww = make_float2(ws[c], ws[c]);
       acc[0] = fma2(ww, make_float2(vs[c].x, vs[c].y), acc[0]);
       acc[1] = fma2(ww, make_float2(vs[c].z, vs[c].w), acc[1]);

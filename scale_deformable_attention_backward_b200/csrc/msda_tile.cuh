@@ -21,12 +21,16 @@ namespace msda {
 //   two_d == 1  the queries are the value's pixels: Lq == S, every level is
 //               valid and level_start_index is the exclusive prefix sum of H*W.
 //               Level l's H x W queries are cut into nty x ntx rectangles of at
-//               most TH x TW, rows and columns split as evenly as possible.
+//               most TH x TW, rows and columns split as evenly as possible: with
+//               H = qy * nty + ry, tile rows 0 .. ry-1 get qy + 1 rows and the
+//               others qy (likewise for columns).
 //   two_d == 0  anything else: tiles are runs of Q consecutive queries.
 struct TileGrid {
   int two_d;
   int nty[kMaxLevels];
   int ntx[kMaxLevels];
+  int qy[kMaxLevels], ry[kMaxLevels];  // H = qy * nty + ry
+  int qx[kMaxLevels], rx[kMaxLevels];  // W = qx * ntx + rx
   int first[kMaxLevels + 1];  // tiles before level l (two_d)
   int tiles;                  // tiles per (b, m); Lq < 2^31 is required by the caller
 };
@@ -60,6 +64,10 @@ __device__ __forceinline__ void build_tile_grid(TileGrid& tg, const Levels& lv, 
         tg.first[l] = tiles;
         tg.nty[l] = (lv.H[l] + TH - 1) / TH;
         tg.ntx[l] = (lv.W[l] + TW - 1) / TW;
+        tg.qy[l] = lv.H[l] / tg.nty[l];
+        tg.ry[l] = lv.H[l] - tg.qy[l] * tg.nty[l];
+        tg.qx[l] = lv.W[l] / tg.ntx[l];
+        tg.rx[l] = lv.W[l] - tg.qx[l] * tg.ntx[l];
         tiles += tg.nty[l] * tg.ntx[l];
       }
       tg.first[L] = tiles;
@@ -79,16 +87,18 @@ __device__ __forceinline__ TileQueries tile_queries(const TileGrid& tg, const Le
     int l = 0;
     while (l + 1 < L && t >= tg.first[l + 1]) ++l;
     const int u = t - tg.first[l];
-    const int ny = tg.nty[l], nx = tg.ntx[l];
+    const int nx = tg.ntx[l];
     const int ty = u / nx, tx = u - ty * nx;
-    const long long H = lv.H[l], W = lv.W[l];
-    const int r0 = static_cast<int>(ty * H / ny), r1 = static_cast<int>((ty + 1) * H / ny);
-    const int c0 = static_cast<int>(tx * W / nx), c1 = static_cast<int>((tx + 1) * W / nx);
+    const int W = lv.W[l];
+    const int r0 = ty * tg.qy[l] + min(ty, tg.ry[l]);
+    const int h = tg.qy[l] + (ty < tg.ry[l] ? 1 : 0);
+    const int c0 = tx * tg.qx[l] + min(tx, tg.rx[l]);
+    const int w = tg.qx[l] + (tx < tg.rx[l] ? 1 : 0);
     // start + r * W + c < start + H * W <= Lq < 2^31.
-    r.base = static_cast<int>(lv.start[l] + r0 * W + c0);
-    r.pitch = static_cast<int>(W);
-    r.width = c1 - c0;
-    r.count = (r1 - r0) * (c1 - c0);
+    r.base = static_cast<int>(lv.start[l]) + r0 * W + c0;
+    r.pitch = W;
+    r.width = w;
+    r.count = h * w;
   } else {
     r.base = t * Q;
     r.pitch = Q;
