@@ -72,7 +72,7 @@ constexpr int kBwdPoints = 512;  // points set up per unit (two per thread)
 // atomic instruction of a sub-warp covers one contiguous span.  If an input is
 // not finite (header->fixed == 0) the kernel falls back to float atomics into
 // grad_value: the NaN / Inf pattern does not depend on the order either.
-template <typename T, int LANES, bool FIXED>
+template <typename T, int LANES, bool FIXED, int SPLIT>
 __global__ void __launch_bounds__(kBwdThreads)
 backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial_shapes,
                 const int64_t* __restrict__ level_start_index,
@@ -107,11 +107,25 @@ backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial
   const int gi = threadIdx.x / LANES;
   const int LK = L * K;
   const int MD = M * D;  // < 2^31: one image's value block is (checked by the C ABI)
-  const long long tiles = (groups + G - 1) / G;
+  // Point split (SPLIT > 1): SPLIT consecutive sub-warps share one group,
+  // subset s taking its points s, s + SPLIT, ...  Every result of the backward is
+  // per point (or an atomic), so the subsets need no reduction; work units run
+  // over the virtual groups (groups * SPLIT) and their LKv points.
+  const long long vgroups = groups * SPLIT;
+  const int LKv = (LK + SPLIT - 1) / SPLIT;
+  const long long tiles = (vgroups + G - 1) / G;
+  // Virtual point (group v, point jv) -> real group g and point index jr.
+  auto real_point = [&](long long v, int jv, long long& g, int& jr) {
+    g = v / SPLIT;
+    jr = jv * SPLIT + static_cast<int>(v - g * SPLIT);
+  };
 
   for (long long tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
-    const long long g_raw = tile * G + gi;
-    const bool active = g_raw < groups;
+    const long long v_raw = tile * G + gi;
+    const bool active = v_raw < vgroups;
+    long long g_raw;
+    int subset_first;
+    real_point(v_raw, 0, g_raw, subset_first);  // subset_first = this sub-warp's subset s
     const Group grp = decompose(active ? g_raw : groups - 1, 1, M, Lq);
     const int ch = lane * E;
     const bool lane_on = active && ch < D;  // clamped tail groups touch no memory
@@ -143,19 +157,28 @@ backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial
                   ch,
               go);
 
-    for (int q0 = 0; q0 < LK; q0 += PC) {
-      const int pc = min(PC, LK - q0);
+    for (int q0 = 0; q0 < LKv; q0 += PC) {
+      const int pc = min(PC, LKv - q0);
       // Phase 1: the unit's points, two per thread.
 #pragma unroll
       for (int r = 0; r < PER; ++r) {
         const int t = threadIdx.x + r * kBwdThreads;
         const int tg = t / PC, tj = t % PC;
-        const long long g = tile * G + tg;
-        if (tj < pc && g < groups) {
-          const long long pidx = g * LK + q0 + tj;
+        long long g;
+        int jr;
+        real_point(tile * G + tg, q0 + tj, g, jr);
+        if (SPLIT > 1 && tj < pc && g < groups && jr >= LK) {
+          // A subset's slot past its group's last point: no corner, no output.
+          const int slot = tj * G + (tg ^ (tj & 7));
+          s_off[slot] = make_int4(-1, -1, -1, -1);
+          s_w[slot] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+          s_g[slot] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        }
+        if (tj < pc && g < groups && jr < LK) {
+          const long long pidx = g * LK + jr;
           const float2 xy = __ldg(reinterpret_cast<const float2*>(sampling_locations) + pidx);
           const float a = __ldg(attention_weights + pidx);
-          const int l = (q0 + tj) / K;
+          const int l = jr / K;
           const int H = lv.H[l], W = lv.W[l];
           const Cell c = locate(xy.x, xy.y, H, W);
           const float hx = 1.0f - c.fx, hy = 1.0f - c.fy;
@@ -221,14 +244,15 @@ backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial
             for (int i = 0; i < 4; ++i) keep[i] = dot[i];
           }
         }
-        if (active && lane < nb) {
+        const int jr_out = (q0 + j0 + lane) * SPLIT + subset_first;
+        if (active && lane < nb && jr_out < LK) {
           const int j = j0 + lane;
           const float4 gg = s_g[j * G + (gi ^ (j & 7))];
           const float fx = gg.x, fy = gg.y;
           const float s_attn = fmaf(fx, fmaf(fy, keep[3], keep[1]), fmaf(fy, keep[2], keep[0]));
           const float s_x = fmaf(fy, keep[3], keep[1]);
           const float s_y = fmaf(fx, keep[3], keep[2]);
-          const long long pidx = grp.bqm * LK + q0 + j;
+          const long long pidx = grp.bqm * LK + jr_out;
           grad_attention_weights[pidx] = s_attn;
           reinterpret_cast<float2*>(grad_sampling_locations)[pidx] =
               make_float2(gg.z * s_x, gg.w * s_y);
@@ -354,14 +378,24 @@ template <typename T, int LANES, bool FIXED>
 static cudaError_t launch_backward_t(const BackwardArgs& a, unsigned long long* acc,
                                      const FixedHeader* header, cudaStream_t stream) {
   const long long per_block = kBwdThreads / LANES;
-  long long blocks = (a.groups + per_block - 1) / per_block;
+  // Fewer blocks than about two waves of 148 SMs x 4 (a decoder's few hundred
+  // queries): split each group's points over up to 4 sub-warps.
+  int split = 1;
+  while (split < 4 && (a.groups * split * 2 + per_block - 1) / per_block <= 148 * 4 * 2)
+    split *= 2;
+  long long blocks = (a.groups * split + per_block - 1) / per_block;
   if (blocks > (1ll << 30)) blocks = 1ll << 30;
-  backward_kernel<T, LANES, FIXED><<<static_cast<unsigned>(blocks), kBwdThreads, 0, stream>>>(
-      static_cast<const T*>(a.value), a.spatial_shapes, a.level_start_index,
-      a.sampling_locations, a.attention_weights, static_cast<const T*>(a.grad_output),
-      a.grad_value, a.grad_sampling_locations, a.grad_attention_weights, a.S, a.M, a.D, a.Lq,
-      a.L, a.K, a.groups, acc, header);
-  return cudaGetLastError();
+  auto go = [&](auto kernel) {
+    kernel<<<static_cast<unsigned>(blocks), kBwdThreads, 0, stream>>>(
+        static_cast<const T*>(a.value), a.spatial_shapes, a.level_start_index,
+        a.sampling_locations, a.attention_weights, static_cast<const T*>(a.grad_output),
+        a.grad_value, a.grad_sampling_locations, a.grad_attention_weights, a.S, a.M, a.D,
+        a.Lq, a.L, a.K, a.groups, acc, header);
+    return cudaGetLastError();
+  };
+  if (split == 4) return go(backward_kernel<T, LANES, FIXED, 4>);
+  if (split == 2) return go(backward_kernel<T, LANES, FIXED, 2>);
+  return go(backward_kernel<T, LANES, FIXED, 1>);
 }
 
 template <typename T, bool FIXED>

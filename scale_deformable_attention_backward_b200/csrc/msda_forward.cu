@@ -50,8 +50,8 @@ constexpr int kChunkPoints = 512;
 // Tuning per value dtype (measured on the encoder workloads): for float32 the
 // gathers of up to 8 points are issued back to back (predicated corner loads,
 // Corner::accumulate4) and the kernel is held to 5 blocks per SM (48
-// registers); bfloat16 keeps one branch per corner, a 4-point unroll and the
-// compiler's own register choice (64), which measured faster for it.  The two
+// registers); bfloat16 keeps one branch per corner, a 4-point unroll and 4
+// blocks per SM (64 registers), which measured faster for it.  The two
 // dtypes therefore get their own __global__ entry (forward_kernel below) around
 // one body.
 
@@ -63,7 +63,7 @@ constexpr int kChunkPoints = 512;
 // the setup forms each point's location and softmax weight in registers.  This
 // needs a group's L*K points in one unit (L*K <= PC <= 32), so the softmax is a
 // shuffle reduction over the PC consecutive threads that set the group up.
-template <typename T, int LANES, bool FUSED>
+template <typename T, int LANES, bool FUSED, int SPLIT>
 __device__ __forceinline__ void
 forward_body(const T* __restrict__ value, const int64_t* __restrict__ spatial_shapes,
              const int64_t* __restrict__ level_start_index,
@@ -86,7 +86,14 @@ forward_body(const T* __restrict__ value, const int64_t* __restrict__ spatial_sh
   const int gi = threadIdx.x / LANES;
   const int LK = L * K;
   const int MD = M * D;
-  const long long tiles = (groups + G - 1) / G;
+  // Point split (SPLIT > 1, non-fused, chunks == 1): SPLIT consecutive
+  // sub-warps share one group, subset s taking its points s, s + SPLIT, ...;
+  // their partial sums are added with shuffles before the store.  Work units
+  // then run over the virtual groups (groups * SPLIT) and their LKv points.
+  static_assert(SPLIT == 1 || (!FUSED && LANES * SPLIT <= 32), "a split group fits one warp");
+  const long long vgroups = groups * SPLIT;
+  const int LKv = (LK + SPLIT - 1) / SPLIT;
+  const long long tiles = (vgroups + G - 1) / G;
   long long tile = blockIdx.x;
   if (tile >= tiles) return;
   int p0 = 0;
@@ -94,28 +101,43 @@ forward_body(const T* __restrict__ value, const int64_t* __restrict__ spatial_sh
   // Prefetched inputs of the next unit's points.
   float2 pxy[PER];
   float pa[PER];
+  // Virtual point (group v, point q0 + tj) -> real group and point index jr.
+  auto real_point = [&](long long v, int jv, long long& g, int& jr) {
+    g = v / SPLIT;
+    jr = jv * SPLIT + static_cast<int>(v - g * SPLIT);
+  };
   auto prefetch = [&](long long t_, int q0) {
-    const int pc = min(PC, LK - q0);
+    const int pc = min(PC, LKv - q0);
 #pragma unroll
     for (int r = 0; r < PER; ++r) {
       const int t = threadIdx.x + r * kThreads;
       const int tg = t / PC, tj = t % PC;
-      const long long g = t_ * G + tg;
-      if (tj < pc && g < groups) {
+      long long g;
+      int jr;
+      real_point(t_ * G + tg, q0 + tj, g, jr);
+      if (tj < pc && g < groups && jr < LK) {
         const long long bqm = chunks == 1 ? g : g / chunks;
-        pxy[r] = __ldg(reinterpret_cast<const float2*>(sampling_locations) + bqm * LK + q0 + tj);
-        pa[r] = __ldg(attention_weights + bqm * LK + q0 + tj);
+        pxy[r] = __ldg(reinterpret_cast<const float2*>(sampling_locations) + bqm * LK + jr);
+        pa[r] = __ldg(attention_weights + bqm * LK + jr);
       }
     }
   };
   auto setup = [&](long long t_, int q0, int buf) {
-    const int pc = min(PC, LK - q0);
+    const int pc = min(PC, LKv - q0);
 #pragma unroll
     for (int r = 0; r < PER; ++r) {
       const int t = threadIdx.x + r * kThreads;
       const int tg = t / PC, tj = t % PC;
-      const long long g = t_ * G + tg;
-      const bool live = tj < pc && g < groups;
+      long long g;
+      int jr;
+      real_point(t_ * G + tg, q0 + tj, g, jr);
+      const bool live = tj < pc && g < groups && jr < LK;
+      if (SPLIT > 1 && tj < pc && g < groups && jr >= LK) {
+        // A subset's slot past its group's last point reads nothing and adds zero.
+        const int slot = tj * G + (tg ^ (tj & 7));
+        s_off[buf][slot] = make_int4(-1, -1, -1, -1);
+        s_w[buf][slot] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      }
       if constexpr (FUSED) {
         // Softmax over the group's L*K = pc logits, held by PC consecutive lanes.
         float z = live ? pa[r] : -INFINITY;
@@ -131,14 +153,14 @@ forward_body(const T* __restrict__ value, const int64_t* __restrict__ spatial_sh
         for (int o = PC / 2; o > 0; o >>= 1) sum += __shfl_xor_sync(kFullMask, sum, o, PC);
         pa[r] = e * (1.0f / sum);
         if (live) {
-          const int l = (q0 + tj) / K;
+          const int l = jr / K;
           const long long bq = decompose(g, chunks, M, Lq).bq;
           pxy[r] = fused_location(reference_points + (bq * L + l) * R, pxy[r], R, lv.W[l],
                                   lv.H[l], K);
         }
       }
       if (live) {
-        const int l = (q0 + tj) / K;
+        const int l = jr / K;
         const PointSetup su = setup_point(pxy[r].x, pxy[r].y, pa[r], lv.H[l], lv.W[l], lv.start[l], MD);
         const int slot = tj * G + (tg ^ (tj & 7));
         s_off[buf][slot] = su.off;
@@ -158,19 +180,20 @@ forward_body(const T* __restrict__ value, const int64_t* __restrict__ spatial_sh
     // The unit after this one: the next chunk of this tile, or the next tile.
     long long ntile = tile;
     int np0 = p0 + PC;
-    if (np0 >= LK) {
+    if (np0 >= LKv) {
       ntile = tile + gridDim.x;
       np0 = 0;
     }
     const bool more = ntile < tiles;
     if (more) prefetch(ntile, np0);
-    const long long g_raw = tile * G + gi;
-    const bool active = g_raw < groups;
+    const long long v_raw = tile * G + gi;
+    const bool active = v_raw < vgroups;
+    const long long g_raw = v_raw / SPLIT;
     const Group grp = decompose(active ? g_raw : groups - 1, chunks, M, Lq);
     const int ch = (grp.chunk * LANES + lane) * E;
     const bool lane_on = active && ch < D;
     const T* vbase = value + (grp.b * S * M + grp.m) * static_cast<long long>(D) + ch;
-    const int pc = min(PC, LK - p0);
+    const int pc = min(PC, LKv - p0);
     if (lane_on) {
       if constexpr (std::is_same<T, float>::value) {
 #pragma unroll 8
@@ -193,8 +216,20 @@ forward_body(const T* __restrict__ value, const int64_t* __restrict__ spatial_sh
         }
       }
     }
-    if (p0 + PC >= LK) {
-      if (lane_on) C::store(output + grp.bq * MD + static_cast<long long>(grp.m) * D + ch, acc);
+    if (p0 + PC >= LKv) {
+      if constexpr (SPLIT > 1) {
+        // The split sub-warps of a group are consecutive in the warp.
+#pragma unroll
+        for (int o = LANES; o < LANES * SPLIT; o <<= 1) {
+#pragma unroll
+          for (int e = 0; e < E / 2; ++e) {
+            acc[e].x += __shfl_xor_sync(kFullMask, acc[e].x, o);
+            acc[e].y += __shfl_xor_sync(kFullMask, acc[e].y, o);
+          }
+        }
+      }
+      if (lane_on && v_raw % SPLIT == 0)
+        C::store(output + grp.bq * MD + static_cast<long long>(grp.m) * D + ch, acc);
 #pragma unroll
       for (int e = 0; e < E / 2; ++e) acc[e] = make_float2(0.0f, 0.0f);
     }
@@ -218,30 +253,30 @@ forward_body(const T* __restrict__ value, const int64_t* __restrict__ spatial_sh
   value, spatial_shapes, level_start_index, sampling_locations, attention_weights, output, \
       S, M, D, Lq, L, K, chunks, groups, reference_points, R
 
-template <int LANES, bool FUSED>
+template <int LANES, bool FUSED, int SPLIT>
 __global__ void __launch_bounds__(kThreads, 5) forward_kernel_f32(MSDA_FORWARD_PARAMS(float)) {
-  forward_body<float, LANES, FUSED>(MSDA_FORWARD_ARGS);
+  forward_body<float, LANES, FUSED, SPLIT>(MSDA_FORWARD_ARGS);
 }
 
-template <int LANES, bool FUSED>
-__global__ void __launch_bounds__(kThreads)
+template <int LANES, bool FUSED, int SPLIT>
+__global__ void __launch_bounds__(kThreads, 4)
     forward_kernel_bf16(MSDA_FORWARD_PARAMS(__nv_bfloat16)) {
-  forward_body<__nv_bfloat16, LANES, FUSED>(MSDA_FORWARD_ARGS);
+  forward_body<__nv_bfloat16, LANES, FUSED, SPLIT>(MSDA_FORWARD_ARGS);
 }
 
 #undef MSDA_FORWARD_PARAMS
 #undef MSDA_FORWARD_ARGS
 
 // The entry of each value dtype.
-template <typename T, int LANES, bool FUSED>
+template <typename T, int LANES, bool FUSED, int SPLIT = 1>
 struct ForwardKernel;
-template <int LANES, bool FUSED>
-struct ForwardKernel<float, LANES, FUSED> {
-  static constexpr auto fn = forward_kernel_f32<LANES, FUSED>;
+template <int LANES, bool FUSED, int SPLIT>
+struct ForwardKernel<float, LANES, FUSED, SPLIT> {
+  static constexpr auto fn = forward_kernel_f32<LANES, FUSED, SPLIT>;
 };
-template <int LANES, bool FUSED>
-struct ForwardKernel<__nv_bfloat16, LANES, FUSED> {
-  static constexpr auto fn = forward_kernel_bf16<LANES, FUSED>;
+template <int LANES, bool FUSED, int SPLIT>
+struct ForwardKernel<__nv_bfloat16, LANES, FUSED, SPLIT> {
+  static constexpr auto fn = forward_kernel_bf16<LANES, FUSED, SPLIT>;
 };
 
 // Blocks of this kernel that are resident on the current device at once
@@ -265,14 +300,30 @@ static long long resident_blocks() {
 template <typename T, int LANES>
 static cudaError_t launch_forward_t(const ForwardArgs& a, cudaStream_t stream) {
   constexpr int G = kThreads / LANES;
-  const long long tiles = (a.groups + G - 1) / G;
-  long long blocks = resident_blocks<T, LANES, false>();
+  const long long resident = resident_blocks<T, LANES, false>();
+  // Too few tiles to fill the GPU (a decoder's few hundred queries): split each
+  // group's points over up to 4 sub-warps of one warp.
+  int split = 1;
+  if (a.chunks == 1)
+    while (split < 4 && LANES * split * 2 <= 32 && (a.groups * split + G - 1) / G * 2 <= resident)
+      split *= 2;
+  const long long tiles = (a.groups * split + G - 1) / G;
+  long long blocks = resident;
   if (blocks > tiles) blocks = tiles;
-  ForwardKernel<T, LANES, false>::fn<<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(
-      static_cast<const T*>(a.value), a.spatial_shapes, a.level_start_index,
-      a.sampling_locations, a.attention_weights, static_cast<T*>(a.output), a.S, a.M, a.D,
-      a.Lq, a.L, a.K, a.chunks, a.groups, nullptr, 0);
-  return cudaGetLastError();
+  auto go = [&](auto kernel) {
+    kernel<<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(
+        static_cast<const T*>(a.value), a.spatial_shapes, a.level_start_index,
+        a.sampling_locations, a.attention_weights, static_cast<T*>(a.output), a.S, a.M, a.D,
+        a.Lq, a.L, a.K, a.chunks, a.groups, nullptr, 0);
+    return cudaGetLastError();
+  };
+  if constexpr (LANES <= 8) {
+    if (split == 4) return go(ForwardKernel<T, LANES, false, 4>::fn);
+  }
+  if constexpr (LANES <= 16) {
+    if (split == 2) return go(ForwardKernel<T, LANES, false, 2>::fn);
+  }
+  return go(ForwardKernel<T, LANES, false, 1>::fn);
 }
 
 template <typename T, int LANES>

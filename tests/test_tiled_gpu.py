@@ -4,10 +4,12 @@ and each CTA stages the value windows of a rectangle of queries in shared
 memory.
 
 Every case is compared with the float64 oracle, and with the per-point gather
-kernel (selected by MSDA_FORWARD_KERNEL=gather) on the same inputs.  Both add
-the same float32 products in the same order -- level, point, corner -- so their
-outputs must agree bit for bit (a corner outside the map adds w * 0 in the tiled
-kernel, which can only flip the sign of a zero).
+kernel (selected by MSDA_FORWARD_KERNEL=gather) on the same inputs.  The tiled
+kernels add the same float32 products as the gather kernel in the same order --
+level, point, corner -- so at full size they agree with it bit for bit.  On the
+small cases here the gather kernel spreads each query's points over several
+sub-warps (too few queries to fill the GPU otherwise) and adds partial sums, so
+there the comparison is within the float32 forward tolerance.
 
 The cases cover the three kinds of step the kernel has: windows that fit the
 shared buffer (encoder locality), windows that do not (non-local samples: the
@@ -60,8 +62,15 @@ def check(inp, what):
     assert not binding.wait_failed(), f"{what}: a bounded wait ran out"
     ref = G.oracle_forward(inp)
     for name in TILED_KERNELS:
-        assert np.array_equal(out[name], out["gather"], equal_nan=True), \
-            f"{what}: {name} != gather"
+        if inp.config.dtype == "bf16":
+            # Two roundings of float32 sums that differ in their last bits can be
+            # one bfloat16 step (2^-7 relative) apart.
+            a, b = out[name], out["gather"]
+            scale = np.abs(b).max()
+            assert np.all(np.abs(a - b) <= 2.0 ** -7 * np.abs(b) + 1e-5 * scale), \
+                f"{what} ({name} vs gather)"
+        else:
+            G.assert_forward_f32(out[name], out["gather"], f"{what} ({name} vs gather)")
         if inp.config.dtype == "bf16":
             G.assert_forward_bf16(out[name], ref, f"{what} ({name})")
         else:
