@@ -120,6 +120,20 @@ def recorded_traffic(key: str):
     return rec.get("dram_bytes_per_launch")
 
 
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def measured_bf16_peak():
+    """Dense bf16 GEMM burst peak in TF/s: MEASURED_PEAKS.json's, else the pool's
+    earlier measurement (fallback)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except (OSError, ValueError, KeyError):
+        return FALLBACK_BF16_TFLOPS, "fallback"
+
+
 def measured_peak():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -214,6 +228,64 @@ def oracle_sample(cfg: W.Config, target_s: float = 12.0, per_step_target_s=None)
             f"each of the B={cfg.B} images (value over all {cfg.S} tokens), float64 oracle, "
             f"single thread, {dt:.2f} s")
     return queries / dt, desc, dt
+
+
+def host_threads() -> int:
+    """Host cores this process may run on."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        return os.cpu_count() or 1
+
+
+def host_cpu() -> dict:
+    """CPU model and core counts of the host (from /proc/cpuinfo)."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"model": model, "logical_cpus": os.cpu_count(), "usable_cpus": host_threads()}
+
+
+def oracle_threaded(cfg: W.Config, n: int, threads: int):
+    """The same sample as oracle_sample (the first n queries of every image),
+    forward + backward, split into `threads` runs of consecutive queries that
+    call the float64 oracle at once from `threads` host threads (the oracle's
+    plain loops, unchanged; the foreign calls release the GIL).  Each run keeps
+    its own grad_value, and the runs' grad_values are added at the end.
+    Returns (queries/s, description)."""
+    import oracle  # test infrastructure: used here only for the CPU baseline
+    from concurrent.futures import ThreadPoolExecutor
+    inp = W.select_queries(W.make_inputs(cfg, seed=0, with_grad=True), np.arange(n))
+    orc = oracle.default()
+    bounds = np.linspace(0, n, threads + 1).astype(int)
+    parts = [W.select_queries(inp, np.arange(lo, hi))
+             for lo, hi in zip(bounds[:-1], bounds[1:]) if hi > lo]
+
+    def run(sub):
+        orc.forward(sub.value, sub.spatial_shapes, sub.level_start_index,
+                    sub.sampling_locations, sub.attention_weights)
+        gv, _, _ = orc.backward(sub.value, sub.spatial_shapes, sub.level_start_index,
+                                sub.sampling_locations, sub.attention_weights,
+                                sub.grad_output)
+        return gv
+
+    with ThreadPoolExecutor(max_workers=len(parts)) as pool:
+        t0 = time.perf_counter()
+        grads = list(pool.map(run, parts))
+        total = grads[0]
+        for g in grads[1:]:
+            total += g
+        dt = time.perf_counter() - t0
+    desc = (f"{cfg.name}: the same {n} queries of each of the B={cfg.B} images, in "
+            f"{len(parts)} runs on {len(parts)} host threads (private grad_value per run, "
+            f"added at the end), float64 oracle, {dt:.2f} s")
+    return cfg.B * n / dt, desc
 
 
 # ---------------------------------------------------------------------------
@@ -482,9 +554,8 @@ def run_b200(args, world, rank, local):
     proj_rows = B * Lq
     proj_bytes = proj_rows * M * D * 4 * 2 + M * D * M * D * 4 + M * D * 4
     proj_flops = 2.0 * proj_rows * (M * D) * (M * D)
-    with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
-        bf16_peak = float(json.load(f).get("bf16_tflops", 0.0)) or None
-    tf32_peak = None if bf16_peak is None else bf16_peak * 1.1 / 2.25
+    bf16_peak, bf16_source = measured_bf16_peak()
+    tf32_peak = bf16_peak * 1.1 / 2.25
     proj_gbs = proj_bytes / (proj_ms * 1e-3) / 1e9
     projection = {
         "workload": f"output_proj Linear {M * D}->{M * D} on the step's forward output "
@@ -495,8 +566,9 @@ def run_b200(args, world, rank, local):
                      "unit": "GB/s", "frac": round(proj_gbs / peak, 4),
                      "algorithmic_bytes": proj_bytes},
         "tensor": {"achieved_tflops": round(proj_flops / (proj_ms * 1e-3) / 1e12, 1),
-                   "tf32_peak_tflops": None if tf32_peak is None else round(tf32_peak, 1),
-                   "peak_source": "measured bf16 burst x nominal tf32/bf16 ratio 1.1/2.25"},
+                   "tf32_peak_tflops": round(tf32_peak, 1),
+                   "peak_source": f"{bf16_source} bf16 burst x nominal tf32/bf16 ratio "
+                                  f"1.1/2.25"},
     }
 
     # The bfloat16 training step (value and grad_output bf16; float32 arithmetic and
@@ -526,6 +598,46 @@ def run_b200(args, world, rank, local):
         "queries_per_s": round(world * bq / (bf16_ms * 1e-3), 1),
         "steps": n_fused,
     }
+
+    # The decoder cross-attention workloads (a few hundred queries over the
+    # encoder's whole value): forward of decoder_fp32, backward of
+    # decoder_box_train_fp32.  Their compulsory bytes count the whole value
+    # tensor, which the gathers touch only in part (latency / random-access bound).
+    decoder = {}
+    for dname, passes in (("decoder_fp32", ("forward",)),
+                          ("decoder_box_train_fp32", ("forward", "backward"))):
+        dcfg = W.CONFIGS[dname]
+        dinp = W.make_inputs(dcfg, seed=0, with_grad=True)
+        dd = _device_inputs(dinp, device)
+        dout = torch.empty((dcfg.B, dcfg.queries, dcfg.M * dcfg.D), dtype=torch.float32,
+                           device=device)
+        dgv = torch.empty(dinp.value.shape, dtype=torch.float32, device=device)
+        dgl = torch.empty_like(dd["sampling_locations"])
+        dga = torch.empty_like(dd["attention_weights"])
+        dalgo = algorithmic_bytes(dcfg, dinp)
+        entry = {"workload": dcfg.description}
+        for pas in passes:
+            if pas == "forward":
+                fn = lambda: binding.forward(dd["value"], dd["spatial_shapes"],
+                                             dd["level_start_index"], dd["sampling_locations"],
+                                             dd["attention_weights"], output=dout)
+            else:
+                fn = lambda: binding.backward(dd["value"], dd["spatial_shapes"],
+                                              dd["level_start_index"],
+                                              dd["sampling_locations"],
+                                              dd["attention_weights"], dd["grad_output"],
+                                              grad_value=dgv, grad_sampling_locations=dgl,
+                                              grad_attention_weights=dga)
+            t_ms = max_over_ranks(time_steps(fn, n_fused), world, device)
+            gbs = dalgo[pas] / (t_ms * 1e-3) / 1e9
+            entry[pas] = {"mean_us": round(t_ms * 1e3, 2),
+                          "queries_per_s": round(world * dcfg.B * dcfg.queries / (t_ms * 1e-3), 1),
+                          "achieved_gbs_whole_value": round(gbs, 1),
+                          "frac_whole_value": round(gbs / peak, 4)}
+        entry["note"] = ("bytes count the whole value tensor (and for the backward the "
+                         "whole grad_value, zeroed in the call); the gathers read only "
+                         "the lines their points touch, as random 128-byte lines")
+        decoder[dname] = entry
 
     # The encoder self-attention forward alone (B=2), the spec workload.
     fcfg = W.CONFIGS[FORWARD_WORKLOAD]
@@ -631,17 +743,18 @@ def run_b200(args, world, rank, local):
     e2e_ms = max_over_ranks(ee0.elapsed_time(ee1), world, device) / e2e_steps
     barrier(world)
     # The pipeline returns what one plain call on the device-resident inputs
-    # returns (the output and grad_sampling_locations do not depend on the order
-    # of atomics, so they must match bit for bit).
+    # returns (the output, grad_sampling_locations and grad_attention_weights do
+    # not depend on the order of atomics, so they must match bit for bit).
     ref_out = binding.forward(d["value"], d["spatial_shapes"], d["level_start_index"],
                               d["sampling_locations"], d["attention_weights"])
-    _, ref_gl, _ = binding.backward(d["value"], d["spatial_shapes"], d["level_start_index"],
-                                    d["sampling_locations"], d["attention_weights"],
-                                    d["grad_output"])
+    _, ref_gl, ref_ga = binding.backward(d["value"], d["spatial_shapes"],
+                                         d["level_start_index"], d["sampling_locations"],
+                                         d["attention_weights"], d["grad_output"])
     last = host_out[(e2e_steps - 1) % n_buf]
-    if not (torch.equal(last["out"], ref_out.cpu()) and torch.equal(last["gl"], ref_gl.cpu())):
+    if not (torch.equal(last["out"], ref_out.cpu()) and torch.equal(last["gl"], ref_gl.cpu())
+            and torch.equal(last["ga"], ref_ga.cpu())):
         raise RuntimeError("end-to-end pipeline results differ from a plain call's")
-    del ref_out, ref_gl
+    del ref_out, ref_gl, ref_ga
 
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": "queries/s", "n_gpus": world,
@@ -656,6 +769,7 @@ def run_b200(args, world, rank, local):
         "forward_encoder": forward_encoder,
         "fused": fused,
         "bf16_train": bf16_train,
+        "decoder": decoder,
         "projection": projection,
         "e2e": {"value": round(world * queries / (e2e_ms * 1e-3), 1), "unit": "queries/s",
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": int(h2d),
@@ -667,9 +781,14 @@ def run_b200(args, world, rank, local):
         "cpu_baseline": None,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        qps, desc, _ = oracle_sample(cfg)
+        qps, desc, dt = oracle_sample(cfg)
+        n = int(round(qps * dt / cfg.B))
+        threads = host_threads()
+        mt_qps, mt_desc = oracle_threaded(cfg, n, threads)
         result["cpu_baseline"] = {"value": round(qps, 2), "unit": "queries/s", "cores": 1,
-                                  "kind": "oracle", "sample": desc}
+                                  "kind": "oracle", "sample": desc, "host": host_cpu(),
+                                  "threaded": {"value": round(mt_qps, 2), "unit": "queries/s",
+                                               "cores": threads, "sample": mt_desc}}
     return result
 
 
@@ -772,7 +891,7 @@ def run_reference(args):
         "config": {"workload": cfg.description, "step": "oracle forward + backward",
                    "queries_per_step": cfg.B * n},
         "cpu_baseline": {"value": round(value, 3), "unit": "queries/s", "cores": 1,
-                         "kind": "oracle", "sample": sample},
+                         "kind": "oracle", "sample": sample, "host": host_cpu()},
         "e2e": {"value": round(value, 3), "unit": "queries/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }

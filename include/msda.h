@@ -114,7 +114,13 @@ msda_status msda_forward(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq,
  * inputs (the softmax before them is not differentiated).
  *
  *   value, spatial_shapes, level_start_index, sampling_locations,
- *   attention_weights   as for msda_forward; D <= 128.  value_dtype MSDA_F32,
+ *   attention_weights   as for msda_forward; D <= 128 (one sub-warp of at
+ *                       most 32 lanes holds a head's D channels, 4 per lane,
+ *                       and reduces each point's corner dot products over
+ *                       them; larger D returns MSDA_ERR_UNSUPPORTED -- the
+ *                       forward splits larger heads into channel chunks, which
+ *                       would make those reductions cross sub-warps).
+ *                       value_dtype MSDA_F32,
  *                       or MSDA_BF16 without a workspace (value and
  *                       grad_output then only need 8-byte alignment; the
  *                       arithmetic and every gradient stay float32)
