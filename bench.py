@@ -590,12 +590,35 @@ def run_b200(args, world, rank, local):
                          grad_value=bgv, grad_sampling_locations=bgl, grad_attention_weights=bga)
 
     bf16_ms = max_over_ranks(time_steps(bf16_step, n_fused), world, device)
+
+    # The same bf16 step through the fused op (raw reference points, offsets and
+    # logits; bf16 value and grad_output).
+    bfz = W.make_fused_inputs(bcfg, seed=0)
+    bfd = {k: torch.from_numpy(getattr(bfz, k)).to(device) for k in
+           ("spatial_shapes", "level_start_index", "reference_points", "sampling_offsets",
+            "attention_logits")}
+    bfd["value"] = bd["value"]
+    bfd["grad_output"] = bd["grad_output"]
+
+    def bf16_fused_step():
+        binding.fused_forward(bfd["value"], bfd["spatial_shapes"], bfd["level_start_index"],
+                              bfd["reference_points"], bfd["sampling_offsets"],
+                              bfd["attention_logits"], output=bout)
+        binding.fused_backward(bfd["value"], bfd["spatial_shapes"], bfd["level_start_index"],
+                               bfd["reference_points"], bfd["sampling_offsets"],
+                               bfd["attention_logits"], bfd["grad_output"],
+                               reference_grad=False)
+
+    bf16_fused_ms = max_over_ranks(time_steps(bf16_fused_step, n_fused), world, device)
     bq = bcfg.B * bcfg.queries
     bf16_train = {
         "workload": bcfg.description, "step": "msda_forward + msda_backward, bf16 value and "
                                               "grad_output",
         "ms_per_step": round(bf16_ms, 4),
         "queries_per_s": round(world * bq / (bf16_ms * 1e-3), 1),
+        "fused_ms_per_step": round(bf16_fused_ms, 4),
+        "fused_step": "msda_fused_forward + msda_fused_backward on the same workload's raw "
+                      "reference points, offsets and logits (reference points detached)",
         "steps": n_fused,
     }
 

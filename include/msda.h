@@ -271,7 +271,10 @@ msda_status msda_fused_forward(int64_t B, int64_t S, int64_t M, int64_t D, int64
  * The derivative is that of the real-number formula (the float32 rounding of
  * loc is not differentiated); the pages print no backward.
  *
- *   value_dtype must be MSDA_F32, D <= 128 (as msda_backward)
+ *   value_dtype MSDA_F32, or MSDA_BF16 (value and grad_output bfloat16, 8-byte
+ *       aligned; the arithmetic and every gradient stay float32, as in
+ *       msda_backward); D <= 128 (as msda_backward)
+ *   grad_output              [B, Lq, M * D]        value_dtype
  *   grad_value               [B, S, M, D]          overwritten (zeroed, then
  *                                                  atomics; 16-byte aligned)
  *   grad_sampling_offsets    [B, Lq, M, L, K, 2]   overwritten (8-byte aligned)
@@ -288,7 +291,7 @@ msda_status msda_fused_backward(int64_t B, int64_t S, int64_t M, int64_t D, int6
                                 const int64_t *level_start_index,
                                 const float *reference_points,
                                 const float *sampling_offsets,
-                                const float *attention_logits, const float *grad_output,
+                                const float *attention_logits, const void *grad_output,
                                 float *grad_value, float *grad_sampling_offsets,
                                 float *grad_attention_logits,
                                 float *grad_reference_points, void *stream);

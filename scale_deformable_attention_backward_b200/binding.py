@@ -352,14 +352,17 @@ def fused_backward(value: torch.Tensor, spatial_shapes, level_start_index,
                    reference_grad: bool = True):
     """Backward of :func:`fused_forward` (``msda_fused_backward``): returns
     (grad_value, grad_sampling_offsets, grad_attention_logits,
-    grad_reference_points or None), all float32."""
+    grad_reference_points or None), all float32.  value and grad_output are both
+    float32 or both bfloat16."""
     dev = value.device
     B, S, M, D, Lq, L, K, R = _fused_dims(value, reference_points, sampling_offsets,
                                           attention_logits)
-    _require(value, "value", torch.float32, dev)
+    _require(value, "value", None, dev)
+    code = _value_code(value)
     for t, name in ((reference_points, "reference_points"), (sampling_offsets, "sampling_offsets"),
-                    (attention_logits, "attention_logits"), (grad_output, "grad_output")):
+                    (attention_logits, "attention_logits")):
         _require(t, name, torch.float32, dev)
+    _require(grad_output, "grad_output", value.dtype, dev)
     if tuple(grad_output.shape) != (B, Lq, M * D):
         raise ValueError("grad_output must be [B, Lq, M*D]")
     ss, st = _metadata(spatial_shapes, level_start_index, S, dev)
@@ -371,7 +374,7 @@ def fused_backward(value: torch.Tensor, spatial_shapes, level_start_index,
     gref = torch.empty((B, Lq, L, R), dtype=torch.float32, device=dev) if reference_grad else None
     with torch.cuda.device(dev):
         stream = torch.cuda.current_stream(dev).cuda_stream
-        _check(library().msda_fused_backward(B, S, M, D, Lq, L, K, R, MSDA_F32, _ptr(value),
+        _check(library().msda_fused_backward(B, S, M, D, Lq, L, K, R, code, _ptr(value),
                                              _ptr(ss), _ptr(st), _ptr(reference_points),
                                              _ptr(sampling_offsets), _ptr(attention_logits),
                                              _ptr(grad_output), _ptr(gv), _ptr(goff), _ptr(gz),
@@ -397,9 +400,10 @@ class MSDeformAttnFusedFunction(torch.autograd.Function):
         value, ref, off, logits = ctx.saved_tensors
         ss, st = ctx.meta
         gv, goff, gz, gref = fused_backward(value, ss, st, ref, off, logits,
-                                            grad_output.contiguous(),
+                                            grad_output.to(value.dtype).contiguous(),
                                             reference_grad=ctx.needs_input_grad[3])
-        return gv, None, None, gref, goff, gz
+        # The op returns float32 gradients; autograd wants value's dtype.
+        return gv.to(value.dtype), None, None, gref, goff, gz
 
 
 def ms_deform_attn_fused(value, spatial_shapes, level_start_index, reference_points,

@@ -375,14 +375,15 @@ msda_status msda_fused_backward(int64_t B, int64_t S, int64_t M, int64_t D, int6
                                 const void* value, const int64_t* spatial_shapes,
                                 const int64_t* level_start_index, const float* reference_points,
                                 const float* sampling_offsets, const float* attention_logits,
-                                const float* grad_output, float* grad_value,
+                                const void* grad_output, float* grad_value,
                                 float* grad_sampling_offsets, float* grad_attention_logits,
                                 float* grad_reference_points, void* stream) {
   Common c;
   msda_status st = check_common(B, S, M, D, Lq, L, K, &c);
   if (st != MSDA_OK) return st;
   if (R != 2 && R != 4) return MSDA_ERR_BAD_SHAPE;
-  if (value_dtype != MSDA_F32) return MSDA_ERR_UNSUPPORTED;
+  if (value_dtype != MSDA_F32 && value_dtype != MSDA_BF16) return MSDA_ERR_UNSUPPORTED;
+  const uintptr_t in_align = value_dtype == MSDA_F32 ? 16 : 8;
   if (D % 4 != 0 || D > 128 || M > INT32_MAX) return MSDA_ERR_UNSUPPORTED;
   int64_t ref_elems = 0;
   if (!product_ok({B, Lq, L, R}, &ref_elems)) return MSDA_ERR_BAD_SHAPE;
@@ -395,7 +396,7 @@ msda_status msda_fused_backward(int64_t B, int64_t S, int64_t M, int64_t D, int6
                attention_logits == nullptr || grad_output == nullptr ||
                grad_sampling_offsets == nullptr || grad_attention_logits == nullptr))
     return MSDA_ERR_NULL_POINTER;
-  if (work && (!aligned(value, 16) || !aligned(grad_output, 16) ||
+  if (work && (!aligned(value, in_align) || !aligned(grad_output, in_align) ||
                !aligned(sampling_offsets, 8) || !aligned(grad_sampling_offsets, 8) ||
                !aligned(reference_points, 4) || !aligned(attention_logits, 4) ||
                !aligned(grad_attention_logits, 4) || !aligned(spatial_shapes, 8) ||
@@ -413,6 +414,7 @@ msda_status msda_fused_backward(int64_t B, int64_t S, int64_t M, int64_t D, int6
   a.sampling_offsets = sampling_offsets;
   a.attention_logits = attention_logits;
   a.grad_output = grad_output;
+  a.bf16 = value_dtype == MSDA_BF16;
   a.grad_value = grad_value;
   a.grad_sampling_offsets = grad_sampling_offsets;
   a.grad_attention_logits = grad_attention_logits;

@@ -149,19 +149,21 @@ fused_forward_kernel(const T* __restrict__ value, const int64_t* __restrict__ sp
 // tile's weights.  grad_logits holds dA until the group's sum_j A_j dA_j is
 // known, then d z.  Lane i of a group combines (and later revisits) the points
 // p with p % LANES == i.
-template <int LANES>
+// T: dtype of value and grad_output (float32, or bfloat16 read 8 bytes per
+// lane); arithmetic and every gradient are float32 for both.
+template <typename T, int LANES>
 __global__ void __launch_bounds__(kThreads)
-fused_backward_kernel(const float* __restrict__ value, const int64_t* __restrict__ spatial_shapes,
+fused_backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial_shapes,
                       const int64_t* __restrict__ level_start_index,
                       const float* __restrict__ reference_points,
                       const float* __restrict__ sampling_offsets,
                       const float* __restrict__ attention_logits,
-                      const float* __restrict__ grad_output, float* __restrict__ grad_value,
+                      const T* __restrict__ grad_output, float* __restrict__ grad_value,
                       float* __restrict__ grad_offsets, float* __restrict__ grad_logits,
                       float* __restrict__ grad_reference, long long S, int M, int D,
                       long long Lq, int L, int K, int R, long long groups) {
-  using V = Vec<float>;
-  constexpr int E = V::N;
+  using V = Vec4<T>;
+  constexpr int E = 4;
   constexpr int G = kThreads / LANES;
   constexpr int PC = kChunkPoints / G;
   constexpr int PER = kChunkPoints / kThreads;
@@ -188,7 +190,7 @@ fused_backward_kernel(const float* __restrict__ value, const int64_t* __restrict
     const int ch = lane * E;
     const bool lane_on = active && ch < D;
     const long long vofs = (grp.b * S * M + grp.m) * static_cast<long long>(D) + ch;
-    const float* vbase = value + vofs;
+    const T* vbase = value + vofs;
     float* gvbase = grad_value + vofs;
     const float* zg = attention_logits + grp.bqm * LK;
     const float2 nz = softmax_norm<LANES>(zg, LK, lane);
@@ -378,17 +380,31 @@ cudaError_t fused_forward_lanes(const FusedArgs& a, cudaStream_t stream) {
   }
 }
 
-template <int LANES>
+template <typename T, int LANES>
 cudaError_t launch_fused_backward_t(const FusedArgs& a, cudaStream_t stream) {
   const long long per_block = kThreads / LANES;
   long long blocks = (a.groups + per_block - 1) / per_block;
   if (blocks > (1ll << 30)) blocks = 1ll << 30;
-  fused_backward_kernel<LANES><<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(
-      static_cast<const float*>(a.value), a.spatial_shapes, a.level_start_index,
-      a.reference_points, a.sampling_offsets, a.attention_logits, a.grad_output, a.grad_value,
+  fused_backward_kernel<T, LANES><<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(
+      static_cast<const T*>(a.value), a.spatial_shapes, a.level_start_index,
+      a.reference_points, a.sampling_offsets, a.attention_logits,
+      static_cast<const T*>(a.grad_output), a.grad_value,
       a.grad_sampling_offsets, a.grad_attention_logits, a.grad_reference_points, a.S, a.M, a.D,
       a.Lq, a.L, a.K, a.R, a.groups);
   return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t fused_backward_lanes(const FusedArgs& a, cudaStream_t stream) {
+  switch (a.lanes) {
+    case 1: return launch_fused_backward_t<T, 1>(a, stream);
+    case 2: return launch_fused_backward_t<T, 2>(a, stream);
+    case 4: return launch_fused_backward_t<T, 4>(a, stream);
+    case 8: return launch_fused_backward_t<T, 8>(a, stream);
+    case 16: return launch_fused_backward_t<T, 16>(a, stream);
+    case 32: return launch_fused_backward_t<T, 32>(a, stream);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace
@@ -411,15 +427,8 @@ cudaError_t launch_fused_backward(const FusedArgs& a, cudaStream_t stream) {
     if (err != cudaSuccess) return err;
   }
   if (a.groups == 0) return cudaSuccess;
-  switch (a.lanes) {
-    case 1: return launch_fused_backward_t<1>(a, stream);
-    case 2: return launch_fused_backward_t<2>(a, stream);
-    case 4: return launch_fused_backward_t<4>(a, stream);
-    case 8: return launch_fused_backward_t<8>(a, stream);
-    case 16: return launch_fused_backward_t<16>(a, stream);
-    case 32: return launch_fused_backward_t<32>(a, stream);
-    default: return cudaErrorInvalidValue;
-  }
+  return a.bf16 ? fused_backward_lanes<__nv_bfloat16>(a, stream)
+                : fused_backward_lanes<float>(a, stream);
 }
 
 }  // namespace msda

@@ -59,7 +59,7 @@ struct FusedArgs {
   int chunks;                      // forward channel chunks per (b, q, m); 1 for the backward
   long long groups;                // B * Lq * M * chunks
   void* output;                    // forward
-  const float* grad_output;        // backward
+  const void* grad_output;         // backward: value's dtype
   float* grad_value;
   float* grad_sampling_offsets;
   float* grad_attention_logits;

@@ -179,9 +179,13 @@ def test_fused_argument_errors(lib):
     assert _ffwd(lib, B=-1) == BAD
     assert _ffwd(lib, L=17) == UNSUP and _fbwd(lib, K=65) == UNSUP
     assert _ffwd(lib, D=6) == UNSUP
-    # The backward is float32 only, D <= 128; the forward also takes bfloat16.
-    assert _fbwd(lib, dtype=1) == UNSUP
+    # Both passes take float32 or bfloat16 value; the backward needs D <= 128.
+    assert _fbwd(lib, dtype=2) == UNSUP
     assert _fbwd(lib, D=132) == UNSUP
+    for i in (0, 6):                        # bfloat16 value / grad_output: 8-byte aligned
+        ptrs = [FAKE] * 11
+        ptrs[i] = FAKE + 4
+        assert _fbwd(lib, dtype=1, ptrs=ptrs) == MISAL, i
     # Every required pointer; grad_reference_points (the 11th) may be NULL.
     for i in range(7):
         ptrs = [FAKE] * 7

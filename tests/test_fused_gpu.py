@@ -88,6 +88,19 @@ def test_fused_backward_matches_oracle_full_size(name):
     check_fused_backward(inp, fused_device(inp), f"{name} fused")
 
 
+def test_fused_backward_bf16_matches_oracle_full_size():
+    """The bf16 training workload through the fused backward: bfloat16 value and
+    grad_output (the oracle reads the same values widened exactly), float32
+    arithmetic and gradients, so the float32 backward tolerances apply."""
+    import dataclasses
+    inp = W.make_fused_inputs(W.CONFIGS["encoder_train_bf16"], seed=0)
+    bits = W.bf16_round_bits(inp.grad_output)
+    inp = dataclasses.replace(inp, grad_output=W.bf16_bits_to_f32(bits))
+    d = fused_device(inp)
+    d["grad_output"] = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).cuda()
+    check_fused_backward(inp, d, "encoder_train_bf16 fused")
+
+
 def _random_fused(rng, B, Lq, M, D, K, shapes, R):
     ss, st = W.level_metadata(shapes)
     S = int((ss[:, 0] * ss[:, 1]).sum())
