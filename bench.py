@@ -551,6 +551,11 @@ def run_b200(args, world, rank, local):
         binding.output_projection(px, pw, pb, out=py)
 
     proj_ms = max_over_ranks(time_steps(proj_step, n_fused), world, device)
+
+    def proj_f32_step():
+        binding.output_projection(px, pw, pb, out=py, precise=True)
+
+    proj_f32_ms = max_over_ranks(time_steps(proj_f32_step, n_fused), world, device)
     proj_rows = B * Lq
     proj_bytes = proj_rows * M * D * 4 * 2 + M * D * M * D * 4 + M * D * 4
     proj_flops = 2.0 * proj_rows * (M * D) * (M * D)
@@ -569,6 +574,11 @@ def run_b200(args, world, rank, local):
                    "tf32_peak_tflops": round(tf32_peak, 1),
                    "peak_source": f"{bf16_source} bf16 burst x nominal tf32/bf16 ratio "
                                   f"1.1/2.25"},
+        "precise": {"kernel": "proj_kernel<true>: float32 accuracy from 3 x TF32 MMAs, operands "
+                              "split into TF32 heads and float32 remainders in shared memory",
+                    "mean_ms": round(proj_f32_ms, 4),
+                    "achieved_gbs": round(proj_bytes / (proj_f32_ms * 1e-3) / 1e9, 1),
+                    "achieved_tflops_3x": round(3 * proj_flops / (proj_f32_ms * 1e-3) / 1e12, 1)},
     }
 
     # The bfloat16 training step (value and grad_output bf16; float32 arithmetic and

@@ -220,6 +220,22 @@ msda_status msda_output_projection(int64_t rows, int64_t c_in, int64_t c_out, co
                                    void *stream);
 
 /*
+ * The same Linear layer at float32 accuracy (the pages' output_proj is a
+ * float32 nn.Linear), still on the tensor cores: every operand element is split
+ * into its TF32 head (its 13 low mantissa bits cleared) and the float32
+ * remainder, and each K step takes three kind::tf32 MMAs, hi_x hi_w + hi_x lo_w +
+ * lo_x hi_w, accumulated in float32.  The dropped lo_x lo_w term and the TF32
+ * reading of the remainders leave each product within about 3 * 2^-20 of
+ * |x w|; the float32 accumulation adds its own rounding, so
+ * |error| <= 1e-5 * sum_k |x[r,k] * weight[n,k]| holds with margin for
+ * c_in <= 4096.  Arguments, limits, status codes and the bounded waits
+ * (msda_output_projection_check) as for msda_output_projection.
+ */
+msda_status msda_output_projection_f32(int64_t rows, int64_t c_in, int64_t c_out,
+                                       const float *x, const float *weight, const float *bias,
+                                       float *y, void *stream);
+
+/*
  * *failed = 1 if a projection since the last check gave up waiting (for a
  * copy, an MMA or its epilogue), else 0; clears the flag.  Synchronises with the device (it copies the
  * flag to the host).

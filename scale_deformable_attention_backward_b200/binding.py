@@ -40,6 +40,7 @@ SIGNATURES = {
     "msda_fused_forward": (_I32, [_I64] * 8 + [_I32] + [_VP] * 8),
     "msda_fused_backward": (_I32, [_I64] * 8 + [_I32] + [_VP] * 12),
     "msda_output_projection": (_I32, [_I64] * 3 + [_VP] * 5),
+    "msda_output_projection_f32": (_I32, [_I64] * 3 + [_VP] * 5),
     "msda_output_projection_check": (_I32, [ctypes.POINTER(_I32)]),
     "msda_wait_check": (_I32, [ctypes.POINTER(_I32)]),
     "msda_check_metadata": (_I32, [_I64, _I64, _VP, _VP]),
@@ -415,10 +416,11 @@ def ms_deform_attn_fused(value, spatial_shapes, level_start_index, reference_poi
 
 
 def output_projection(x: torch.Tensor, weight: torch.Tensor, bias: Optional[torch.Tensor] = None,
-                      out: Optional[torch.Tensor] = None) -> torch.Tensor:
+                      out: Optional[torch.Tensor] = None, precise: bool = False) -> torch.Tensor:
     """The Linear layer after the op on the tensor cores (``msda_output_projection``):
     ``x [..., c_in] @ weight[c_out, c_in].T + bias``, float32 in and out (TF32
-    products, float32 sums)."""
+    products, float32 sums).  ``precise=True`` calls ``msda_output_projection_f32``:
+    float32 accuracy from three TF32 products per step."""
     dev = x.device
     if x.dim() < 1 or weight.dim() != 2:
         raise ValueError("x must be [..., c_in] and weight [c_out, c_in]")
@@ -441,9 +443,10 @@ def output_projection(x: torch.Tensor, weight: torch.Tensor, bias: Optional[torc
             raise ValueError("out must be [..., c_out]")
     with torch.cuda.device(dev):
         stream = torch.cuda.current_stream(dev).cuda_stream
-        _check(library().msda_output_projection(rows, c_in, c_out, _ptr(x), _ptr(weight),
-                                                _ptr(bias), _ptr(out), ctypes.c_void_p(stream)),
-               "msda_output_projection")
+        fn = library().msda_output_projection_f32 if precise else library().msda_output_projection
+        _check(fn(rows, c_in, c_out, _ptr(x), _ptr(weight), _ptr(bias), _ptr(out),
+                  ctypes.c_void_p(stream)),
+               "msda_output_projection_f32" if precise else "msda_output_projection")
     return out
 
 

@@ -76,6 +76,28 @@ msda_status check_common(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq,
   return MSDA_OK;
 }
 
+msda_status output_projection(int64_t rows, int64_t c_in, int64_t c_out, const float* x,
+                              const float* weight, const float* bias, float* y, bool precise,
+                              void* stream) {
+  if (rows < 0 || c_in < 0 || c_out < 0) return MSDA_ERR_BAD_SHAPE;
+  if (c_in % 8 != 0 || c_in < 8 || c_in > 4096 || c_out % 16 != 0 || c_out < 16 ||
+      c_out > 256 || rows > static_cast<int64_t>(INT32_MAX) - 128)
+    return MSDA_ERR_UNSUPPORTED;
+  int64_t xe = 0, ye = 0;
+  if (!product_ok({rows, c_in}, &xe) || !product_ok({rows, c_out}, &ye))
+    return MSDA_ERR_BAD_SHAPE;
+  if (rows == 0) return MSDA_OK;
+  if (x == nullptr || weight == nullptr || y == nullptr) return MSDA_ERR_NULL_POINTER;
+  if (!aligned(x, 16) || !aligned(weight, 16) || !aligned(y, 16) || !aligned(bias, 4))
+    return MSDA_ERR_MISALIGNED;
+  return msda::launch_projection(x, weight, bias, y, rows, static_cast<int>(c_in),
+                                 static_cast<int>(c_out), precise,
+                                 static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? MSDA_OK
+             : MSDA_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
@@ -279,22 +301,13 @@ msda_status msda_backward_deterministic(int64_t B, int64_t S, int64_t M, int64_t
 msda_status msda_output_projection(int64_t rows, int64_t c_in, int64_t c_out, const float* x,
                                    const float* weight, const float* bias, float* y,
                                    void* stream) {
-  if (rows < 0 || c_in < 0 || c_out < 0) return MSDA_ERR_BAD_SHAPE;
-  if (c_in % 8 != 0 || c_in < 8 || c_in > 4096 || c_out % 16 != 0 || c_out < 16 ||
-      c_out > 256 || rows > static_cast<int64_t>(INT32_MAX) - 128)
-    return MSDA_ERR_UNSUPPORTED;
-  int64_t xe = 0, ye = 0;
-  if (!product_ok({rows, c_in}, &xe) || !product_ok({rows, c_out}, &ye))
-    return MSDA_ERR_BAD_SHAPE;
-  if (rows == 0) return MSDA_OK;
-  if (x == nullptr || weight == nullptr || y == nullptr) return MSDA_ERR_NULL_POINTER;
-  if (!aligned(x, 16) || !aligned(weight, 16) || !aligned(y, 16) || !aligned(bias, 4))
-    return MSDA_ERR_MISALIGNED;
-  return msda::launch_projection(x, weight, bias, y, rows, static_cast<int>(c_in),
-                                 static_cast<int>(c_out), static_cast<cudaStream_t>(stream)) ==
-                 cudaSuccess
-             ? MSDA_OK
-             : MSDA_ERR_CUDA;
+  return output_projection(rows, c_in, c_out, x, weight, bias, y, false, stream);
+}
+
+msda_status msda_output_projection_f32(int64_t rows, int64_t c_in, int64_t c_out,
+                                       const float* x, const float* weight, const float* bias,
+                                       float* y, void* stream) {
+  return output_projection(rows, c_in, c_out, x, weight, bias, y, true, stream);
 }
 
 msda_status msda_output_projection_check(int* failed) {

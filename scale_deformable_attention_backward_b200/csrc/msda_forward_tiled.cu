@@ -69,7 +69,6 @@ constexpr int kThreads = kProducers + kConsumers;
 constexpr int kStages = 2;
 constexpr int kMaxTileQueries = 128;
 constexpr int kStepPoints = 512;                  // queries x K per step, at most
-constexpr int kPer = kStepPoints / kProducers;    // points set up per producer thread
 constexpr int kMaxK = 8;                          // samples per level per query, at most
 // The consumers' records (int4 offsets + float4 weights) and per slot the raw points.
 constexpr int kRecordBytes = kStepPoints * 32 + kStages * kStepPoints * 16;

@@ -110,8 +110,10 @@ cudaError_t launch_zero(float* p, long long n, cudaStream_t stream);
 // Output projection Y = X Wt^T + bias on the tensor cores (msda_proj.cu):
 // rows x c_in float32 X, c_out x c_in Wt; c_in % 8 == 0, c_out % 16 == 0,
 // 16 <= c_out <= 256, all pointers 16-byte aligned (bias 4-byte, may be null).
+// precise: float32 accuracy from three TF32 products per step (3 x TF32).
 cudaError_t launch_projection(const float* x, const float* weight, const float* bias, float* y,
-                              long long rows, int c_in, int c_out, cudaStream_t stream);
+                              long long rows, int c_in, int c_out, bool precise,
+                              cudaStream_t stream);
 // Device address of the flag a projection CTA sets when its MMA wait times out.
 cudaError_t projection_failed_flag(int** flag);
 

@@ -25,6 +25,21 @@
 //                      the rows and releases the accumulator.
 // Two accumulators (2 x 256 of the SM's 512 tensor-memory columns) alternate
 // between tiles, so a tile's epilogue overlaps the next tile's loads and MMAs.
+//
+// Precise mode (PRECISE, msda_output_projection_f32): float32 accuracy from
+// three TF32 products.  Each operand is split into a TF32 head and a float32
+// remainder, x = hi + lo with hi = x with its 13 low mantissa bits cleared (so
+// x - hi is exact in float32 and |lo| < 2^-10 |x|), and
+//     x w ~ hi_x hi_w + hi_x lo_w + lo_x hi_w,
+// dropping lo_x lo_w (< 2^-20 |x w|); lo read as TF32 loses < 2^-10 |lo|.  Two
+// more warps do the split: the CTA has 384 threads, and warps 2..3 and 8..11 wait
+// for a stage's copies, rewrite its X and W elements as their heads in place and
+// write the remainders into a second buffer of the stage at the same (swizzled)
+// offsets, then arrive on the stage's "split" barrier, which the MMA issuer
+// waits for instead of "full".  The
+// heads are written back explicitly so that the split is exact whether the
+// tensor cores truncate or round a TF32 operand.  A stage then holds the four
+// operand buffers (96 KB), so two stages fit.
 // TMA fills rows and K columns past the end with zeros.  Every wait is bounded
 // in time: past the limit the waiting thread sets a flag that stops every role;
 // the CTA then waits (bounded again) for its copies and MMAs in flight, releases
@@ -55,6 +70,13 @@ constexpr int kProjStageBytes = kProjXBytes + kProjMaxOut * kProjChunk * 4;  // 
 constexpr int kProjOutBytes = 32 * 32 * 4;
 constexpr int kProjOutOffset = kProjStages * kProjStageBytes;
 constexpr int kProjSmemBytes = kProjOutOffset + 4 * 2 * kProjOutBytes + 1024;  // + alignment
+// Precise mode: two stages of X, W heads then X, W remainders.
+constexpr int kPreciseStages = 2;
+constexpr int kPreciseStageBytes = 2 * kProjStageBytes;  // 96 KB
+constexpr int kPreciseOutOffset = kPreciseStages * kPreciseStageBytes;
+constexpr int kPreciseSmemBytes = kPreciseOutOffset + 4 * 2 * kProjOutBytes + 1024;
+constexpr int kPreciseThreads = 384;
+constexpr int kSplitThreads = 192;  // warps 2..3 and 8..11
 constexpr uint32_t kAccColumns = 256;                           // per accumulator
 constexpr unsigned long long kProjWaitNs = 1000000000ull;       // 1 s per wait
 
@@ -64,6 +86,7 @@ struct ProjBarriers {
   uint64_t acc_full[2];         // an accumulator holds a finished tile
   uint64_t acc_empty[2];        // the 4 epilogue warps have read an accumulator
   uint64_t drain;               // every MMA issued has finished (failure path)
+  uint64_t split[kProjStages];  // precise mode: a stage's heads and remainders are written
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -141,6 +164,17 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t sr
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
 
+// D (tensor memory) [+]= A * B, kind::tf32, operands from shared-memory descriptors.
+__device__ __forceinline__ void mma_tf32(uint32_t d, uint64_t da, uint64_t db, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}"
+      :
+      : "r"(d), "l"(da), "l"(db), "r"(idesc), "r"(accumulate));
+}
+
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile(
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -165,10 +199,19 @@ __host__ __device__ constexpr uint32_t tf32_idesc(int n) {
          (static_cast<uint32_t>(kProjRows >> 4) << 24);
 }
 
-__global__ void __launch_bounds__(kProjThreads, 1)
+// The TF32 head of x: its 13 low mantissa bits cleared (x itself if not finite).
+__device__ __forceinline__ float tf32_head(float x) {
+  return isfinite(x) ? __int_as_float(__float_as_int(x) & static_cast<int>(0xffffe000u)) : x;
+}
+
+template <bool PRECISE>
+__global__ void __launch_bounds__(PRECISE ? kPreciseThreads : kProjThreads, 1)
 proj_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
             const __grid_constant__ CUtensorMap tmap_y, const float* __restrict__ bias,
             long long rows, int c_in, int c_out, int* __restrict__ status) {
+  constexpr int STAGES = PRECISE ? kPreciseStages : kProjStages;
+  constexpr int STAGE_BYTES = PRECISE ? kPreciseStageBytes : kProjStageBytes;
+  constexpr int OUT_OFFSET = PRECISE ? kPreciseOutOffset : kProjOutOffset;
   extern __shared__ unsigned char smem_raw[];
   __shared__ __align__(8) ProjBarriers bars;
   __shared__ uint32_t tmem_base;
@@ -186,9 +229,10 @@ proj_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   if (tid == 32) {
-    for (int s = 0; s < kProjStages; ++s) {
+    for (int s = 0; s < STAGES; ++s) {
       mbar_init(&bars.full[s], 1);
       mbar_init(&bars.empty[s], 1);
+      if (PRECISE) mbar_init(&bars.split[s], kSplitThreads);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&bars.acc_full[a], 1);
@@ -220,17 +264,17 @@ proj_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
       long long issued = 0;
       bool ok = true;
       for (long long g = 0; g < total; ++g) {
-        const int s = static_cast<int>(g % kProjStages);
-        // Stage s was last read by the MMAs of chunk g - kProjStages.
-        if (g >= kProjStages &&
-            !wait_bounded(&bars.empty[s], static_cast<uint32_t>((g / kProjStages - 1) & 1),
+        const int s = static_cast<int>(g % STAGES);
+        // Stage s was last read by the MMAs of chunk g - STAGES.
+        if (g >= STAGES &&
+            !wait_bounded(&bars.empty[s], static_cast<uint32_t>((g / STAGES - 1) & 1),
                           failed, failed)) {
           ok = false;
           break;
         }
         const long long tile = blockIdx.x + (g / nch) * gridDim.x;
         const int k0 = static_cast<int>(g % nch) * kProjChunk;
-        const uint32_t st = stages + static_cast<uint32_t>(s * kProjStageBytes);
+        const uint32_t st = stages + static_cast<uint32_t>(s * STAGE_BYTES);
         mbar_expect_tx(&bars.full[s], stage_tx);
         tma_load_2d(st, &tmap_x, k0, static_cast<int>(tile * kProjRows), &bars.full[s]);
         tma_load_2d(st + kProjXBytes, &tmap_w, k0, 0, &bars.full[s]);
@@ -241,14 +285,14 @@ proj_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
       // flight).  Then, on the normal path, wait for each stage's last MMA
       // commit, so that no MMA still reads shared memory and no arrival is
       // pending at exit.
-      const long long first = issued > kProjStages ? issued - kProjStages : 0;
+      const long long first = issued > STAGES ? issued - STAGES : 0;
       for (long long g = first; g < issued; ++g)
-        wait_bounded(&bars.full[g % kProjStages], static_cast<uint32_t>((g / kProjStages) & 1),
-                     failed, nullptr);
+        wait_bounded(&bars.full[g % STAGES], static_cast<uint32_t>((g / STAGES) & 1), failed,
+                     nullptr);
       if (ok)
         for (long long g = first; g < issued; ++g)
-          wait_bounded(&bars.empty[g % kProjStages],
-                       static_cast<uint32_t>((g / kProjStages) & 1), failed, failed);
+          wait_bounded(&bars.empty[g % STAGES], static_cast<uint32_t>((g / STAGES) & 1), failed,
+                       failed);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -268,26 +312,28 @@ proj_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         const uint32_t d = tmem + static_cast<uint32_t>(acc) * kAccColumns;
         for (int c = 0; c < nch; ++c, ++g) {
-          const int s = static_cast<int>(g % kProjStages);
-          if (!wait_bounded(&bars.full[s], static_cast<uint32_t>((g / kProjStages) & 1), failed,
-                            failed)) {
+          const int s = static_cast<int>(g % STAGES);
+          // Plain mode: the stage's copies have landed.  Precise mode: its
+          // heads and remainders have been written.
+          uint64_t* ready = PRECISE ? &bars.split[s] : &bars.full[s];
+          if (!wait_bounded(ready, static_cast<uint32_t>((g / STAGES) & 1), failed, failed)) {
             ok = false;
             break;
           }
           asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-          const uint32_t xa = stages + static_cast<uint32_t>(s * kProjStageBytes);
+          const uint32_t xa = stages + static_cast<uint32_t>(s * STAGE_BYTES);
           const uint32_t wa = xa + kProjXBytes;
           const int ksteps = min(kProjChunk, c_in - c * kProjChunk) / 8;
           for (int k = 0; k < ksteps; ++k) {
             const uint64_t da = sw128_desc(xa + 32 * k);
             const uint64_t db = sw128_desc(wa + 32 * k);
             const uint32_t accumulate = (c > 0 || k > 0) ? 1u : 0u;
-            asm volatile(
-                "{\n\t.reg .pred p;\n\t"
-                "setp.ne.b32 p, %4, 0;\n\t"
-                "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}"
-                :
-                : "r"(d), "l"(da), "l"(db), "r"(idesc), "r"(accumulate));
+            mma_tf32(d, da, db, idesc, accumulate);
+            if constexpr (PRECISE) {
+              // hi_x lo_w + lo_x hi_w (the remainders sit kProjStageBytes on).
+              mma_tf32(d, da, sw128_desc(wa + kProjStageBytes + 32 * k), idesc, 1u);
+              mma_tf32(d, sw128_desc(xa + kProjStageBytes + 32 * k), db, idesc, 1u);
+            }
           }
           mma_commit(&bars.empty[s]);
         }
@@ -300,14 +346,48 @@ proj_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
       }
     }
     __syncwarp();
-  } else if (warp >= 4) {
+  } else if (PRECISE && (warp == 2 || warp == 3 || warp >= 8)) {
+    // ---- splitter (precise mode) --------------------------------------------
+    const int t = warp < 8 ? tid - 64 : tid - 256 + 64;
+    const int n16 = (kProjXBytes + c_out * kProjChunk * 4) / 16;  // X then W, 16 bytes each
+    for (long long g = 0; g < total; ++g) {
+      const int s = static_cast<int>(g % STAGES);
+      const bool ok = wait_bounded(&bars.full[s], static_cast<uint32_t>((g / STAGES) & 1),
+                                   failed, failed);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      const uint32_t hi = stages + static_cast<uint32_t>(s * STAGE_BYTES);
+      const uint32_t lo = hi + kProjStageBytes;
+      for (int i = t; i < n16; i += kSplitThreads) {
+        float4 v;
+        asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                     : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                     : "r"(hi + 16 * i));
+        const float4 h = make_float4(tf32_head(v.x), tf32_head(v.y), tf32_head(v.z),
+                                     tf32_head(v.w));
+        // x - hi is exact; a non-finite x keeps all of itself in the head.
+        const float4 r = make_float4(isfinite(v.x) ? v.x - h.x : 0.0f,
+                                     isfinite(v.y) ? v.y - h.y : 0.0f,
+                                     isfinite(v.z) ? v.z - h.z : 0.0f,
+                                     isfinite(v.w) ? v.w - h.w : 0.0f);
+        asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(hi + 16 * i), "f"(h.x),
+                     "f"(h.y), "f"(h.z), "f"(h.w)
+                     : "memory");
+        asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(lo + 16 * i), "f"(r.x),
+                     "f"(r.y), "f"(r.z), "f"(r.w)
+                     : "memory");
+      }
+      // The MMAs read the stage through the async proxy.
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive(&bars.split[s]);
+    }
+  } else if (warp >= 4 && warp < 8) {
     // ---- epilogue -------------------------------------------------------------
     const int quarter = warp - 4;  // tcgen05.ld: warp w reaches lanes 32 (w % 4) .. + 31
     if (lane == 0)
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_y))
                    : "memory");
     const uint32_t out0 =
-        stages + static_cast<uint32_t>(kProjOutOffset + quarter * 2 * kProjOutBytes);
+        stages + static_cast<uint32_t>(OUT_OFFSET + quarter * 2 * kProjOutBytes);
     int nbuf = 0;  // blocks this warp has staged (buffer = nbuf & 1)
     for (long long lt = 0; lt < my_tiles; ++lt) {
       const int acc = static_cast<int>(lt & 1);
@@ -427,8 +507,10 @@ cudaError_t projection_failed_flag(int** flag) {
 }
 
 cudaError_t launch_projection(const float* x, const float* weight, const float* bias, float* y,
-                              long long rows, int c_in, int c_out, cudaStream_t stream) {
+                              long long rows, int c_in, int c_out, bool precise,
+                              cudaStream_t stream) {
   static_assert(kProjSmemBytes <= 227 * 1024, "the stages must fit one CTA");
+  static_assert(kPreciseSmemBytes + 256 <= 227 * 1024, "the precise stages must fit one CTA");
   if (rows == 0) return cudaSuccess;
   // Coordinates of the row tiles are 32-bit in the TMA instruction.
   if (rows > static_cast<long long>(INT32_MAX) - kProjRows) return cudaErrorInvalidValue;
@@ -443,12 +525,14 @@ cudaError_t launch_projection(const float* x, const float* weight, const float* 
   if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
   if ((err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
     return err;
-  if ((err = cudaFuncSetAttribute(proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  kProjSmemBytes)) != cudaSuccess)
+  const auto kernel = precise ? proj_kernel<true> : proj_kernel<false>;
+  const int smem = precise ? kPreciseSmemBytes : kProjSmemBytes;
+  if ((err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
+      cudaSuccess)
     return err;
   const long long tiles = (rows + kProjRows - 1) / kProjRows;
   const long long grid = tiles < sms ? tiles : sms;
-  proj_kernel<<<static_cast<unsigned>(grid), kProjThreads, kProjSmemBytes, stream>>>(
+  kernel<<<static_cast<unsigned>(grid), precise ? kPreciseThreads : kProjThreads, smem, stream>>>(
       map_x, map_w, map_y, bias, rows, c_in, c_out, status);
   return cudaGetLastError();
 }

@@ -248,11 +248,13 @@ def test_deterministic_backward_arguments(lib):
     assert _dbwd(lib, B=0, ptrs=[None] * 9, ws=None) == OK
 
 
-def test_output_projection_arguments(lib):
+@pytest.mark.parametrize("entry", ["msda_output_projection", "msda_output_projection_f32"])
+def test_output_projection_arguments(lib, entry):
     v = lambda p: None if p is None else ctypes.c_void_p(p)
+    fn = getattr(lib, entry)
 
     def proj(rows=128, c_in=256, c_out=256, x=FAKE, w=FAKE, b=FAKE, y=FAKE):
-        return lib.msda_output_projection(rows, c_in, c_out, v(x), v(w), v(b), v(y), None)
+        return fn(rows, c_in, c_out, v(x), v(w), v(b), v(y), None)
 
     # Every call below fails validation before any launch.
     assert proj(rows=-1) == BAD

@@ -16,7 +16,14 @@ parity arithmetic as the kernel:
 
 and checks that every role finishes, that no stage is refilled while its MMAs
 may still read it, and that no accumulator is overwritten before the epilogue
-has read it.  An mbarrier phase with parity P counts as complete while the
+has read it.
+
+The precise (3 x TF32) variant runs 2 stages and adds a splitter role between
+the copies and the MMAs:
+
+  splitter     chunk g waits full[g % S] for parity (g / S) & 1, splits the
+               stage into TF32 heads and remainders, then arrives on split[g % S]
+  MMA issuer   chunk g waits split[g % S] (instead of full) for parity (g / S) & 1  An mbarrier phase with parity P counts as complete while the
 barrier's current phase parity differs from P, as mbarrier.try_wait.parity
 defines it."""
 import random
@@ -44,10 +51,11 @@ class Barrier:
         return (self.phase & 1) != parity
 
 
-def run_protocol(tiles, chunks_per_tile, seed):
+def run_protocol(tiles, chunks_per_tile, seed, precise=False):
     rng = random.Random(seed)
-    S = STAGES
+    S = 2 if precise else STAGES
     full = [Barrier(1) for _ in range(S)]
+    split = [Barrier(1) for _ in range(S)]
     empty = [Barrier(1) for _ in range(S)]
     acc_full = [Barrier(1), Barrier(1)]
     acc_empty = [Barrier(EPILOGUE_WARPS), Barrier(EPILOGUE_WARPS)]
@@ -55,7 +63,7 @@ def run_protocol(tiles, chunks_per_tile, seed):
     stage_state = [None] * S          # None | ("loading", g) | ("landed", g) | ("used", g)
     acc_state = [None, None]          # None | "busy" | "full" | "read"
     copies, mma_work = [], []
-    st = {"pg": 0, "mg": 0, "mt": 0, "mc": 0}
+    st = {"pg": 0, "mg": 0, "mt": 0, "mc": 0, "sg": 0}
     epi = [0] * EPILOGUE_WARPS
     read_count = [0, 0]
 
@@ -81,9 +89,10 @@ def run_protocol(tiles, chunks_per_tile, seed):
             return False
         g = st["mg"]
         s = g % S
-        if not full[s].complete((g // S) & 1):
+        ready = split[s] if precise else full[s]
+        if not ready.complete((g // S) & 1):
             return False
-        assert stage_state[s] == ("landed", g), (g, stage_state[s])
+        assert stage_state[s] == (("split" if precise else "landed"), g), (g, stage_state[s])
         if st["mc"] == 0:
             assert acc_state[acc] in (None, "read"), (t, acc_state[acc])
             acc_state[acc] = "busy"
@@ -94,6 +103,19 @@ def run_protocol(tiles, chunks_per_tile, seed):
             mma_work.append(("tile", t, acc))
             st["mc"] = 0
             st["mt"] += 1
+        return True
+
+    def splitter():
+        g = st["sg"]
+        if not precise or g >= total:
+            return False
+        s = g % S
+        if not full[s].complete((g // S) & 1):
+            return False
+        assert stage_state[s] == ("landed", g), (g, stage_state[s])
+        stage_state[s] = ("split", g)
+        split[s].arrive()
+        st["sg"] += 1
         return True
 
     def epilogue(w):
@@ -136,7 +158,7 @@ def run_protocol(tiles, chunks_per_tile, seed):
             acc_full[acc].arrive()
         return True
 
-    actors = [producer, mma_issuer, tma_engine, tensor_core] + \
+    actors = [producer, mma_issuer, tma_engine, tensor_core, splitter] + \
              [lambda w=w: epilogue(w) for w in range(EPILOGUE_WARPS)]
     while True:
         order = actors[:]
@@ -150,10 +172,12 @@ def run_protocol(tiles, chunks_per_tile, seed):
         assert empty[g % S].complete((g // S) & 1)
 
 
+@pytest.mark.parametrize("precise", [False, True])
 @pytest.mark.parametrize("seed", range(60))
-def test_protocol_random_interleavings(seed):
+def test_protocol_random_interleavings(seed, precise):
     r = random.Random(1000 + seed)
-    run_protocol(tiles=r.randint(0, 7), chunks_per_tile=r.randint(1, 9), seed=seed)
+    run_protocol(tiles=r.randint(0, 7), chunks_per_tile=r.randint(1, 9), seed=seed,
+                 precise=precise)
 
 
 def test_protocol_catches_a_wrong_parity():
