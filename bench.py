@@ -259,33 +259,61 @@ def oracle_threaded(cfg: W.Config, n: int, threads: int):
     plain loops, unchanged; the foreign calls release the GIL).  Each run keeps
     its own grad_value, and the runs' grad_values are added at the end.
     Returns (queries/s, description)."""
+    inp = W.select_queries(W.make_inputs(cfg, seed=0, with_grad=True), np.arange(n))
+    step, parts = threaded_oracle_step(inp, threads)
+    t0 = time.perf_counter()
+    step()
+    dt = time.perf_counter() - t0
+    desc = (f"{cfg.name}: the same {n} queries of each of the B={cfg.B} images, in "
+            f"{parts} runs (one image, a range of its queries) on {threads} host threads "
+            f"(private grad_value per run, added per image), float64 oracle, {dt:.2f} s")
+    return cfg.B * n / dt, desc
+
+
+def threaded_oracle_step(inp, threads: int):
+    """A callable that runs the float64 oracle's forward + backward on `inp` from
+    `threads` host threads: the work is cut into runs of (one image, a range of its
+    queries), each run keeps its own grad_value of its image, and the runs'
+    grad_values are added per image at the end.  The oracle's C loops are
+    unchanged; its foreign calls release the GIL.  Returns (step, number of runs)."""
+    import dataclasses
     import oracle  # test infrastructure: used here only for the CPU baseline
     from concurrent.futures import ThreadPoolExecutor
-    inp = W.select_queries(W.make_inputs(cfg, seed=0, with_grad=True), np.arange(n))
     orc = oracle.default()
-    bounds = np.linspace(0, n, threads + 1).astype(int)
-    parts = [W.select_queries(inp, np.arange(lo, hi))
-             for lo, hi in zip(bounds[:-1], bounds[1:]) if hi > lo]
+    B = inp.value.shape[0]
+    n = inp.sampling_locations.shape[1]
+    per_image = max(1, -(-threads // B))
+    bounds = np.linspace(0, n, per_image + 1).astype(int)
+    runs = []
+    for b in range(B):
+        img = dataclasses.replace(
+            inp, value=inp.value[b:b + 1], sampling_locations=inp.sampling_locations[b:b + 1],
+            attention_weights=inp.attention_weights[b:b + 1],
+            grad_output=inp.grad_output[b:b + 1])
+        for lo, hi in zip(bounds[:-1], bounds[1:]):
+            if hi > lo:
+                runs.append((b, W.select_queries(img, np.arange(lo, hi))))
 
-    def run(sub):
+    def run(item):
+        b, sub = item
         orc.forward(sub.value, sub.spatial_shapes, sub.level_start_index,
                     sub.sampling_locations, sub.attention_weights)
         gv, _, _ = orc.backward(sub.value, sub.spatial_shapes, sub.level_start_index,
                                 sub.sampling_locations, sub.attention_weights,
                                 sub.grad_output)
-        return gv
+        return b, gv
 
-    with ThreadPoolExecutor(max_workers=len(parts)) as pool:
-        t0 = time.perf_counter()
-        grads = list(pool.map(run, parts))
-        total = grads[0]
-        for g in grads[1:]:
-            total += g
-        dt = time.perf_counter() - t0
-    desc = (f"{cfg.name}: the same {n} queries of each of the B={cfg.B} images, in "
-            f"{len(parts)} runs on {len(parts)} host threads (private grad_value per run, "
-            f"added at the end), float64 oracle, {dt:.2f} s")
-    return cfg.B * n / dt, desc
+    def step():
+        with ThreadPoolExecutor(max_workers=threads) as pool:
+            total = {}
+            for b, gv in pool.map(run, runs):
+                if b in total:
+                    total[b] += gv
+                else:
+                    total[b] = gv
+        return total
+
+    return step, len(runs)
 
 
 # ---------------------------------------------------------------------------
@@ -807,7 +835,9 @@ def run_b200(args, world, rank, local):
         "e2e": {"value": round(world * queries / (e2e_ms * 1e-3), 1), "unit": "queries/s",
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h),
-                "pipeline": "upload / compute / download on three streams, two buffer sets"},
+                "pipeline": "upload / compute / download on three streams, two buffer sets",
+                "api": "the Python binding of the C ABI (msda_forward, msda_backward) with torch "
+                       "tensors as memory; host buffers are pinned torch CPU tensors"},
         "gpu_launches": (1 + BACKWARD_LAUNCHES) * args.steps,
         "clocks": clocks.summary(),
         "wall_s_timed_region": round(wall, 3),
@@ -889,22 +919,18 @@ def run_case(args, local):
 
 
 def run_reference(args):
-    """The reference arm: the float64 oracle as it stands, on the host cores."""
+    """The reference arm: the float64 oracle as it stands, on all the host's cores
+    (threaded_oracle_step).  Each step is the whole workload when the run fits the
+    time budget, else the first n queries of every image."""
     cfg = W.CONFIGS[STEP_WORKLOAD]
     budget = 150.0
+    threads = host_threads()
     per_step = max(0.5, min(10.0, budget / max(1, args.steps + args.warmup)))
-    qps, desc, dt = oracle_sample(cfg, per_step_target_s=per_step)
-    # Warm-up and timed steps on the calibrated sample size.
-    import oracle
-    n = int(round(qps * dt / cfg.B))
+    # Calibrate on a sample: single-thread rate times the threads is the estimate.
+    qps1, _, _ = oracle_sample(cfg, target_s=2.0)
+    n = min(cfg.queries, max(64, int(qps1 * threads * 0.7 * per_step / cfg.B)))
     inp = W.select_queries(W.make_inputs(cfg, seed=0, with_grad=True), np.arange(n))
-    orc = oracle.default()
-
-    def step():
-        orc.forward(inp.value, inp.spatial_shapes, inp.level_start_index,
-                    inp.sampling_locations, inp.attention_weights)
-        orc.backward(inp.value, inp.spatial_shapes, inp.level_start_index,
-                     inp.sampling_locations, inp.attention_weights, inp.grad_output)
+    step, _ = threaded_oracle_step(inp, threads)
 
     for _ in range(args.warmup):
         step()
@@ -914,16 +940,19 @@ def run_reference(args):
     total = time.perf_counter() - t0
     ms = total / args.steps * 1e3
     value = cfg.B * n / (ms * 1e-3)
-    sample = (f"{cfg.name}: forward + backward of the first {n} of {cfg.queries} queries of "
-              f"each of the B={cfg.B} images per step, float64 oracle, single thread")
+    what = ("the whole workload" if n == cfg.queries else
+            f"the first {n} of {cfg.queries} queries of each of the B={cfg.B} images")
+    sample = (f"{cfg.name}: forward + backward of {what} per step, float64 oracle on {threads} "
+              f"host threads (runs of one image and a range of its queries, private grad_value "
+              f"per run)")
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "queries/s",
         "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded numpy; no dataset)",
         "config": {"workload": cfg.description, "step": "oracle forward + backward",
-                   "queries_per_step": cfg.B * n},
-        "cpu_baseline": {"value": round(value, 3), "unit": "queries/s", "cores": 1,
+                   "queries_per_step": cfg.B * n, "whole_workload": n == cfg.queries},
+        "cpu_baseline": {"value": round(value, 3), "unit": "queries/s", "cores": threads,
                          "kind": "oracle", "sample": sample, "host": host_cpu()},
         "e2e": {"value": round(value, 3), "unit": "queries/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
