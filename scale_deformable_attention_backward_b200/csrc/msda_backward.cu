@@ -94,7 +94,6 @@ backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial
   __shared__ int4 s_off[kBwdPoints];
   __shared__ float4 s_w[kBwdPoints];
   __shared__ float4 s_g[kBwdPoints];
-  stage_levels(lv, spatial_shapes, level_start_index, L, S);
   bool use_fixed = false;
   float scale = 1.0f;
   if constexpr (FIXED) {
@@ -119,6 +118,24 @@ backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial
     g = v / SPLIT;
     jr = jv * SPLIT + static_cast<int>(v - g * SPLIT);
   };
+
+  // The first unit's locations and weights are pulled into L2 before the level
+  // metadata is staged, so the two memory round trips overlap.
+  if (blockIdx.x < tiles) {
+#pragma unroll
+    for (int r = 0; r < PER; ++r) {
+      const int t = threadIdx.x + r * kBwdThreads;
+      const int tg = t / PC, tj = t % PC;
+      long long g;
+      int jr;
+      real_point(blockIdx.x * G + tg, tj, g, jr);
+      if (tj < min(PC, LKv) && g < groups && jr < LK) {
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(sampling_locations + 2 * (g * LK + jr)));
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(attention_weights + g * LK + jr));
+      }
+    }
+  }
+  stage_levels(lv, spatial_shapes, level_start_index, L, S);
 
   for (long long tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
     const long long v_raw = tile * G + gi;
@@ -197,7 +214,11 @@ backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial
       }
       __syncthreads();
 
-      // Phase 2: gathers, scatters and the corner dot products.
+      // Phase 2: gathers, scatters and the corner dot products.  The first
+      // scatter waits for the kernel that zeroes grad_value, which may still be
+      // running when this one starts (programmatic dependent launch; without it
+      // the wait returns at once).
+      if (!FIXED) asm volatile("griddepcontrol.wait;" ::: "memory");
       for (int j0 = 0; j0 < pc; j0 += LANES) {
         const int nb = min(LANES, pc - j0);
         float keep[4] = {0.0f, 0.0f, 0.0f, 0.0f};
@@ -265,6 +286,9 @@ backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial
 }
 
 __global__ void zero_kernel(float4* __restrict__ p, long long n4) {
+  // A kernel launched after this one with programmatic stream serialization may
+  // start now; it waits (griddepcontrol.wait) before touching p.
+  asm volatile("griddepcontrol.launch_dependents;");
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n4;
        i += static_cast<long long>(gridDim.x) * blockDim.x)
     p[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
@@ -386,12 +410,24 @@ static cudaError_t launch_backward_t(const BackwardArgs& a, unsigned long long* 
   long long blocks = (a.groups * split + per_block - 1) / per_block;
   if (blocks > (1ll << 30)) blocks = 1ll << 30;
   auto go = [&](auto kernel) {
-    kernel<<<static_cast<unsigned>(blocks), kBwdThreads, 0, stream>>>(
-        static_cast<const T*>(a.value), a.spatial_shapes, a.level_start_index,
-        a.sampling_locations, a.attention_weights, static_cast<const T*>(a.grad_output),
-        a.grad_value, a.grad_sampling_locations, a.grad_attention_weights, a.S, a.M, a.D,
-        a.Lq, a.L, a.K, a.groups, acc, header);
-    return cudaGetLastError();
+    // The plain backward overlaps its start (metadata, locations, corner loads)
+    // with the zeroing of grad_value launched just before it; the deterministic
+    // one reads the scale pass's header first, so it is launched plainly.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(blocks));
+    cfg.blockDim = dim3(kBwdThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = FIXED ? 0 : 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<const T*>(a.value), a.spatial_shapes,
+                              a.level_start_index, a.sampling_locations, a.attention_weights,
+                              static_cast<const T*>(a.grad_output), a.grad_value,
+                              a.grad_sampling_locations, a.grad_attention_weights, a.S, a.M,
+                              a.D, a.Lq, a.L, a.K, a.groups, acc, header);
   };
   if (split == 4) return go(backward_kernel<T, LANES, FIXED, 4>);
   if (split == 2) return go(backward_kernel<T, LANES, FIXED, 2>);

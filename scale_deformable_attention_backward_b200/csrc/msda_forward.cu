@@ -80,7 +80,6 @@ forward_body(const T* __restrict__ value, const int64_t* __restrict__ spatial_sh
   __shared__ Levels lv;
   __shared__ int4 s_off[2][kChunkPoints];
   __shared__ float4 s_w[2][kChunkPoints];
-  stage_levels(lv, spatial_shapes, level_start_index, L, S);
 
   const int lane = threadIdx.x % LANES;
   const int gi = threadIdx.x / LANES;
@@ -95,7 +94,6 @@ forward_body(const T* __restrict__ value, const int64_t* __restrict__ spatial_sh
   const int LKv = (LK + SPLIT - 1) / SPLIT;
   const long long tiles = (vgroups + G - 1) / G;
   long long tile = blockIdx.x;
-  if (tile >= tiles) return;
   int p0 = 0;
 
   // Prefetched inputs of the next unit's points.
@@ -169,7 +167,11 @@ forward_body(const T* __restrict__ value, const int64_t* __restrict__ spatial_sh
     }
   };
 
-  prefetch(tile, 0);
+  // The first unit's locations and weights are requested before the level
+  // metadata is staged, so the two memory round trips overlap.
+  if (tile < tiles) prefetch(tile, 0);
+  stage_levels(lv, spatial_shapes, level_start_index, L, S);
+  if (tile >= tiles) return;
   setup(tile, 0, 0);
   __syncthreads();
   int buf = 0;
