@@ -35,6 +35,64 @@ struct FixedHeader {
 static_assert(sizeof(FixedHeader) <= kFixedHeaderBytes, "header must fit its slot");
 
 constexpr int kBwdThreads = 256;
+
+// Weight of a corner whose grad_value contribution was merged into another
+// point's (a signalling NaN: float arithmetic never produces one).
+constexpr unsigned kNoScatterBits = 0x7f800001u;
+
+// Two points of one group and one level can share a corner pixel (same or
+// neighbouring cells).  Their grad_value contributions there are w1 gO and
+// w2 gO with the group's gO, so one reduction of (w1 + w2) gO does the work of
+// two.  The level's K = 4 points sit in 4 aligned consecutive lanes, each with
+// its cell (x0, y0), the mask vm of its corners that may merge (inside the map,
+// bit i + 2j for corner (x0 + i, y0 + j)) and its corner weights `w`.  Partner cells at
+// (dx, dy) with |dx|, |dy| <= 1 share corner c of this point with the
+// partner's corner c - dx - 2 dy.  The lowest lane holding a pixel adds the
+// others' weights to its own; the others mark theirs kNoScatterBits, which the
+// scatter skips while the gathers still read the corner.  A NaN or Inf weight
+// lands on the same pixel either way.  All 32 lanes of the warp must call this.
+__device__ __forceinline__ void merge_shared_corners(int x0, int y0, unsigned vm, float4& w) {
+  const int me = threadIdx.x & 3;
+  // y0 and vm in one word (y0 of a point with a corner in the map is below 2^22).
+  const unsigned ky = (static_cast<unsigned>(y0) << 4) | vm;
+  const float w0[4] = {w.x, w.y, w.z, w.w};
+  float sum[4] = {w.x, w.y, w.z, w.w};
+  unsigned merged = 0;
+#pragma unroll
+  for (int o = 1; o < 4; ++o) {
+    const int px = __shfl_xor_sync(kFullMask, x0, o, 4);
+    const unsigned pky = __shfl_xor_sync(kFullMask, ky, o, 4);
+    float pw[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) pw[c] = __shfl_xor_sync(kFullMask, w0[c], o, 4);
+    // Unsigned differences: a point with no corner in the map (vm = 0) may
+    // carry any cell, and it matches nothing below.
+    const unsigned ux = static_cast<unsigned>(px) - static_cast<unsigned>(x0);
+    const unsigned uy = static_cast<unsigned>(static_cast<int>(pky) >> 4) -
+                        static_cast<unsigned>(y0);
+    if (ux + 1u <= 2u && uy + 1u <= 2u) {
+      const int dx = static_cast<int>(ux), dy = static_cast<int>(uy);
+      const int sh = dx + 2 * dy;  // partner corner = this corner - sh
+      const unsigned mx = dx == 0 ? 15u : (dx > 0 ? 0xau : 0x5u);  // corners with x0 + i in both cells
+      const unsigned my = dy == 0 ? 15u : (dy > 0 ? 0xcu : 0x3u);
+      const unsigned pvm = pky & 15u;
+      const unsigned m = mx & my & vm & (sh >= 0 ? pvm << sh : pvm >> -sh) & 15u;
+      if ((me ^ o) < me) {
+        merged |= m;
+      } else {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int i = c - sh;
+          const float v = i == 0 ? pw[0] : i == 1 ? pw[1] : i == 2 ? pw[2] : pw[3];
+          if ((m >> c) & 1u) sum[c] += v;
+        }
+      }
+    }
+  }
+  const float skip = __uint_as_float(kNoScatterBits);
+  w = make_float4((merged & 1u) ? skip : sum[0], (merged & 2u) ? skip : sum[1],
+                  (merged & 4u) ? skip : sum[2], (merged & 8u) ? skip : sum[3]);
+}
 constexpr int kBwdPoints = 512;  // points set up per unit (two per thread)
 
 // T: dtype of value and grad_output (float32, or bfloat16 read 8 bytes per lane);
@@ -61,6 +119,11 @@ constexpr int kBwdPoints = 512;  // points set up per unit (two per thread)
 //              grad_x    = A W_l (Ex + fy Exy)
 //              grad_y    = A H_l (Ey + fx Exy)
 // These are the derivatives above, regrouped with hx + fx = hy + fy = 1.
+// In the float path with K = 4, phase 1 also merges the corners that two points
+// of one level share (merge_shared_corners), so such a pixel takes one
+// reduction of (w1 + w2) gO instead of two; on the encoder workloads that is
+// about one corner in nine.  The block is held to 5 per SM (48 registers),
+// which measured faster than the compiler's own choice.
 //
 // FIXED (the deterministic backward): each grad_value contribution A w_ij gO[d]
 // (the same float32 product as the default path) is multiplied by 2^e, rounded
@@ -73,7 +136,7 @@ constexpr int kBwdPoints = 512;  // points set up per unit (two per thread)
 // not finite (header->fixed == 0) the kernel falls back to float atomics into
 // grad_value: the NaN / Inf pattern does not depend on the order either.
 template <typename T, int LANES, bool FIXED, int SPLIT>
-__global__ void __launch_bounds__(kBwdThreads)
+__global__ void __launch_bounds__(kBwdThreads, 5)
 backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial_shapes,
                 const int64_t* __restrict__ level_start_index,
                 const float* __restrict__ sampling_locations,
@@ -101,6 +164,9 @@ backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial
     scale = header->scale;
   }
   const int dq = D / 4;
+  // Corners shared by two points of one level of one group are merged before the
+  // scatter (merge_shared_corners); the deterministic path scatters every corner.
+  constexpr bool kMerge = !FIXED && SPLIT == 1 && PC % 4 == 0;
 
   const int lane = threadIdx.x % LANES;
   const int gi = threadIdx.x / LANES;
@@ -184,14 +250,15 @@ backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial
         long long g;
         int jr;
         real_point(tile * G + tg, q0 + tj, g, jr);
-        if (SPLIT > 1 && tj < pc && g < groups && jr >= LK) {
-          // A subset's slot past its group's last point: no corner, no output.
-          const int slot = tj * G + (tg ^ (tj & 7));
-          s_off[slot] = make_int4(-1, -1, -1, -1);
-          s_w[slot] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-          s_g[slot] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-        }
-        if (tj < pc && g < groups && jr < LK) {
+        // A subset's slot past its group's last point (SPLIT > 1) is written
+        // with no corner and no output.
+        const bool live = tj < pc && g < groups && jr < LK;
+        int4 off = make_int4(-1, -1, -1, -1);
+        float4 w = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        float4 fg = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        int cx0 = 0, cy0 = 0;
+        unsigned vm = 0;
+        if (live) {
           const long long pidx = g * LK + jr;
           const float2 xy = __ldg(reinterpret_cast<const float2*>(sampling_locations) + pidx);
           const float a = __ldg(attention_weights + pidx);
@@ -201,15 +268,37 @@ backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial
           const float hx = 1.0f - c.fx, hy = 1.0f - c.fy;
           // Offsets only for corners inside the map (0 <= pixel < S).
           const int base = static_cast<int>(lv.start[l] + static_cast<long long>(c.y0) * W + c.x0);
-          int4 off;
           off.x = (c.vx0 && c.vy0) ? base * MD : -1;
           off.y = (c.vx1 && c.vy0) ? (base + 1) * MD : -1;
           off.z = (c.vx0 && c.vy1) ? (base + W) * MD : -1;
           off.w = (c.vx1 && c.vy1) ? (base + W + 1) * MD : -1;
+          w = make_float4(a * hx * hy, a * c.fx * hy, a * hx * c.fy, a * c.fx * c.fy);
+          cx0 = c.x0;
+          cy0 = c.y0;
+          vm = (off.x >= 0 ? 1u : 0u) | (off.y >= 0 ? 2u : 0u) | (off.z >= 0 ? 4u : 0u) |
+               (off.w >= 0 ? 8u : 0u);
+          fg = make_float4(c.fx, c.fy, a * static_cast<float>(W), a * static_cast<float>(H));
+        }
+        if constexpr (kMerge) {
+          // K = 4 and PC % 4 == 0: a level's points are 4 aligned lanes.
+          // A zero weight is not merged: 0 * gO is NaN where gO is infinite, and
+          // (0 + w2) gO would not be.
+          const unsigned nz = (w.x != 0.0f ? 1u : 0u) | (w.y != 0.0f ? 2u : 0u) |
+                              (w.z != 0.0f ? 4u : 0u) | (w.w != 0.0f ? 8u : 0u);
+          if (K == 4) merge_shared_corners(cx0, cy0, vm & nz, w);
+          // A corner outside the map scatters nothing either, so the scatter
+          // tests only the weight.
+          const float skip = __uint_as_float(kNoScatterBits);
+          if (off.x < 0) w.x = skip;
+          if (off.y < 0) w.y = skip;
+          if (off.z < 0) w.z = skip;
+          if (off.w < 0) w.w = skip;
+        }
+        if (live || (SPLIT > 1 && tj < pc && g < groups)) {
           const int slot = tj * G + (tg ^ (tj & 7));
           s_off[slot] = off;
-          s_w[slot] = make_float4(a * hx * hy, a * c.fx * hy, a * hx * c.fy, a * c.fx * c.fy);
-          s_g[slot] = make_float4(c.fx, c.fy, a * static_cast<float>(W), a * static_cast<float>(H));
+          s_w[slot] = w;
+          s_g[slot] = fg;
         }
       }
       __syncthreads();
@@ -252,7 +341,8 @@ backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial
             }
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-              if (os[i] >= 0) scatter(os[i], ws[i], go);
+              if (kMerge ? __float_as_uint(ws[i]) != kNoScatterBits : os[i] >= 0)
+                scatter(os[i], ws[i], go);
             }
           }
 #pragma unroll

@@ -5,12 +5,13 @@
 // "Deformable DETR Deformable Transformers for End-to-End Object Detection",
 // multi-scale deformable attention equation, sampled as in "Deformable DETR模型
 // 解读（附源码+论文）", ms_deform_attn_core_pytorch).  All three gradients of a
-// point are linear in the four corner dot products
-//     G_ij = sum_d gO[d] * V(x0 + i, y0 + j)[d]
-// of its cell:
-//     grad_attn  = hy (hx G00 + fx G10) + fy (hx G01 + fx G11)
-//     grad_loc.x = A W (hy (G10 - G00) + fy (G11 - G01))
-//     grad_loc.y = A H (hx (G01 - G00) + fx (G11 - G10))
+// point are linear in four sums over the channels of its cell's corners,
+// with the corner differences taken per channel (corner_sums):
+//     P = sum_d gO V00,  Ex = sum_d gO (V10 - V00),  Ey = sum_d gO (V01 - V00),
+//     Exy = sum_d gO (V11 - V01 - V10 + V00)
+//     grad_attn  = P + fx Ex + fy Ey + fx fy Exy
+//     grad_loc.x = A W (Ex + fy Exy)
+//     grad_loc.y = A H (Ey + fx Exy)
 // and its grad_value contribution to corner ij is A w_ij gO.  Points that
 // share a cell (the same (b, m, level, x0, y0)) add to the same four rows of
 // grad_value, so they are summed in registers first.
@@ -147,9 +148,10 @@ __device__ __forceinline__ int point_cell(const Cell& c, int W) {
 __global__ void __launch_bounds__(kThreads)
 hist_kernel(const int64_t* __restrict__ spatial_shapes, const int64_t* __restrict__ level_start,
             const float* __restrict__ sampling_locations,
-            const float* __restrict__ attention_weights, float* __restrict__ grad_loc,
+            const float* __restrict__ attention_weights,
+            const float* __restrict__ grad_output, float* __restrict__ grad_loc,
             float* __restrict__ grad_attn, int* __restrict__ counts, int* __restrict__ slots,
-            long long S, int M, long long Lq, int L, int K, long long cells_per_bm,
+            long long S, int M, int D, long long Lq, int L, int K, long long cells_per_bm,
             int chunks, long long keys) {
   extern __shared__ int hist[];
   __shared__ Levels lv;
@@ -194,14 +196,18 @@ hist_kernel(const int64_t* __restrict__ spatial_shapes, const int64_t* __restric
         if (cell >= lo && cell < lo + span) {
           __stcs(slots + p, atomicAdd(hist + (cell - lo), 1));
         } else if (cell < 0 && lo == 0) {
-          // No corner in the map: every corner dot product is 0.  The products
+          // No corner in the map: every corner sum is sum_d gO[d] * 0, which is 0,
+          // or NaN when the group's grad_output holds an Inf or NaN.  The products
           // with the weights keep the NaN of a non-finite location, as the
           // oracle does.
+          const float* g = grad_output + ((sg.b * Lq + q) * M + sg.m) * static_cast<long long>(D);
+          float z = 0.0f;
+          for (int d = 0; d < D; ++d) z += 0.0f * __ldg(g + d);
           const float a = __ldg(attention_weights + p);
-          grad_attn[p] = 0.0f * (c.fx + c.fy);
+          grad_attn[p] = 0.0f * (c.fx + c.fy) + z;
           reinterpret_cast<float2*>(grad_loc)[p] =
-              make_float2(a * static_cast<float>(W) * (0.0f * c.fy),
-                          a * static_cast<float>(H) * (0.0f * c.fx));
+              make_float2(a * static_cast<float>(W) * (0.0f * c.fy + z),
+                          a * static_cast<float>(H) * (0.0f * c.fx + z));
         }
       }
     }
@@ -428,12 +434,27 @@ __device__ __forceinline__ void red_row(float* p, const Row<CPL>& r, const bool 
                 make_float4(r.v[4 * h], r.v[4 * h + 1], r.v[4 * h + 2], r.v[4 * h + 3]));
 }
 
+// The four corner sums of a record over this lane's channels, with the corner
+// differences taken per channel before any sum (a common offset of the value
+// field cancels exactly, and an infinite grad_output channel meets one
+// difference, as in the pages' per-channel product):
+//   P = sum gO V00, Ex = sum gO (V10 - V00), Ey = sum gO (V01 - V00),
+//   Exy = sum gO ((V11 - V01) - (V10 - V00)).
 template <int CPL>
-__device__ __forceinline__ float dot_row(const Row<CPL>& a, const Row<CPL>& b) {
-  float s = a.v[0] * b.v[0];
+__device__ __forceinline__ void corner_sums(const Row<CPL>& go, const Row<CPL>& c00,
+                                            const Row<CPL>& c10, const Row<CPL>& c01,
+                                            const Row<CPL>& c11, float (&s)[4]) {
+  s[0] = s[1] = s[2] = s[3] = 0.0f;
 #pragma unroll
-  for (int i = 1; i < CPL; ++i) s = fmaf(a.v[i], b.v[i], s);
-  return s;
+  for (int i = 0; i < CPL; ++i) {
+    const float dx = c10.v[i] - c00.v[i];
+    const float dy = c01.v[i] - c00.v[i];
+    const float dxy = (c11.v[i] - c01.v[i]) - dx;
+    s[0] = fmaf(go.v[i], c00.v[i], s[0]);
+    s[1] = fmaf(go.v[i], dx, s[1]);
+    s[2] = fmaf(go.v[i], dy, s[2]);
+    s[3] = fmaf(go.v[i], dxy, s[3]);
+  }
 }
 
 template <int CPL>
@@ -642,10 +663,12 @@ cell_kernel(const float* __restrict__ value, const int64_t* __restrict__ spatial
           go.v[4 * h + 2] = x.z;
           go.v[4 * h + 3] = x.w;
         }
-      part[0][j] = dot_row(go, c00);
-      part[1][j] = dot_row(go, c10);
-      part[2][j] = dot_row(go, c01);
-      part[3][j] = dot_row(go, c11);
+      float cs[4];
+      corner_sums(go, c00, c10, c01, c11, cs);
+      part[0][j] = cs[0];
+      part[1][j] = cs[1];
+      part[2][j] = cs[2];
+      part[3][j] = cs[3];
       const float hx = 1.0f - fx, hy = 1.0f - fy;
       axpy_row(a * hx * hy, go, a00);
       axpy_row(a * fx * hy, go, a10);
@@ -676,12 +699,11 @@ cell_kernel(const float* __restrict__ value, const int64_t* __restrict__ spatial
     if (lane < NB && key_cur >= 0) {
       const int p = __float_as_int(rec_cur.x);
       const float a = rec_cur.y, fx = rec_cur.z, fy = rec_cur.w;
-      const float hx = 1.0f - fx, hy = 1.0f - fy;
-      const float g00 = part[0][0], g10 = part[1][0], g01 = part[2][0], g11 = part[3][0];
-      grad_attn[p] = fmaf(hy, fmaf(fx, g10, hx * g00), fy * fmaf(fx, g11, hx * g01));
+      const float P = part[0][0], Ex = part[1][0], Ey = part[2][0], Exy = part[3][0];
+      // The derivatives regrouped with hx + fx = hy + fy = 1.
+      grad_attn[p] = fmaf(fx, fmaf(fy, Exy, Ex), fmaf(fy, Ey, P));
       reinterpret_cast<float2*>(grad_loc)[p] =
-          make_float2(a * myW * fmaf(hy, g10 - g00, fy * (g11 - g01)),
-                      a * myH * fmaf(hx, g01 - g00, fx * (g11 - g10)));
+          make_float2(a * myW * fmaf(fy, Exy, Ex), a * myH * fmaf(fx, Exy, Ey));
     }
     rec_cur = rec_nxt;
     key_cur = key_nxt;
@@ -783,8 +805,9 @@ cudaError_t launch_backward_sorted(const BackwardArgs& a, void* workspace,
   const int chunks = static_cast<int>(w.chunks);
   hist_kernel<<<blocks, kThreads, cell_smem, stream>>>(
       a.spatial_shapes, a.level_start_index, a.sampling_locations, a.attention_weights,
-      a.grad_sampling_locations, a.grad_attention_weights, counts, slots, a.S, a.M, a.Lq, a.L,
-      a.K, w.cells_per_bm, chunks, w.keys);
+      static_cast<const float*>(a.grad_output), a.grad_sampling_locations,
+      a.grad_attention_weights, counts, slots, a.S, a.M, a.D, a.Lq, a.L, a.K, w.cells_per_bm,
+      chunks, w.keys);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   // Key-major positions from the chunk-major counts: per-key totals, their
   // exclusive scan, then each (key, chunk) run's offset.

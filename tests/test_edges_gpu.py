@@ -146,6 +146,74 @@ def test_locations_at_pixel_boundaries():
     G.check_backward_paths(d, inp, "at pixel boundaries")
 
 
+@pytest.mark.parametrize("special", ["finite", "nonfinite"])
+def test_points_sharing_corners(special):
+    """The four points of one level of one (b, q, m) placed in the same,
+    side-by-side and diagonal cells, also across the map's edges, so that their
+    corners coincide: the float backward merges such corners' grad_value
+    contributions (K = 4) before the scatter.  Every backward path against the
+    oracle; in the second case with NaN and Inf weights and an Inf grad_output
+    on groups whose corners are shared."""
+    shapes = [(6, 7), (3, 5), (1, 4), (2, 1)]
+    rng = np.random.default_rng(41)
+    B, M, D, K, Lq = 2, 3, 16, 4, 57
+    L = len(shapes)
+    loc = np.empty((B, Lq, M, L, K, 2), dtype=np.float32)
+    for l, (h, w) in enumerate(shapes):
+        cx = rng.integers(-1, w, size=(B, Lq, M))
+        cy = rng.integers(-1, h, size=(B, Lq, M))
+        for k in range(K):
+            same = rng.random((B, Lq, M)) < 0.3
+            dx = np.where(same, 0, rng.integers(-1, 2, size=(B, Lq, M)))
+            dy = np.where(same, 0, rng.integers(-1, 2, size=(B, Lq, M)))
+            # pixel coordinate loc * n - 0.5 inside cell c + d
+            loc[:, :, :, l, k, 0] = (cx + dx + rng.random((B, Lq, M)) + 0.5) / w
+            loc[:, :, :, l, k, 1] = (cy + dy + rng.random((B, Lq, M)) + 0.5) / h
+    inp = random_inputs(42, B, M, D, K, shapes, Lq)
+    attn = inp.attention_weights.copy()
+    go = inp.grad_output.copy()
+    if special == "nonfinite":
+        attn[0, 3, 1, 0, 2] = np.nan
+        attn[1, 5, 0, 1, 1] = np.inf
+        attn[1, 6, 2, 0, 0] = -np.inf
+        go[0, 7, 1 * D + 3] = np.inf
+        # Two points of that group on exact pixel centres of the 1 x 4 level: the
+        # corner they share has weight 0 in one of them, and 0 * Inf is NaN.
+        loc[0, 7, 1, 2, 0] = (1.5 / 4, 0.5)
+        loc[0, 7, 1, 2, 1] = (2.5 / 4, 0.5)
+    inp = dataclasses.replace(inp, sampling_locations=loc, attention_weights=attn,
+                              grad_output=go)
+    d = G.device_inputs(inp)
+    got, ref = G.gpu_forward(d), G.oracle_forward(inp)
+    if special == "nonfinite":
+        # An infinite weight: the pages scale the interpolated value, A * sum_c b_c V_c
+        # (+-Inf); the kernels fold A into the corner weights, sum_c (A b_c) V_c, which
+        # is NaN when the corner values differ in sign.  Elsewhere the outputs agree.
+        inf = np.isinf(ref)
+        assert np.all(np.isinf(got[inf]) | np.isnan(got[inf]))
+        got, ref = np.where(inf, 0.0, got), np.where(inf, 0.0, ref)
+    G.assert_forward_f32(got, ref)
+    if special == "finite":
+        G.check_backward_paths(d, inp, "shared corners")
+        return
+    # grad_value is a sum of products A w gO, so its NaN / +-Inf pattern does not
+    # depend on the order of the sums.  grad_attn and grad_loc sum over the
+    # channels first and combine the corner sums after (P + fx Ex + ...), where an
+    # Inf channel can meet Inf - Inf; the oracle combines per channel.  There NaN
+    # may stand for the oracle's +-Inf.
+    rv, rl, ra = G.oracle_backward(inp)
+    for path in G.backward_paths(d):
+        gv, gl, ga = G.gpu_backward(d, path)
+        for got_t, ref_t, name, relaxed in ((gv, rv, "grad_value", False),
+                                            (gl, rl, "grad_sampling_locations", True),
+                                            (ga, ra, "grad_attention_weights", True)):
+            inf = np.isinf(ref_t)
+            what = f"{name} shared corners, non-finite ({path})"
+            same = got_t[inf] == ref_t[inf]
+            assert np.all(same | np.isnan(got_t[inf]) if relaxed else same), what
+            G.assert_backward_f32(got_t[~inf], ref_t[~inf], what)
+
+
 def test_far_and_nonfinite_locations():
     inp = random_inputs(8, B=2, M=2, D=8, K=3, shapes=SHAPES[1], Lq=11)
     loc = inp.sampling_locations.copy()
