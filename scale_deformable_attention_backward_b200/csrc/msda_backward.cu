@@ -228,8 +228,10 @@ backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial
           return;
         }
       }
-      atomicAdd(reinterpret_cast<float4*>(gvbase + o),
-                make_float4(w * g[0], w * g[1], w * g[2], w * g[3]));
+      const float2 ww = make_float2(w, w);
+      const float2 lo = mul2(ww, make_float2(g[0], g[1]));
+      const float2 hi = mul2(ww, make_float2(g[2], g[3]));
+      atomicAdd(reinterpret_cast<float4*>(gvbase + o), make_float4(lo.x, lo.y, hi.x, hi.y));
     };
 
     float go[E];
@@ -327,18 +329,29 @@ backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial
               for (int e = 0; e < E; ++e) q[i][e] = 0.0f;
               if (os[i] >= 0) V::load(vbase + os[i], q[i]);
             }
+            // Corner differences per channel: a common offset of the value field
+            // cancels here exactly, not between large dot products.  Channel pairs
+            // go through the packed two-wide float32 unit.
+            float2 d2[4];
 #pragma unroll
-            for (int e = 0; e < E; ++e) {
-              // Corner differences per channel: a common offset of the value
-              // field cancels here exactly, not between large dot products.
-              const float dx = q[1][e] - q[0][e];            // V10 - V00
-              const float dy = q[2][e] - q[0][e];            // V01 - V00
-              const float dxy = (q[3][e] - q[2][e]) - dx;    // V11 - V01 - V10 + V00
-              dot[0] = fmaf(go[e], q[0][e], dot[0]);
-              dot[1] = fmaf(go[e], dx, dot[1]);
-              dot[2] = fmaf(go[e], dy, dot[2]);
-              dot[3] = fmaf(go[e], dxy, dot[3]);
+            for (int k = 0; k < 4; ++k) d2[k] = make_float2(0.0f, 0.0f);
+#pragma unroll
+            for (int h = 0; h < E / 2; ++h) {
+              const float2 v00 = make_float2(q[0][2 * h], q[0][2 * h + 1]);
+              const float2 v10 = make_float2(q[1][2 * h], q[1][2 * h + 1]);
+              const float2 v01 = make_float2(q[2][2 * h], q[2][2 * h + 1]);
+              const float2 v11 = make_float2(q[3][2 * h], q[3][2 * h + 1]);
+              const float2 dx = sub2(v10, v00);                 // V10 - V00
+              const float2 dy = sub2(v01, v00);                 // V01 - V00
+              const float2 dxy = sub2(sub2(v11, v01), dx);      // V11 - V01 - V10 + V00
+              const float2 g = make_float2(go[2 * h], go[2 * h + 1]);
+              d2[0] = fma2(g, v00, d2[0]);
+              d2[1] = fma2(g, dx, d2[1]);
+              d2[2] = fma2(g, dy, d2[2]);
+              d2[3] = fma2(g, dxy, d2[3]);
             }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) dot[k] = d2[k].x + d2[k].y;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               if (kMerge ? __float_as_uint(ws[i]) != kNoScatterBits : os[i] >= 0)
