@@ -36,63 +36,6 @@ static_assert(sizeof(FixedHeader) <= kFixedHeaderBytes, "header must fit its slo
 
 constexpr int kBwdThreads = 256;
 
-// Weight of a corner whose grad_value contribution was merged into another
-// point's (a signalling NaN: float arithmetic never produces one).
-constexpr unsigned kNoScatterBits = 0x7f800001u;
-
-// Two points of one group and one level can share a corner pixel (same or
-// neighbouring cells).  Their grad_value contributions there are w1 gO and
-// w2 gO with the group's gO, so one reduction of (w1 + w2) gO does the work of
-// two.  The level's K = 4 points sit in 4 aligned consecutive lanes, each with
-// its cell (x0, y0), the mask vm of its corners that may merge (inside the map,
-// bit i + 2j for corner (x0 + i, y0 + j)) and its corner weights `w`.  Partner cells at
-// (dx, dy) with |dx|, |dy| <= 1 share corner c of this point with the
-// partner's corner c - dx - 2 dy.  The lowest lane holding a pixel adds the
-// others' weights to its own; the others mark theirs kNoScatterBits, which the
-// scatter skips while the gathers still read the corner.  A NaN or Inf weight
-// lands on the same pixel either way.  All 32 lanes of the warp must call this.
-__device__ __forceinline__ void merge_shared_corners(int x0, int y0, unsigned vm, float4& w) {
-  const int me = threadIdx.x & 3;
-  // y0 and vm in one word (y0 of a point with a corner in the map is below 2^22).
-  const unsigned ky = (static_cast<unsigned>(y0) << 4) | vm;
-  const float w0[4] = {w.x, w.y, w.z, w.w};
-  float sum[4] = {w.x, w.y, w.z, w.w};
-  unsigned merged = 0;
-#pragma unroll
-  for (int o = 1; o < 4; ++o) {
-    const int px = __shfl_xor_sync(kFullMask, x0, o, 4);
-    const unsigned pky = __shfl_xor_sync(kFullMask, ky, o, 4);
-    float pw[4];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) pw[c] = __shfl_xor_sync(kFullMask, w0[c], o, 4);
-    // Unsigned differences: a point with no corner in the map (vm = 0) may
-    // carry any cell, and it matches nothing below.
-    const unsigned ux = static_cast<unsigned>(px) - static_cast<unsigned>(x0);
-    const unsigned uy = static_cast<unsigned>(static_cast<int>(pky) >> 4) -
-                        static_cast<unsigned>(y0);
-    if (ux + 1u <= 2u && uy + 1u <= 2u) {
-      const int dx = static_cast<int>(ux), dy = static_cast<int>(uy);
-      const int sh = dx + 2 * dy;  // partner corner = this corner - sh
-      const unsigned mx = dx == 0 ? 15u : (dx > 0 ? 0xau : 0x5u);  // corners with x0 + i in both cells
-      const unsigned my = dy == 0 ? 15u : (dy > 0 ? 0xcu : 0x3u);
-      const unsigned pvm = pky & 15u;
-      const unsigned m = mx & my & vm & (sh >= 0 ? pvm << sh : pvm >> -sh) & 15u;
-      if ((me ^ o) < me) {
-        merged |= m;
-      } else {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int i = c - sh;
-          const float v = i == 0 ? pw[0] : i == 1 ? pw[1] : i == 2 ? pw[2] : pw[3];
-          if ((m >> c) & 1u) sum[c] += v;
-        }
-      }
-    }
-  }
-  const float skip = __uint_as_float(kNoScatterBits);
-  w = make_float4((merged & 1u) ? skip : sum[0], (merged & 2u) ? skip : sum[1],
-                  (merged & 4u) ? skip : sum[2], (merged & 8u) ? skip : sum[3]);
-}
 constexpr int kBwdPoints = 512;  // points set up per unit (two per thread)
 
 // T: dtype of value and grad_output (float32, or bfloat16 read 8 bytes per lane);
@@ -228,10 +171,7 @@ backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial
           return;
         }
       }
-      const float2 ww = make_float2(w, w);
-      const float2 lo = mul2(ww, make_float2(g[0], g[1]));
-      const float2 hi = mul2(ww, make_float2(g[2], g[3]));
-      atomicAdd(reinterpret_cast<float4*>(gvbase + o), make_float4(lo.x, lo.y, hi.x, hi.y));
+      scatter_row4(gvbase + o, w, g);
     };
 
     float go[E];
@@ -259,7 +199,6 @@ backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial
         float4 w = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
         float4 fg = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
         int cx0 = 0, cy0 = 0;
-        unsigned vm = 0;
         if (live) {
           const long long pidx = g * LK + jr;
           const float2 xy = __ldg(reinterpret_cast<const float2*>(sampling_locations) + pidx);
@@ -277,25 +216,10 @@ backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial
           w = make_float4(a * hx * hy, a * c.fx * hy, a * hx * c.fy, a * c.fx * c.fy);
           cx0 = c.x0;
           cy0 = c.y0;
-          vm = (off.x >= 0 ? 1u : 0u) | (off.y >= 0 ? 2u : 0u) | (off.z >= 0 ? 4u : 0u) |
-               (off.w >= 0 ? 8u : 0u);
           fg = make_float4(c.fx, c.fy, a * static_cast<float>(W), a * static_cast<float>(H));
         }
-        if constexpr (kMerge) {
-          // K = 4 and PC % 4 == 0: a level's points are 4 aligned lanes.
-          // A zero weight is not merged: 0 * gO is NaN where gO is infinite, and
-          // (0 + w2) gO would not be.
-          const unsigned nz = (w.x != 0.0f ? 1u : 0u) | (w.y != 0.0f ? 2u : 0u) |
-                              (w.z != 0.0f ? 4u : 0u) | (w.w != 0.0f ? 8u : 0u);
-          if (K == 4) merge_shared_corners(cx0, cy0, vm & nz, w);
-          // A corner outside the map scatters nothing either, so the scatter
-          // tests only the weight.
-          const float skip = __uint_as_float(kNoScatterBits);
-          if (off.x < 0) w.x = skip;
-          if (off.y < 0) w.y = skip;
-          if (off.z < 0) w.z = skip;
-          if (off.w < 0) w.w = skip;
-        }
+        // K = 4 and PC % 4 == 0: a level's points are 4 aligned lanes.
+        if constexpr (kMerge) prepare_scatter_weights(cx0, cy0, off, K == 4, w);
         if (live || (SPLIT > 1 && tj < pc && g < groups)) {
           const int slot = tj * G + (tg ^ (tj & 7));
           s_off[slot] = off;
@@ -329,29 +253,7 @@ backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial
               for (int e = 0; e < E; ++e) q[i][e] = 0.0f;
               if (os[i] >= 0) V::load(vbase + os[i], q[i]);
             }
-            // Corner differences per channel: a common offset of the value field
-            // cancels here exactly, not between large dot products.  Channel pairs
-            // go through the packed two-wide float32 unit.
-            float2 d2[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) d2[k] = make_float2(0.0f, 0.0f);
-#pragma unroll
-            for (int h = 0; h < E / 2; ++h) {
-              const float2 v00 = make_float2(q[0][2 * h], q[0][2 * h + 1]);
-              const float2 v10 = make_float2(q[1][2 * h], q[1][2 * h + 1]);
-              const float2 v01 = make_float2(q[2][2 * h], q[2][2 * h + 1]);
-              const float2 v11 = make_float2(q[3][2 * h], q[3][2 * h + 1]);
-              const float2 dx = sub2(v10, v00);                 // V10 - V00
-              const float2 dy = sub2(v01, v00);                 // V01 - V00
-              const float2 dxy = sub2(sub2(v11, v01), dx);      // V11 - V01 - V10 + V00
-              const float2 g = make_float2(go[2 * h], go[2 * h + 1]);
-              d2[0] = fma2(g, v00, d2[0]);
-              d2[1] = fma2(g, dx, d2[1]);
-              d2[2] = fma2(g, dy, d2[2]);
-              d2[3] = fma2(g, dxy, d2[3]);
-            }
-#pragma unroll
-            for (int k = 0; k < 4; ++k) dot[k] = d2[k].x + d2[k].y;
+            corner_sums4(q, go, dot);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               if (kMerge ? __float_as_uint(ws[i]) != kNoScatterBits : os[i] >= 0)

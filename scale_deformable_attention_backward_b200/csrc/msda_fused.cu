@@ -151,8 +151,11 @@ fused_forward_kernel(const T* __restrict__ value, const int64_t* __restrict__ sp
 // p with p % LANES == i.
 // T: dtype of value and grad_output (float32, or bfloat16 read 8 bytes per
 // lane); arithmetic and every gradient are float32 for both.
+//
+// As in backward_kernel, the corners shared by two points of one level
+// (K = 4) are merged before the scatter, and the block is held to 5 per SM.
 template <typename T, int LANES>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 5)
 fused_backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial_shapes,
                       const int64_t* __restrict__ level_start_index,
                       const float* __restrict__ reference_points,
@@ -214,7 +217,12 @@ fused_backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ s
         const int t = threadIdx.x + r * kThreads;
         const int tg = t / PC, tj = t % PC;
         const long long g = tile * G + tg;
-        if (tj < pc && g < groups) {
+        const bool live = tj < pc && g < groups;
+        int4 off = make_int4(-1, -1, -1, -1);
+        float4 w = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        float4 fg = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        int cx0 = 0, cy0 = 0;
+        if (live) {
           const long long pidx = g * LK + q0 + tj;
           const int l = (q0 + tj) / K;
           const int H = lv.H[l], W = lv.W[l];
@@ -227,15 +235,22 @@ fused_backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ s
           const float hx = 1.0f - c.fx, hy = 1.0f - c.fy;
           // Offsets only for corners inside the map (0 <= pixel < S).
           const int base = static_cast<int>(lv.start[l] + static_cast<long long>(c.y0) * W + c.x0);
-          int4 off;
           off.x = (c.vx0 && c.vy0) ? base * MD : -1;
           off.y = (c.vx1 && c.vy0) ? (base + 1) * MD : -1;
           off.z = (c.vx0 && c.vy1) ? (base + W) * MD : -1;
           off.w = (c.vx1 && c.vy1) ? (base + W + 1) * MD : -1;
+          w = make_float4(a * hx * hy, a * c.fx * hy, a * hx * c.fy, a * c.fx * c.fy);
+          fg = make_float4(c.fx, c.fy, a, 0.0f);
+          cx0 = c.x0;
+          cy0 = c.y0;
+        }
+        // A level's K = 4 points are 4 aligned lanes (PC % 4 == 0).
+        prepare_scatter_weights(cx0, cy0, off, K == 4 && PC % 4 == 0, w);
+        if (live) {
           const int slot = tj * G + (tg ^ (tj & 7));
           s_off[slot] = off;
-          s_w[slot] = make_float4(a * hx * hy, a * c.fx * hy, a * hx * c.fy, a * c.fx * c.fy);
-          s_g[slot] = make_float4(c.fx, c.fy, a, 0.0f);
+          s_w[slot] = w;
+          s_g[slot] = fg;
         }
       }
       __syncthreads();
@@ -260,23 +275,10 @@ fused_backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ s
               for (int e = 0; e < E; ++e) q[i][e] = 0.0f;
               if (os[i] >= 0) V::load(vbase + os[i], q[i]);
             }
-#pragma unroll
-            for (int e = 0; e < E; ++e) {
-              // Corner differences per channel: a common offset of the value
-              // field cancels here exactly, not between large dot products.
-              const float dx = q[1][e] - q[0][e];            // V10 - V00
-              const float dy = q[2][e] - q[0][e];            // V01 - V00
-              const float dxy = (q[3][e] - q[2][e]) - dx;    // V11 - V01 - V10 + V00
-              dot[0] = fmaf(go[e], q[0][e], dot[0]);
-              dot[1] = fmaf(go[e], dx, dot[1]);
-              dot[2] = fmaf(go[e], dy, dot[2]);
-              dot[3] = fmaf(go[e], dxy, dot[3]);
-            }
+            corner_sums4(q, go, dot);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-              if (os[i] >= 0)
-                atomicAdd(reinterpret_cast<float4*>(gvbase + os[i]),
-                          make_float4(ws[i] * go[0], ws[i] * go[1], ws[i] * go[2], ws[i] * go[3]));
+              if (__float_as_uint(ws[i]) != kNoScatterBits) scatter_row4(gvbase + os[i], ws[i], go);
             }
           }
 #pragma unroll
