@@ -32,8 +32,8 @@
 //   1. hist    one block per (segment, chunk): the cell of each point and its slot
 //              among the chunk's points of that cell (shared-memory atomic);
 //              the chunk's per-cell counts go to counts[chunk][key] (coalesced
-//              rows).  Points with no corner in the map get their (zero or NaN)
-//              gradients here.
+//              rows).  no_corner_kernel, launched after it, gives the points
+//              with no corner in the map their (zero or NaN) gradients.
 //   2. offsets per-key totals over the chunks, their exclusive prefix sum (three
 //              launches), then counts[chunk][key] becomes the position of the
 //              (key, chunk) run in the sorted record array.
@@ -145,14 +145,104 @@ __device__ __forceinline__ int point_cell(const Cell& c, int W) {
   return ((c.vx0 || c.vx1) && (c.vy0 || c.vy1)) ? (c.y0 + 1) * (W + 1) + (c.x0 + 1) : -1;
 }
 
+// The gradients of the points with no corner in the map, which take no part in
+// the sort.  Every corner sum of such a point is sum_d gO[d] * 0: 0, or NaN when
+// the group's grad_output holds an Inf or NaN.  The products with the weights
+// keep the NaN of a non-finite location, as the oracle does.  Two streaming
+// passes, each with its loads issued ahead of their use:
+//   no_corner_kernel         the location-only gradients of every such point
+//                            (reads all locations and weights);
+//   nonfinite_output_kernel  reads grad_output once; a (rare) group whose row
+//                            holds an Inf or NaN makes its no-corner points' gradients NaN.
+// I: the point index type (32-bit when the points fit).
+constexpr int kNoCornerUnroll = 4;
+
+template <typename I>
+__global__ void __launch_bounds__(kThreads)
+no_corner_kernel(const int64_t* __restrict__ spatial_shapes, const int64_t* __restrict__ level_start,
+                 const float* __restrict__ sampling_locations,
+                 const float* __restrict__ attention_weights, float* __restrict__ grad_loc,
+                 float* __restrict__ grad_attn, long long S, int L, int K, I points) {
+  constexpr int U = kNoCornerUnroll;
+  __shared__ Levels lv;
+  stage_levels(lv, spatial_shapes, level_start, L, S);
+  const I step = static_cast<I>(gridDim.x) * kThreads * U;
+  for (I p0 = static_cast<I>(blockIdx.x) * kThreads * U + threadIdx.x; p0 < points; p0 += step) {
+    float2 xy[U];
+    float a[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const I p = p0 + static_cast<I>(u) * kThreads;
+      if (p < points) {
+        xy[u] = __ldcs(reinterpret_cast<const float2*>(sampling_locations) + p);
+        a[u] = __ldcs(attention_weights + p);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const I p = p0 + static_cast<I>(u) * kThreads;
+      if (p >= points) continue;
+      const int l = static_cast<int>((p / static_cast<I>(K)) % static_cast<I>(L));
+      const int H = lv.H[l], W = lv.W[l];
+      const Cell c = locate(xy[u].x, xy[u].y, H, W);
+      if (point_cell(c, W) >= 0) continue;
+      grad_attn[p] = 0.0f * (c.fx + c.fy);
+      reinterpret_cast<float2*>(grad_loc)[p] =
+          make_float2(a[u] * static_cast<float>(W) * (0.0f * c.fy),
+                      a[u] * static_cast<float>(H) * (0.0f * c.fx));
+    }
+  }
+}
+
+template <typename I>
+__global__ void __launch_bounds__(kThreads)
+nonfinite_output_kernel(const int64_t* __restrict__ spatial_shapes,
+                        const int64_t* __restrict__ level_start,
+                        const float* __restrict__ sampling_locations,
+                        const float* __restrict__ grad_output, float* __restrict__ grad_loc,
+                        float* __restrict__ grad_attn, long long S, int D, int L, int K, I n4) {
+  constexpr int U = kNoCornerUnroll;
+  __shared__ Levels lv;
+  stage_levels(lv, spatial_shapes, level_start, L, S);
+  // 16-byte loads: D % 4 == 0 and grad_output is 16-byte aligned.
+  const float4* go = reinterpret_cast<const float4*>(grad_output);
+  const I step = static_cast<I>(gridDim.x) * kThreads * U;
+  for (I i0 = static_cast<I>(blockIdx.x) * kThreads * U + threadIdx.x; i0 < n4; i0 += step) {
+    float4 v[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const I i = i0 + static_cast<I>(u) * kThreads;
+      if (i < n4) v[u] = __ldcs(go + i);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const I i = i0 + static_cast<I>(u) * kThreads;
+      if (i >= n4) continue;
+      const float t = (0.0f * v[u].x + 0.0f * v[u].y) + (0.0f * v[u].z + 0.0f * v[u].w);
+      if (t == t) continue;
+      // This group's grad_output holds an Inf or NaN: its points with no corner
+      // in the map get NaN (other threads of the group may write the same NaNs).
+      const I g = i / static_cast<I>(D / 4);
+      const int LK = L * K;
+      const float nan = __int_as_float(0x7fffffff);
+      for (int j = 0; j < LK; ++j) {
+        const I p = g * static_cast<I>(LK) + static_cast<I>(j);
+        const int l = j / K;
+        const float2 xy = __ldg(reinterpret_cast<const float2*>(sampling_locations) + p);
+        const Cell c = locate(xy.x, xy.y, lv.H[l], lv.W[l]);
+        if (point_cell(c, lv.W[l]) >= 0) continue;
+        grad_attn[p] = nan;
+        reinterpret_cast<float2*>(grad_loc)[p] = make_float2(nan, nan);
+      }
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kThreads)
 hist_kernel(const int64_t* __restrict__ spatial_shapes, const int64_t* __restrict__ level_start,
             const float* __restrict__ sampling_locations,
-            const float* __restrict__ attention_weights,
-            const float* __restrict__ grad_output, float* __restrict__ grad_loc,
-            float* __restrict__ grad_attn, int* __restrict__ counts, int* __restrict__ slots,
-            long long S, int M, int D, long long Lq, int L, int K, long long cells_per_bm,
-            int chunks, long long keys) {
+            int* __restrict__ counts, int* __restrict__ slots, long long S, int M, long long Lq,
+            int L, int K, long long cells_per_bm, int chunks, long long keys) {
   extern __shared__ int hist[];
   __shared__ Levels lv;
   __shared__ CellLevels cl;
@@ -195,19 +285,6 @@ hist_kernel(const int64_t* __restrict__ spatial_shapes, const int64_t* __restric
         const int cell = ncells > 0 ? point_cell(c, W) : -1;
         if (cell >= lo && cell < lo + span) {
           __stcs(slots + p, atomicAdd(hist + (cell - lo), 1));
-        } else if (cell < 0 && lo == 0) {
-          // No corner in the map: every corner sum is sum_d gO[d] * 0, which is 0,
-          // or NaN when the group's grad_output holds an Inf or NaN.  The products
-          // with the weights keep the NaN of a non-finite location, as the
-          // oracle does.
-          const float* g = grad_output + ((sg.b * Lq + q) * M + sg.m) * static_cast<long long>(D);
-          float z = 0.0f;
-          for (int d = 0; d < D; ++d) z += 0.0f * __ldg(g + d);
-          const float a = __ldg(attention_weights + p);
-          grad_attn[p] = 0.0f * (c.fx + c.fy) + z;
-          reinterpret_cast<float2*>(grad_loc)[p] =
-              make_float2(a * static_cast<float>(W) * (0.0f * c.fy + z),
-                          a * static_cast<float>(H) * (0.0f * c.fx + z));
         }
       }
     }
@@ -804,11 +881,45 @@ cudaError_t launch_backward_sorted(const BackwardArgs& a, void* workspace,
   const unsigned blocks = static_cast<unsigned>(w.segments * w.chunks);
   const int chunks = static_cast<int>(w.chunks);
   hist_kernel<<<blocks, kThreads, cell_smem, stream>>>(
-      a.spatial_shapes, a.level_start_index, a.sampling_locations, a.attention_weights,
-      static_cast<const float*>(a.grad_output), a.grad_sampling_locations,
-      a.grad_attention_weights, counts, slots, a.S, a.M, a.D, a.Lq, a.L, a.K, w.cells_per_bm,
-      chunks, w.keys);
+      a.spatial_shapes, a.level_start_index, a.sampling_locations, counts, slots, a.S, a.M,
+      a.Lq, a.L, a.K, w.cells_per_bm, chunks, w.keys);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  {
+    // The points with no corner in the map (see no_corner_kernel); the second
+    // launch runs after the first, so its NaNs win.
+    const long long points = a.groups * a.L * a.K;
+    const long long n4 = a.groups * (a.D / 4);
+    const long long per_block = static_cast<long long>(kThreads) * kNoCornerUnroll;
+    long long b1 = (points + per_block - 1) / per_block, b2 = (n4 + per_block - 1) / per_block;
+    if (b1 > 148 * 16) b1 = 148 * 16;
+    if (b2 > 148 * 16) b2 = 148 * 16;
+    const bool narrow = points < (1ll << 31) - per_block * 148 * 16 &&
+                        n4 < (1ll << 31) - per_block * 148 * 16;
+    const float* go = static_cast<const float*>(a.grad_output);
+    if (narrow) {
+      no_corner_kernel<unsigned><<<static_cast<unsigned>(b1), kThreads, 0, stream>>>(
+          a.spatial_shapes, a.level_start_index, a.sampling_locations, a.attention_weights,
+          a.grad_sampling_locations, a.grad_attention_weights, a.S, a.L, a.K,
+          static_cast<unsigned>(points));
+      if ((err = cudaGetLastError()) != cudaSuccess) return err;
+      nonfinite_output_kernel<unsigned><<<static_cast<unsigned>(b2), kThreads, 0, stream>>>(
+          a.spatial_shapes, a.level_start_index, a.sampling_locations, go,
+          a.grad_sampling_locations, a.grad_attention_weights, a.S, a.D, a.L, a.K,
+          static_cast<unsigned>(n4));
+    } else {
+      no_corner_kernel<unsigned long long><<<static_cast<unsigned>(b1), kThreads, 0, stream>>>(
+          a.spatial_shapes, a.level_start_index, a.sampling_locations, a.attention_weights,
+          a.grad_sampling_locations, a.grad_attention_weights, a.S, a.L, a.K,
+          static_cast<unsigned long long>(points));
+      if ((err = cudaGetLastError()) != cudaSuccess) return err;
+      nonfinite_output_kernel<unsigned long long><<<static_cast<unsigned>(b2), kThreads, 0,
+                                                    stream>>>(
+          a.spatial_shapes, a.level_start_index, a.sampling_locations, go,
+          a.grad_sampling_locations, a.grad_attention_weights, a.S, a.D, a.L, a.K,
+          static_cast<unsigned long long>(n4));
+    }
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  }
   // Key-major positions from the chunk-major counts: per-key totals, their
   // exclusive scan, then each (key, chunk) run's offset.
   column_totals_kernel<<<grid_for(w.keys + 1, kThreads), kThreads, 0, stream>>>(

@@ -177,3 +177,44 @@ def test_fused_autograd():
     G.assert_backward_f32(o.grad.cpu().numpy().astype(np.float64), roff, "autograd grad_offsets")
     G.assert_backward_f32(z.grad.cpu().numpy().astype(np.float64), rz, "autograd grad_logits")
     G.assert_backward_f32(r.grad.cpu().numpy().astype(np.float64), rref, "autograd grad_reference")
+
+
+def test_offset_init_grid():
+    """The pages' initial sampling pattern: point k of head m at (k + 1) pixels
+    along the head's compass direction from pixel-centre reference points, on
+    maps whose sides are powers of two.  On a token's own level every sample
+    lands exactly on a pixel centre, so three of its four corner weights are
+    exactly zero, and neighbouring points share corners where one side's weight
+    is zero (which the backward's corner merge must leave unmerged).  The fused
+    op, and the core on the same float32 locations and weights, against the
+    oracle."""
+    import dataclasses
+    from oracle_pins import load_offset_init_directions
+
+    shapes = ((16, 32), (8, 16), (4, 8), (2, 4))
+    cfg = W.Config("init_grid", 1, 8, 32, 4, shapes, "encoder", "f32", True)
+    fz = W.make_fused_inputs(cfg, seed=3)
+    B, Lq, M, L, K = 1, cfg.queries, 8, 4, 4
+    dirs = load_offset_init_directions().astype(np.float32)         # [8, (dx, dy)]
+    off = np.empty((B, Lq, M, L, K, 2), dtype=np.float32)
+    for k in range(K):
+        off[:, :, :, :, k, :] = (k + 1) * dirs[None, None, :, None, :]
+    fz = dataclasses.replace(fz, sampling_offsets=off)
+    d = fused_device(fz)
+    G.assert_forward_f32(gpu_fused_forward(d), oracle_fused_forward(fz), "init grid fused forward")
+    check_fused_backward(fz, d, "init grid fused")
+
+    # The core on the locations and weights the pages form (float32, their order).
+    wh = fz.spatial_shapes[:, ::-1].astype(np.float32)              # [L, (W, H)]
+    loc = (fz.reference_points[:, :, None, :, None, :] + off / wh[None, None, None, :, None, :])
+    z = fz.attention_logits.astype(np.float64)
+    a = np.exp(z - z.max(-1, keepdims=True))
+    a = (a / a.sum(-1, keepdims=True)).astype(np.float32).reshape(B, Lq, M, L, K)
+    inp = W.Inputs(cfg, fz.value, None, fz.spatial_shapes, fz.level_start_index,
+                   np.ascontiguousarray(loc.astype(np.float32)), np.ascontiguousarray(a),
+                   fz.grad_output)
+    x = loc[..., 0].astype(np.float64) * wh[None, None, None, :, None, 0] - 0.5
+    assert np.mean(x == np.floor(x)) > 0.2, "too few samples on pixel centres"
+    cd = G.device_inputs(inp)
+    G.assert_forward_f32(G.gpu_forward(cd), G.oracle_forward(inp), "init grid forward")
+    G.check_backward_paths(cd, inp, "init grid")
