@@ -236,14 +236,19 @@ backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial
       if (!FIXED) asm volatile("griddepcontrol.wait;" ::: "memory");
       for (int j0 = 0; j0 < pc; j0 += LANES) {
         const int nb = min(LANES, pc - j0);
-        float keep[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-        for (int jj = 0; jj < nb; ++jj) {
-          const int j = j0 + jj;
+        // Point j's three sums over this lane's channels, with its fx, fy
+        // applied before the reduction over the lanes (linear, so the order of
+        // the two does not matter in real arithmetic):
+        //   t0 = P + fx Ex + fy Ey + fx fy Exy (grad_attn),
+        //   t1 = Ex + fy Exy,  t2 = Ey + fx Exy   (grad_loc / (A W, A H)).
+        // The gathers and the grad_value scatters happen here.
+        auto point_part = [&](int j, float (&t)[3]) {
+          t[0] = t[1] = t[2] = 0.0f;
           const int slot = j * G + (gi ^ (j & 7));
           const int4 o = s_off[slot];
-          float dot[4] = {0.0f, 0.0f, 0.0f, 0.0f};
           if (lane_on) {
             const float4 w = s_w[slot];
+            const float2 f = *reinterpret_cast<const float2*>(&s_g[slot]);  // fx, fy
             const int os[4] = {o.x, o.y, o.z, o.w};
             const float ws[4] = {w.x, w.y, w.z, w.w};
             float q[4][E];
@@ -253,35 +258,65 @@ backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial
               for (int e = 0; e < E; ++e) q[i][e] = 0.0f;
               if (os[i] >= 0) V::load(vbase + os[i], q[i]);
             }
+            float dot[4];
             corner_sums4(q, go, dot);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               if (kMerge ? __float_as_uint(ws[i]) != kNoScatterBits : os[i] >= 0)
                 scatter(os[i], ws[i], go);
             }
+            t[1] = fmaf(f.y, dot[3], dot[1]);
+            t[2] = fmaf(f.x, dot[3], dot[2]);
+            t[0] = fmaf(f.x, t[1], fmaf(f.y, dot[2], dot[0]));
           }
+        };
+        float keep[3] = {0.0f, 0.0f, 0.0f};
+        int jl = lane;  // this lane's point of the batch
+        if constexpr (LANES == 1) {
+          if (nb > 0) point_part(j0, keep);
+        } else {
+          // Two points per reduction: the first exchange sends the lower half of
+          // the sub-warp point B's partials and the upper half point A's, so the
+          // halves end with A's and B's totals after log2(LANES) rounds of three
+          // shuffles.  Lane u keeps the totals of point 2u and lane HALF + u
+          // those of point 2u + 1.
+          constexpr int HALF = LANES / 2;
+          const bool upper = (lane & HALF) != 0;
+          for (int jj = 0; jj < nb; jj += 2) {
+            float ta[3], tb[3];
+            point_part(j0 + jj, ta);
+            if (jj + 1 < nb) {
+              point_part(j0 + jj + 1, tb);
+            } else {
+              tb[0] = tb[1] = tb[2] = 0.0f;
+            }
+            float v[3];
 #pragma unroll
-          for (int sh = LANES / 2; sh > 0; sh >>= 1) {
+            for (int i = 0; i < 3; ++i) {
+              const float send = upper ? ta[i] : tb[i];
+              const float mine = upper ? tb[i] : ta[i];
+              v[i] = mine + __shfl_xor_sync(kFullMask, send, HALF, LANES);
+            }
 #pragma unroll
-            for (int i = 0; i < 4; ++i) dot[i] += __shfl_xor_sync(kFullMask, dot[i], sh, LANES);
+            for (int sh = HALF / 2; sh > 0; sh >>= 1) {
+#pragma unroll
+              for (int i = 0; i < 3; ++i) v[i] += __shfl_xor_sync(kFullMask, v[i], sh, LANES);
+            }
+            if ((lane & (HALF - 1)) == (jj >> 1)) {
+#pragma unroll
+              for (int i = 0; i < 3; ++i) keep[i] = v[i];
+            }
           }
-          if (lane == jj) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) keep[i] = dot[i];
-          }
+          jl = upper ? 2 * (lane - HALF) + 1 : 2 * lane;
         }
-        const int jr_out = (q0 + j0 + lane) * SPLIT + subset_first;
-        if (active && lane < nb && jr_out < LK) {
-          const int j = j0 + lane;
+        const int jr_out = (q0 + j0 + jl) * SPLIT + subset_first;
+        if (active && jl < nb && jr_out < LK) {
+          const int j = j0 + jl;
           const float4 gg = s_g[j * G + (gi ^ (j & 7))];
-          const float fx = gg.x, fy = gg.y;
-          const float s_attn = fmaf(fx, fmaf(fy, keep[3], keep[1]), fmaf(fy, keep[2], keep[0]));
-          const float s_x = fmaf(fy, keep[3], keep[1]);
-          const float s_y = fmaf(fx, keep[3], keep[2]);
           const long long pidx = grp.bqm * LK + jr_out;
-          grad_attention_weights[pidx] = s_attn;
+          grad_attention_weights[pidx] = keep[0];
           reinterpret_cast<float2*>(grad_sampling_locations)[pidx] =
-              make_float2(gg.z * s_x, gg.w * s_y);
+              make_float2(gg.z * keep[1], gg.w * keep[2]);
         }
       }
       // The next unit's setup overwrites the table.
