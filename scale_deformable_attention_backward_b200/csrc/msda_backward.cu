@@ -108,8 +108,10 @@ backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial
   }
   const int dq = D / 4;
   // Corners shared by two points of one level of one group are merged before the
-  // scatter (merge_shared_corners); the deterministic path scatters every corner.
-  constexpr bool kMerge = !FIXED && SPLIT == 1 && PC % 4 == 0;
+  // scatter (merge_shared_corners).  The merge depends only on the inputs (the
+  // weights are summed in lane order), so the deterministic path keeps its
+  // bit-identical results with it.
+  constexpr bool kMerge = SPLIT == 1 && PC % 4 == 0;
 
   const int lane = threadIdx.x % LANES;
   const int gi = threadIdx.x / LANES;
