@@ -238,12 +238,8 @@ backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial
       if (!FIXED) asm volatile("griddepcontrol.wait;" ::: "memory");
       for (int j0 = 0; j0 < pc; j0 += LANES) {
         const int nb = min(LANES, pc - j0);
-        // Point j's three sums over this lane's channels, with its fx, fy
-        // applied before the reduction over the lanes (linear, so the order of
-        // the two does not matter in real arithmetic):
-        //   t0 = P + fx Ex + fy Ey + fx fy Exy (grad_attn),
-        //   t1 = Ex + fy Exy,  t2 = Ey + fx Exy   (grad_loc / (A W, A H)).
-        // The gathers and the grad_value scatters happen here.
+        // Point j's three sums over this lane's channels (point_sums3); the
+        // gathers and the grad_value scatters happen here.
         auto point_part = [&](int j, float (&t)[3]) {
           t[0] = t[1] = t[2] = 0.0f;
           const int slot = j * G + (gi ^ (j & 7));
@@ -267,50 +263,29 @@ backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial
               if (kMerge ? __float_as_uint(ws[i]) != kNoScatterBits : os[i] >= 0)
                 scatter(os[i], ws[i], go);
             }
-            t[1] = fmaf(f.y, dot[3], dot[1]);
-            t[2] = fmaf(f.x, dot[3], dot[2]);
-            t[0] = fmaf(f.x, t[1], fmaf(f.y, dot[2], dot[0]));
+            point_sums3(dot, f.x, f.y, t);
           }
         };
         float keep[3] = {0.0f, 0.0f, 0.0f};
-        int jl = lane;  // this lane's point of the batch
         if constexpr (LANES == 1) {
           if (nb > 0) point_part(j0, keep);
         } else {
-          // Two points per reduction: the first exchange sends the lower half of
-          // the sub-warp point B's partials and the upper half point A's, so the
-          // halves end with A's and B's totals after log2(LANES) rounds of three
-          // shuffles.  Lane u keeps the totals of point 2u and lane HALF + u
-          // those of point 2u + 1.
-          constexpr int HALF = LANES / 2;
-          const bool upper = (lane & HALF) != 0;
           for (int jj = 0; jj < nb; jj += 2) {
-            float ta[3], tb[3];
+            float ta[3], tb[3], v[3];
             point_part(j0 + jj, ta);
             if (jj + 1 < nb) {
               point_part(j0 + jj + 1, tb);
             } else {
               tb[0] = tb[1] = tb[2] = 0.0f;
             }
-            float v[3];
-#pragma unroll
-            for (int i = 0; i < 3; ++i) {
-              const float send = upper ? ta[i] : tb[i];
-              const float mine = upper ? tb[i] : ta[i];
-              v[i] = mine + __shfl_xor_sync(kFullMask, send, HALF, LANES);
-            }
-#pragma unroll
-            for (int sh = HALF / 2; sh > 0; sh >>= 1) {
-#pragma unroll
-              for (int i = 0; i < 3; ++i) v[i] += __shfl_xor_sync(kFullMask, v[i], sh, LANES);
-            }
-            if ((lane & (HALF - 1)) == (jj >> 1)) {
+            reduce_pair3<LANES>(ta, tb, lane, v);
+            if ((lane & (LANES / 2 - 1)) == (jj >> 1)) {
 #pragma unroll
               for (int i = 0; i < 3; ++i) keep[i] = v[i];
             }
           }
-          jl = upper ? 2 * (lane - HALF) + 1 : 2 * lane;
         }
+        const int jl = pair_lane_point<LANES>(lane);  // this lane's point of the batch
         const int jr_out = (q0 + j0 + jl) * SPLIT + subset_first;
         if (active && jl < nb && jr_out < LK) {
           const int j = j0 + jl;

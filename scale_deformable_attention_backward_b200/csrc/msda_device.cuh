@@ -237,6 +237,56 @@ __device__ __forceinline__ void corner_sums4(const float (&q)[4][4], const float
   for (int k = 0; k < 4; ++k) dot[k] = d2[k].x + d2[k].y;
 }
 
+// The lane reduction of the backward kernels, two points at a time.  Each lane
+// of a sub-warp of LANES lanes holds three partial sums of points A and B (ta,
+// tb) over its channels.  The first exchange sends the lower half of the
+// sub-warp B's partials and the upper half A's, so after log2(LANES) rounds of
+// three shuffles lanes [0, LANES/2) hold A's totals and lanes [LANES/2, LANES)
+// B's (4.5 shuffles per point for LANES = 8, against 12 for a butterfly of four
+// sums per point).
+template <int LANES>
+__device__ __forceinline__ void reduce_pair3(const float (&ta)[3], const float (&tb)[3], int lane,
+                                             float (&v)[3]) {
+  constexpr int HALF = LANES / 2;
+  const bool upper = (lane & HALF) != 0;
+#pragma unroll
+  for (int i = 0; i < 3; ++i) {
+    const float send = upper ? ta[i] : tb[i];
+    const float mine = upper ? tb[i] : ta[i];
+    v[i] = mine + __shfl_xor_sync(kFullMask, send, HALF, LANES);
+  }
+#pragma unroll
+  for (int sh = HALF / 2; sh > 0; sh >>= 1) {
+#pragma unroll
+    for (int i = 0; i < 3; ++i) v[i] += __shfl_xor_sync(kFullMask, v[i], sh, LANES);
+  }
+}
+
+// The point of a batch of LANES points whose totals lane `lane` keeps after
+// reduce_pair3 over the pairs (0, 1), (2, 3), ...: lane u keeps point 2u, lane
+// LANES/2 + u point 2u + 1 (lane 0 keeps point 0 when LANES = 1).
+template <int LANES>
+__device__ __forceinline__ int pair_lane_point(int lane) {
+  if constexpr (LANES == 1) {
+    return 0;
+  } else {
+    constexpr int HALF = LANES / 2;
+    return (lane & HALF) ? 2 * (lane - HALF) + 1 : 2 * lane;
+  }
+}
+
+// A point's three sums over a lane's channels from its four corner sums
+// (corner_sums4), with its fx, fy applied before the lane reduction (linear, so
+// the order of the two does not matter in real arithmetic):
+//   t0 = P + fx Ex + fy Ey + fx fy Exy   (grad_attn),
+//   t1 = Ex + fy Exy,  t2 = Ey + fx Exy    (grad_loc / (A W, A H)).
+__device__ __forceinline__ void point_sums3(const float (&dot)[4], float fx, float fy,
+                                            float (&t)[3]) {
+  t[1] = fmaf(fy, dot[3], dot[1]);
+  t[2] = fmaf(fx, dot[3], dot[2]);
+  t[0] = fmaf(fx, t[1], fmaf(fy, dot[2], dot[0]));
+}
+
 // grad_value[p .. p + 3] += w * g[0 .. 3], one 16-byte vector reduction.
 __device__ __forceinline__ void scatter_row4(float* p, float w, const float (&g)[4]) {
   const float2 ww = make_float2(w, w);

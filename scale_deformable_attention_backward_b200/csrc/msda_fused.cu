@@ -148,7 +148,7 @@ fused_forward_kernel(const T* __restrict__ value, const int64_t* __restrict__ sp
 // (max and 1 / sum) into shared memory, so that any thread can form any of the
 // tile's weights.  grad_logits holds dA until the group's sum_j A_j dA_j is
 // known, then d z.  Lane i of a group combines (and later revisits) the points
-// p with p % LANES == i.
+// p with p % LANES == pair_lane_point(i).
 // T: dtype of value and grad_output (float32, or bfloat16 read 8 bytes per
 // lane); arithmetic and every gradient are float32 for both.
 //
@@ -258,14 +258,15 @@ fused_backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ s
       // Phase 2: gathers, scatters, corner dot products, and the chain rule.
       for (int j0 = 0; j0 < pc; j0 += LANES) {
         const int nb = min(LANES, pc - j0);
-        float keep[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-        for (int jj = 0; jj < nb; ++jj) {
-          const int j = j0 + jj;
+        // Point j's three sums over this lane's channels (point_sums3); the
+        // gathers and the grad_value scatters happen here.
+        auto point_part = [&](int j, float (&t)[3]) {
+          t[0] = t[1] = t[2] = 0.0f;
           const int slot = j * G + (gi ^ (j & 7));
           const int4 o = s_off[slot];
-          float dot[4] = {0.0f, 0.0f, 0.0f, 0.0f};
           if (lane_on) {
             const float4 w = s_w[slot];
+            const float2 f = *reinterpret_cast<const float2*>(&s_g[slot]);  // fx, fy
             const int os[4] = {o.x, o.y, o.z, o.w};
             const float ws[4] = {w.x, w.y, w.z, w.w};
             float q[4][E];
@@ -275,31 +276,41 @@ fused_backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ s
               for (int e = 0; e < E; ++e) q[i][e] = 0.0f;
               if (os[i] >= 0) V::load(vbase + os[i], q[i]);
             }
+            float dot[4];
             corner_sums4(q, go, dot);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               if (__float_as_uint(ws[i]) != kNoScatterBits) scatter_row4(gvbase + os[i], ws[i], go);
             }
+            point_sums3(dot, f.x, f.y, t);
           }
+        };
+        float keep[3] = {0.0f, 0.0f, 0.0f};
+        if constexpr (LANES == 1) {
+          if (nb > 0) point_part(j0, keep);
+        } else {
+          for (int jj = 0; jj < nb; jj += 2) {
+            float ta[3], tb[3], v[3];
+            point_part(j0 + jj, ta);
+            if (jj + 1 < nb) {
+              point_part(j0 + jj + 1, tb);
+            } else {
+              tb[0] = tb[1] = tb[2] = 0.0f;
+            }
+            reduce_pair3<LANES>(ta, tb, lane, v);
+            if ((lane & (LANES / 2 - 1)) == (jj >> 1)) {
 #pragma unroll
-          for (int sh = LANES / 2; sh > 0; sh >>= 1) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) dot[i] += __shfl_xor_sync(kFullMask, dot[i], sh, LANES);
-          }
-          if (lane == jj) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) keep[i] = dot[i];
+              for (int i = 0; i < 3; ++i) keep[i] = v[i];
+            }
           }
         }
-        if (active && lane < nb) {
-          const int pj = q0 + j0 + lane;
+        const int jl = pair_lane_point<LANES>(lane);  // this lane's point of the batch
+        if (active && jl < nb) {
+          const int pj = q0 + j0 + jl;
           const long long p = grp.bqm * LK + pj;
           const int lj = pj / K;
-          const float4 gg = s_g[(j0 + lane) * G + (gi ^ ((j0 + lane) & 7))];
-          const float fx = gg.x, fy = gg.y, a = gg.z;
-          const float dA = fmaf(fx, fmaf(fy, keep[3], keep[1]), fmaf(fy, keep[2], keep[0]));
-          const float s_x = fmaf(fy, keep[3], keep[1]);
-          const float s_y = fmaf(fx, keep[3], keep[2]);
+          const float a = s_g[(j0 + jl) * G + (gi ^ ((j0 + jl) & 7))].z;
+          const float dA = keep[0], s_x = keep[1], s_y = keep[2];
           sum_adA = fmaf(a, dA, sum_adA);
           grad_logits[p] = dA;  // dA for now
           const float kx = a * s_x, ky = a * s_y;  // grad_loc / (W, H)
@@ -331,7 +342,7 @@ fused_backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ s
 #pragma unroll
     for (int o = LANES / 2; o > 0; o >>= 1) sum_adA += __shfl_xor_sync(kFullMask, sum_adA, o, LANES);
     if (active) {
-      for (int pj = lane; pj < LK; pj += LANES) {
+      for (int pj = pair_lane_point<LANES>(lane); pj < LK; pj += LANES) {
         const long long p = grp.bqm * LK + pj;
         const float aj = expf(__ldg(zg + pj) - nz.x) * nz.y;
         grad_logits[p] = aj * (grad_logits[p] - sum_adA);
