@@ -816,6 +816,29 @@ def run_b200(args, world, rank, local):
             and torch.equal(last["ga"], ref_ga.cpu())):
         raise RuntimeError("end-to-end pipeline results differ from a plain call's")
     del ref_out, ref_gl, ref_ga
+    # The link's floor for these bytes: the same uploads and downloads alone, on
+    # two streams at once (no kernels).
+    def link_copies():
+        with torch.cuda.stream(s_up):
+            for k, t in pin.items():
+                dev_in[0][k].copy_(t, non_blocking=True)
+        with torch.cuda.stream(s_down):
+            for k in host_out[0]:
+                host_out[0][k].copy_(dev_out[0][k], non_blocking=True)
+
+    link_copies()
+    torch.cuda.synchronize()
+    le0, le1, le2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+    link_reps = 5
+    le0.record(s_up)
+    s_down.wait_event(le0)
+    for _ in range(link_reps):
+        link_copies()
+    le1.record(s_up)
+    le2.record(s_down)
+    torch.cuda.synchronize()
+    link_ms = max(le0.elapsed_time(le1), le0.elapsed_time(le2)) / link_reps
+    link_ms = max_over_ranks(link_ms, world, device)
 
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": "queries/s", "n_gpus": world,
@@ -836,6 +859,10 @@ def run_b200(args, world, rank, local):
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h),
                 "pipeline": "upload / compute / download on three streams, two buffer sets",
+                "link_floor_ms": round(link_ms, 3),
+                "frac_of_link_floor": round(link_ms / e2e_ms, 4),
+                "link_note": "link_floor_ms: the same uploads and downloads alone, concurrently "
+                             "on two streams, no kernels (host link, both directions at once)",
                 "api": "the Python binding of the C ABI (msda_forward, msda_backward) with torch "
                        "tensors as memory; host buffers are pinned torch CPU tensors"},
         "gpu_launches": (1 + BACKWARD_LAUNCHES) * args.steps,
