@@ -434,6 +434,21 @@ def run_b200(args, world, rank, local):
     ms_per_step = total_ms_max / args.steps
     queries = B * Lq
     value = replica_throughput(world, queries, args.steps, total_ms_max)
+    step_median_ms = max_over_ranks(statistics.median(f + b for f, b in zip(fwd_ms, bwd_ms)),
+                                    world, device)
+    # Warm: steps back to back with no L2 flush between them (context only; the
+    # flushed figure above is the metric).
+    warm_n = max(3, min(args.steps, 50))
+    ws0, ws1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    step()
+    step_bwd()
+    ws0.record(stream)
+    for _ in range(warm_n):
+        step()
+        step_bwd()
+    ws1.record(stream)
+    torch.cuda.synchronize()
+    step_warm_ms = max_over_ranks(ws0.elapsed_time(ws1) / warm_n, world, device)
 
     peak, peak_kind = measured_peak()
     algo = algorithmic_bytes(cfg, inp)
@@ -723,13 +738,29 @@ def run_b200(args, world, rank, local):
         fstep()
         fe1[i].record(stream)
     torch.cuda.synchronize()
-    fms = statistics.mean(a.elapsed_time(b) for a, b in zip(fe0, fe1))
-    fms = max_over_ranks(fms, world, device)
+    fms_all = [a.elapsed_time(b) for a, b in zip(fe0, fe1)]
+    fms = max_over_ranks(statistics.mean(fms_all), world, device)
+    fms_median = max_over_ranks(statistics.median(fms_all), world, device)
+    # Warm: the same launches back to back with no flush between them, so the
+    # inputs are partly L2-resident (the cold figures above are the contract's).
+    warm_n = max(3, min(args.steps, 50))
+    we0, we1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    fstep()
+    we0.record(stream)
+    for _ in range(warm_n):
+        fstep()
+    we1.record(stream)
+    torch.cuda.synchronize()
+    fms_warm = max_over_ranks(we0.elapsed_time(we1) / warm_n, world, device)
     fbytes = algorithmic_bytes(fcfg, finp)["forward"]
     fach = fbytes / (fms * 1e-3) / 1e9
     forward_encoder = {
         "workload": fcfg.description, "queries": fcfg.B * fcfg.queries,
         "ms": round(fms, 4), "queries_per_s": round(fcfg.B * fcfg.queries / (fms * 1e-3), 1),
+        "median_ms": round(fms_median, 4),
+        "warm_ms": round(fms_warm, 4),
+        "warm_note": "back-to-back launches with no L2 flush between them (inputs partly "
+                     "L2-resident); ms is the L2-flushed figure",
         "roofline": {"bound": "hbm", "achieved": round(fach, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(fach / peak, 4),
                      "traffic": recorded_traffic(f"{FORWARD_WORKLOAD}.forward"),
@@ -850,6 +881,9 @@ def run_b200(args, world, rank, local):
                    "l2": "flushed before every step by a 256 MiB write (outside the timed events)",
                    "timing": "CUDA events per step on the launching stream, max over ranks"},
         "roofline": roofline,
+        "step_timing": {"mean_ms": round(ms_per_step, 4), "median_ms": round(step_median_ms, 4),
+                        "warm_ms": round(step_warm_ms, 4),
+                        "warm_note": "steps back to back with no L2 flush between them"},
         "forward_encoder": forward_encoder,
         "fused": fused,
         "bf16_train": bf16_train,
