@@ -114,12 +114,15 @@ msda_status msda_forward(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq,
  * inputs (the softmax before them is not differentiated).
  *
  *   value, spatial_shapes, level_start_index, sampling_locations,
- *   attention_weights   as for msda_forward; D <= 128 (one sub-warp of at
- *                       most 32 lanes holds a head's D channels, 4 per lane,
- *                       and reduces each point's corner dot products over
- *                       them; larger D returns MSDA_ERR_UNSUPPORTED -- the
- *                       forward splits larger heads into channel chunks, which
- *                       would make those reductions cross sub-warps).
+ *   attention_weights   as for msda_forward; D <= 256.  One sub-warp of at
+ *                       most 32 lanes holds up to 128 of a head's channels,
+ *                       4 per lane, and reduces each point's corner dot
+ *                       products over them; a wider head runs as two channel
+ *                       passes in stream order, the second adding its share of
+ *                       grad_sampling_locations and grad_attention_weights.
+ *                       D > 256, or D > 128 with a workspace (the cell-sorted
+ *                       path keeps a head in one sub-warp), returns
+ *                       MSDA_ERR_UNSUPPORTED.
  *                       value_dtype MSDA_F32,
  *                       or MSDA_BF16 without a workspace (value and
  *                       grad_output then only need 8-byte alignment; the
@@ -171,7 +174,8 @@ msda_status msda_backward(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq
  * msda_backward; the finite elements are then no longer guaranteed
  * bit-identical across runs.
  *
- *   arguments as msda_backward (value_dtype MSDA_F32 or MSDA_BF16, D <= 128),
+ *   arguments as msda_backward (value_dtype MSDA_F32 or MSDA_BF16), but
+ *   D <= 128 (one pass: the integer accumulators' channel layout is per pass),
  *   workspace, workspace_bytes
  *       device scratch owned by the caller, 256-byte aligned, at least
  *       msda_backward_deterministic_workspace_size() bytes (8 bytes per
@@ -289,7 +293,8 @@ msda_status msda_fused_forward(int64_t B, int64_t S, int64_t M, int64_t D, int64
  *
  *   value_dtype MSDA_F32, or MSDA_BF16 (value and grad_output bfloat16, 8-byte
  *       aligned; the arithmetic and every gradient stay float32, as in
- *       msda_backward); D <= 128 (as msda_backward)
+ *       msda_backward); D <= 128 (one sub-warp per head: the softmax Jacobian
+ *       revisits each point's dA, which a channel pass would not have complete)
  *   grad_output              [B, Lq, M * D]        value_dtype
  *   grad_value               [B, S, M, D]          overwritten (zeroed, then
  *                                                  atomics; 16-byte aligned)

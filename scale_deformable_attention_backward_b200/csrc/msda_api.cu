@@ -164,7 +164,9 @@ msda_status msda_backward(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq
   if (value_dtype != MSDA_F32 && !(value_dtype == MSDA_BF16 && workspace == nullptr))
     return MSDA_ERR_UNSUPPORTED;
   const uintptr_t in_align = value_dtype == MSDA_F32 ? 16 : 8;
-  if (D % 4 != 0 || D > 128 || M > INT32_MAX) return MSDA_ERR_UNSUPPORTED;
+  if (D % 4 != 0 || D > 256 || M > INT32_MAX) return MSDA_ERR_UNSUPPORTED;
+  // The cell-sorted path holds a head's channels in one sub-warp: D <= 128.
+  if (workspace != nullptr && D > 128) return MSDA_ERR_UNSUPPORTED;
   if (workspace != nullptr) {
     size_t need = 0;
     st = msda_backward_workspace_size(B, S, M, D, Lq, L, K, &need);
@@ -208,7 +210,8 @@ msda_status msda_backward(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq
   a.D = static_cast<int>(D);
   a.L = static_cast<int>(L);
   a.K = static_cast<int>(K);
-  a.lanes = pow2_at_least(D / 4);
+  // Lanes of one channel pass (at most 128 channels; wider heads run as passes).
+  a.lanes = pow2_at_least((D > 128 ? 128 : D) / 4);
   a.groups = work ? B * Lq * M : 0;
   a.value_elements = c.value_elems;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);

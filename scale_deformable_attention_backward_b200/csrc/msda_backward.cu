@@ -37,6 +37,8 @@ static_assert(sizeof(FixedHeader) <= kFixedHeaderBytes, "header must fit its slo
 constexpr int kBwdThreads = 256;
 
 constexpr int kBwdPoints = 512;  // points set up per unit (two per thread)
+// Channels of a head per kernel pass: one sub-warp of at most 32 lanes, 4 per lane.
+constexpr int kPassChannels = 128;
 
 // T: dtype of value and grad_output (float32, or bfloat16 read 8 bytes per lane);
 // arithmetic and grad_value are float32 for both.
@@ -87,7 +89,7 @@ backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial
                 const T* __restrict__ grad_output, float* __restrict__ grad_value,
                 float* __restrict__ grad_sampling_locations,
                 float* __restrict__ grad_attention_weights, long long S, int M, int D,
-                long long Lq, int L, int K, long long groups,
+                long long Lq, int L, int K, long long groups, int c0, int Dc,
                 unsigned long long* __restrict__ fixed_acc,
                 const FixedHeader* __restrict__ header) {
   using V = Vec4<T>;
@@ -156,8 +158,8 @@ backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial
     real_point(v_raw, 0, g_raw, subset_first);  // subset_first = this sub-warp's subset s
     const Group grp = decompose(active ? g_raw : groups - 1, 1, M, Lq);
     const int ch = lane * E;
-    const bool lane_on = active && ch < D;  // clamped tail groups touch no memory
-    const long long vofs = (grp.b * S * M + grp.m) * static_cast<long long>(D) + ch;
+    const bool lane_on = active && ch < Dc;  // clamped tail groups touch no memory
+    const long long vofs = (grp.b * S * M + grp.m) * static_cast<long long>(D) + c0 + ch;
     const T* vbase = value + vofs;
     float* gvbase = grad_value + vofs;
     unsigned long long* abase =
@@ -181,7 +183,7 @@ backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial
     for (int e = 0; e < E; ++e) go[e] = 0.0f;
     if (lane_on)
       V::load(grad_output + grp.bq * static_cast<long long>(MD) + static_cast<long long>(grp.m) * D +
-                  ch,
+                  c0 + ch,
               go);
 
     for (int q0 = 0; q0 < LKv; q0 += PC) {
@@ -291,9 +293,17 @@ backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial
           const int j = j0 + jl;
           const float4 gg = s_g[j * G + (gi ^ (j & 7))];
           const long long pidx = grp.bqm * LK + jr_out;
-          grad_attention_weights[pidx] = keep[0];
-          reinterpret_cast<float2*>(grad_sampling_locations)[pidx] =
-              make_float2(gg.z * keep[1], gg.w * keep[2]);
+          float2* gl = reinterpret_cast<float2*>(grad_sampling_locations) + pidx;
+          if (c0 == 0) {
+            grad_attention_weights[pidx] = keep[0];
+            *gl = make_float2(gg.z * keep[1], gg.w * keep[2]);
+          } else {
+            // A later channel pass adds its channels' share (this thread wrote the
+            // earlier passes' value; the passes run in stream order).
+            grad_attention_weights[pidx] += keep[0];
+            const float2 prev = *gl;
+            *gl = make_float2(prev.x + gg.z * keep[1], prev.y + gg.w * keep[2]);
+          }
         }
       }
       // The next unit's setup overwrites the table.
@@ -427,24 +437,33 @@ static cudaError_t launch_backward_t(const BackwardArgs& a, unsigned long long* 
   long long blocks = (a.groups * split + per_block - 1) / per_block;
   if (blocks > (1ll << 30)) blocks = 1ll << 30;
   auto go = [&](auto kernel) {
-    // The plain backward overlaps its start (metadata, locations, corner loads)
-    // with the zeroing of grad_value launched just before it; the deterministic
-    // one reads the scale pass's header first, so it is launched plainly.
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(blocks));
-    cfg.blockDim = dim3(kBwdThreads);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = FIXED ? 0 : 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kernel, static_cast<const T*>(a.value), a.spatial_shapes,
-                              a.level_start_index, a.sampling_locations, a.attention_weights,
-                              static_cast<const T*>(a.grad_output), a.grad_value,
-                              a.grad_sampling_locations, a.grad_attention_weights, a.S, a.M,
-                              a.D, a.Lq, a.L, a.K, a.groups, acc, header);
+    // Heads wider than kPassChannels run as channel passes in stream order: every
+    // pass scatters its channels of grad_value, and the later passes add their
+    // share of grad_attn and grad_loc to what the first wrote.  The first pass
+    // overlaps its start (metadata, locations, corner loads) with the zeroing of
+    // grad_value launched just before it; the deterministic path (one pass) reads
+    // the scale pass's header first, so it is launched plainly.
+    for (int c0 = 0; c0 < a.D; c0 += kPassChannels) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(static_cast<unsigned>(blocks));
+      cfg.blockDim = dim3(kBwdThreads);
+      cfg.dynamicSmemBytes = 0;
+      cfg.stream = stream;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[0].val.programmaticStreamSerializationAllowed = (FIXED || c0 > 0) ? 0 : 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      const int dc = min(kPassChannels, a.D - c0);
+      const cudaError_t err =
+          cudaLaunchKernelEx(&cfg, kernel, static_cast<const T*>(a.value), a.spatial_shapes,
+                             a.level_start_index, a.sampling_locations, a.attention_weights,
+                             static_cast<const T*>(a.grad_output), a.grad_value,
+                             a.grad_sampling_locations, a.grad_attention_weights, a.S, a.M,
+                             a.D, a.Lq, a.L, a.K, a.groups, c0, dc, acc, header);
+      if (err != cudaSuccess) return err;
+    }
+    return cudaSuccess;
   };
   if (split == 4) return go(backward_kernel<T, LANES, FIXED, 4>);
   if (split == 2) return go(backward_kernel<T, LANES, FIXED, 2>);

@@ -119,7 +119,8 @@ def test_backward_argument_errors(lib):
     p = [FAKE] * 9
     p[5] = FAKE + 2                                # bfloat16 grad_output
     assert _bwd(lib, dtype=1, ptrs=p) == MISAL
-    assert _bwd(lib, D=132) == UNSUP               # at most 128 channels per head
+    assert _bwd(lib, D=260) == UNSUP               # at most 256 channels per head
+    assert _bwd(lib, D=132, ws=FAKE, ws_bytes=1 << 40) == UNSUP  # cell-sorted: at most 128
     assert _bwd(lib, D=6) == UNSUP
     assert _bwd(lib, S=-3) == BAD
     p = [FAKE] * 9

@@ -65,6 +65,26 @@ def test_value_with_large_common_offset(offset):
     G.check_backward_paths(d, inp)
 
 
+@pytest.mark.parametrize("D", [132, 192, 256])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_backward_channel_passes(D, dtype):
+    """Heads wider than 128 channels: the scratch-free backward runs two channel
+    passes (the second adds its share of grad_loc and grad_attn); against the
+    oracle.  The cell-sorted path (a workspace) refuses them."""
+    if dtype == "bf16" and D % 8:
+        pytest.skip("bfloat16 needs D % 8 == 0")
+    inp = random_inputs(400 + D, B=2, M=2, D=D, K=4, shapes=SHAPES[2], Lq=41, dtype=dtype)
+    d = G.device_inputs(inp)
+    rv, rl, ra = G.oracle_backward(inp)
+    gv, gl, ga = G.gpu_backward(d, "direct")
+    G.assert_backward_f32(gv, rv, f"{dtype} D={D} grad_value")
+    G.assert_backward_f32(gl, rl, f"{dtype} D={D} grad_sampling_locations")
+    G.assert_backward_f32(ga, ra, f"{dtype} D={D} grad_attention_weights")
+    if dtype == "f32":
+        with pytest.raises(RuntimeError, match="UNSUPPORTED|unsupported"):
+            G.gpu_backward(d, "sorted")
+
+
 @pytest.mark.parametrize("D", [256, 384])
 def test_forward_channel_chunks_f32(D):
     """More than 32 lanes' worth of channels: several chunks per head."""
