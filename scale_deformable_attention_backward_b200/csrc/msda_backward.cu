@@ -57,12 +57,14 @@ constexpr int kPassChannels = 128;
 //              P  = sum_d gO V00,          Ex = sum_d gO (V10 - V00),
 //              Ey = sum_d gO (V01 - V00),  Exy = sum_d gO (V11 - V01 - V10 + V00)
 //            (differences taken per channel, so a common offset of the value
-//            field cancels exactly), then reduces them over the lanes.  Lane j
-//            keeps point j's sums; after each batch of LANES points every lane
-//            turns its point's sums into
+//            field cancels exactly), applies the point's fx, fy to them
+//            (point_sums3) and reduces the three results over the lanes, two
+//            points per exchange (reduce_pair3).  After each batch of LANES
+//            points every lane holds one point's totals
 //              grad_attn = P + fx Ex + fy Ey + fx fy Exy
-//              grad_x    = A W_l (Ex + fy Exy)
-//              grad_y    = A H_l (Ey + fx Exy)
+//              grad_x / (A W_l) = Ex + fy Exy
+//              grad_y / (A H_l) = Ey + fx Exy
+//            and writes its gradients.
 // These are the derivatives above, regrouped with hx + fx = hy + fy = 1.
 // In the float path with K = 4, phase 1 also merges the corners that two points
 // of one level share (merge_shared_corners), so such a pixel takes one
