@@ -34,7 +34,10 @@
  *    the SM count and of kernel attributes.
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *    Work is enqueued asynchronously on it; results are ready once the stream
- *    has been synchronised.
+ *    has been synchronised.  The compute entry points neither allocate nor
+ *    synchronise, so they can be captured into a CUDA graph once a first call on
+ *    the device has loaded their code (with the environment variable
+ *    MSDA_VALIDATE unset: it reads the metadata back to the host).
  *  - Argument errors are detected on the host, before anything is enqueued, and
  *    returned synchronously; nothing is written in that case.  A failed launch
  *    returns MSDA_ERR_CUDA.  A fault during kernel execution surfaces at the
