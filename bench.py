@@ -39,6 +39,7 @@ import json
 import os
 import statistics
 import subprocess
+import threading
 import sys
 import time
 
@@ -160,8 +161,14 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "25"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            # Wait (up to 10 s) for the first sample, taken before the timed
+            # region and not counted, so that the sampler is running when the
+            # region starts.
+            first = threading.Thread(target=self.proc.stdout.readline, daemon=True)
+            first.start()
+            first.join(timeout=10.0)
         except OSError:
             self.proc = None
         return self
