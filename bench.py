@@ -931,7 +931,14 @@ def run_case(args, local):
 
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
-    name = FORWARD_WORKLOAD if args.case == "forward_encoder" else STEP_WORKLOAD
+    if args.case == "forward_encoder":
+        name = FORWARD_WORKLOAD
+    elif args.case == "decoder_forward":
+        name = "decoder_fp32"
+    elif args.case == "decoder_backward":
+        name = "decoder_box_train_fp32"
+    else:
+        name = STEP_WORKLOAD
     cfg = W.CONFIGS[name]
     if args.case.startswith("fused"):
         fz = W.make_fused_inputs(cfg, seed=0)
@@ -939,10 +946,12 @@ def run_case(args, local):
              ("value", "spatial_shapes", "level_start_index", "reference_points",
               "sampling_offsets", "attention_logits", "grad_output")}
     else:
-        inp = W.make_inputs(cfg, seed=0, with_grad=args.case.startswith("backward"))
+        inp = W.make_inputs(cfg, seed=0,
+                            with_grad=args.case.startswith("backward") or
+                            args.case == "decoder_backward")
         d = _device_inputs(inp, device)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
-    if args.case == "projection":
+    if args.case.startswith("projection"):
         # output_proj on the op's output, with the weights the full bench uses.
         px = binding.forward(d["value"], d["spatial_shapes"], d["level_start_index"],
                              d["sampling_locations"], d["attention_weights"])
@@ -959,12 +968,14 @@ def run_case(args, local):
     def launch():
         if args.case == "projection":
             binding.output_projection(px, pw, pb, out=py)
+        elif args.case == "projection_f32":
+            binding.output_projection(px, pw, pb, out=py, precise=True)
         elif args.case == "fused_forward":
             binding.fused_forward(*[d[k] for k in fused_args])
         elif args.case == "fused_backward":
             binding.fused_backward(*[d[k] for k in fused_args], d["grad_output"],
                                    reference_grad=False)
-        elif args.case.startswith("backward"):
+        elif args.case.startswith("backward") or args.case == "decoder_backward":
             binding.backward(d["value"], d["spatial_shapes"], d["level_start_index"],
                              d["sampling_locations"], d["attention_weights"], d["grad_output"],
                              workspace="auto" if args.case == "backward_sorted" else None)
@@ -1037,7 +1048,8 @@ def parse_args(argv=None):
                    help="skip the CPU oracle timing (it takes ~10-20 s)")
     p.add_argument("--case", choices=["step", "forward", "forward_encoder", "backward",
                                       "backward_sorted", "fused_forward", "fused_backward",
-                                      "projection"],
+                                      "projection", "projection_f32", "decoder_forward",
+                                      "decoder_backward"],
                    default="step",
                    help="time one launch type alone (for profiler captures) instead of "
                         "the full benchmark")
