@@ -31,7 +31,8 @@
  *    msda_backward_noalloc (reserved on each device with the library's device
  *    code), two device flags that record a bounded wait that ran out
  *    (msda_output_projection_check, msda_wait_check), and per-device caches of
- *    the SM count and of kernel attributes.
+ *    the SM count and of kernel attributes (the debug build adds its
+ *    registered buffers and its record of refused accesses).
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *    Work is enqueued asynchronously on it; results are ready once the stream
  *    has been synchronised.  The compute entry points neither allocate nor
@@ -392,6 +393,35 @@ msda_status msda_backward_noalloc(int64_t B, int64_t S, int64_t M, int64_t D, in
  * copies the flag to the host).
  */
 msda_status msda_wait_check(int *failed);
+
+/*
+ * Debug build.  libmsda_debug.so is this library compiled with
+ * MSDA_DEBUG_BOUNDS (build.py --debug): the same entry points, in which every
+ * gather of a value or grad_output row and every reduction into grad_value
+ * (or into the deterministic backward's integer accumulators) first checks
+ * that its bytes lie inside a buffer of the current call.  Before it launches,
+ * each compute entry point registers its buffers on its stream: readable
+ * value and grad_output, writable grad_value and the workspace.  An access
+ * outside them is skipped (a read gives zeros) and the first one is recorded.
+ * The checks stand in for a memory checker; they make the kernels several
+ * times slower.  The registered buffers are process-wide, so the debug build
+ * expects one call in flight at a time and is not for CUDA graph capture.
+ *
+ * msda_debug_bounds_check: *kind = 0 if no access has been refused since the
+ * last check, 1 for a read, 2 for a write, and *address = the first refused
+ * access's device address (0 when *kind is 0); clears the record.
+ * Synchronises with the device.  The release library returns
+ * MSDA_ERR_UNSUPPORTED (with *kind = 0, *address = 0).
+ *
+ * msda_debug_bounds_clip: from the next call on, the registered `value`
+ * buffer is taken as its first value_bytes bytes and `grad_value` as its first
+ * grad_value_bytes bytes (0: the whole buffer).  Memory past the clip stays
+ * valid; accesses there are refused as if it were not.  This lets a caller
+ * check that the checks fire, without any access outside real buffers.
+ * Release library: MSDA_ERR_UNSUPPORTED.
+ */
+msda_status msda_debug_bounds_check(int *kind, uint64_t *address);
+msda_status msda_debug_bounds_clip(uint64_t value_bytes, uint64_t grad_value_bytes);
 
 /*
  * Host-side metadata check, for callers that hold host copies of the metadata

@@ -21,7 +21,13 @@ from typing import Optional, Tuple
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIBRARY_PATH = os.path.join(_HERE, "libmsda.so")
+RELEASE_LIBRARY_PATH = os.path.join(_HERE, "libmsda.so")
+# MSDA_DEBUG_BOUNDS=1 in the environment selects the debug build, whose kernels
+# check every gather and scatter address against the call's buffers
+# (debug_bounds_check below); it is read once, when the library is loaded.
+DEBUG_LIBRARY_PATH = os.path.join(_HERE, "libmsda_debug.so")
+LIBRARY_PATH = (DEBUG_LIBRARY_PATH if os.environ.get("MSDA_DEBUG_BOUNDS", "0") not in ("", "0")
+                else RELEASE_LIBRARY_PATH)
 
 MSDA_F32, MSDA_BF16 = 0, 1
 _STATUS = {0: "MSDA_OK", 1: "MSDA_ERR_NULL_POINTER", 2: "MSDA_ERR_BAD_SHAPE",
@@ -43,6 +49,8 @@ SIGNATURES = {
     "msda_output_projection_f32": (_I32, [_I64] * 3 + [_VP] * 5),
     "msda_output_projection_check": (_I32, [ctypes.POINTER(_I32)]),
     "msda_wait_check": (_I32, [ctypes.POINTER(_I32)]),
+    "msda_debug_bounds_check": (_I32, [ctypes.POINTER(_I32), ctypes.POINTER(ctypes.c_uint64)]),
+    "msda_debug_bounds_clip": (_I32, [ctypes.c_uint64, ctypes.c_uint64]),
     "msda_check_metadata": (_I32, [_I64, _I64, _VP, _VP]),
     "msda_status_string": (ctypes.c_char_p, [_I32]),
     "msda_version": (_I32, []),
@@ -69,9 +77,10 @@ def library() -> ctypes.CDLL:
     global _LIB
     if _LIB is None:
         if not os.path.exists(LIBRARY_PATH):
+            flag = " --debug" if LIBRARY_PATH == DEBUG_LIBRARY_PATH else ""
             raise RuntimeError(
                 f"{LIBRARY_PATH} is missing: build it with "
-                "`python scale_deformable_attention_backward_b200/csrc/build.py` "
+                f"`python scale_deformable_attention_backward_b200/csrc/build.py{flag}` "
                 "(there is no fallback implementation)")
         lib = ctypes.CDLL(LIBRARY_PATH)
         for name, (res, args) in SIGNATURES.items():
@@ -467,3 +476,22 @@ def wait_failed() -> bool:
     f = ctypes.c_int(0)
     _check(library().msda_wait_check(ctypes.byref(f)), "msda_wait_check")
     return bool(f.value)
+
+
+def debug_bounds_check() -> Tuple[int, int]:
+    """Debug build: (kind, address) of the first gather (kind 1) or scatter
+    (kind 2) whose address fell outside the call's buffers since the last check,
+    (0, 0) if none; clears the record (synchronises with the device).  The
+    release library raises MSDAError(MSDA_ERR_UNSUPPORTED)."""
+    kind, address = ctypes.c_int(0), ctypes.c_uint64(0)
+    _check(library().msda_debug_bounds_check(ctypes.byref(kind), ctypes.byref(address)),
+           "msda_debug_bounds_check")
+    return kind.value, address.value
+
+
+def debug_bounds_clip(value_bytes: int = 0, grad_value_bytes: int = 0) -> None:
+    """Debug build: take the registered value / grad_value buffers of the
+    following calls as their first value_bytes / grad_value_bytes bytes (0: the
+    whole buffer), so that accesses past the clip are refused and recorded."""
+    _check(library().msda_debug_bounds_clip(value_bytes, grad_value_bytes),
+           "msda_debug_bounds_clip")

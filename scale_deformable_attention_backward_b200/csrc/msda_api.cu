@@ -1,7 +1,9 @@
 // msda_api.cu -- the C ABI declared in include/msda.h: argument validation on
 // the host, then one launch sequence on the caller's stream.  No allocation,
 // no state, no host synchronisation (except the opt-in MSDA_VALIDATE=1 check,
-// which copies the two small metadata arrays to the host).
+// which copies the two small metadata arrays to the host).  The debug build
+// (MSDA_DEBUG_BOUNDS) first registers each call's buffers for its bounds
+// checks (arm_bounds, one small stream-ordered copy).
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
@@ -145,9 +147,11 @@ msda_status msda_forward(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq,
   a.lanes = pow2_at_least(nvec);
   a.chunks = static_cast<int>((nvec + a.lanes - 1) / a.lanes);
   a.groups = B * Lq * M * a.chunks;
-  return msda::launch_forward(a, static_cast<cudaStream_t>(stream)) == cudaSuccess
-             ? MSDA_OK
-             : MSDA_ERR_CUDA;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (msda::arm_bounds(value, c.value_elems * (a.bf16 ? 2 : 4), nullptr, 0, nullptr, 0, nullptr,
+                       0, s) != cudaSuccess)
+    return MSDA_ERR_CUDA;
+  return msda::launch_forward(a, s) == cudaSuccess ? MSDA_OK : MSDA_ERR_CUDA;
 }
 
 msda_status msda_backward(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq, int64_t L,
@@ -215,6 +219,12 @@ msda_status msda_backward(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq
   a.groups = work ? B * Lq * M : 0;
   a.value_elements = c.value_elems;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const long long in_bytes = a.bf16 ? 2 : 4;
+  if (msda::arm_bounds(value, c.value_elems * in_bytes, grad_output, c.out_elems * in_bytes,
+                       grad_value, c.value_elems * 4, workspace,
+                       static_cast<long long>(workspace != nullptr ? workspace_bytes : 0),
+                       s) != cudaSuccess)
+    return MSDA_ERR_CUDA;
   const cudaError_t err = workspace != nullptr ? msda::launch_backward_sorted(a, workspace, s)
                                                : msda::launch_backward(a, s);
   return err == cudaSuccess ? MSDA_OK : MSDA_ERR_CUDA;
@@ -295,10 +305,14 @@ msda_status msda_backward_deterministic(int64_t B, int64_t S, int64_t M, int64_t
   a.lanes = pow2_at_least(D / 4);
   a.groups = work ? B * Lq * M : 0;
   a.value_elements = c.value_elems;
-  return msda::launch_backward_deterministic(a, workspace, static_cast<cudaStream_t>(stream)) ==
-                 cudaSuccess
-             ? MSDA_OK
-             : MSDA_ERR_CUDA;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const long long in_bytes = a.bf16 ? 2 : 4;
+  if (msda::arm_bounds(value, c.value_elems * in_bytes, grad_output, c.out_elems * in_bytes,
+                       grad_value, c.value_elems * 4, workspace,
+                       static_cast<long long>(workspace_bytes), s) != cudaSuccess)
+    return MSDA_ERR_CUDA;
+  return msda::launch_backward_deterministic(a, workspace, s) == cudaSuccess ? MSDA_OK
+                                                                             : MSDA_ERR_CUDA;
 }
 
 msda_status msda_output_projection(int64_t rows, int64_t c_in, int64_t c_out, const float* x,
@@ -381,9 +395,11 @@ msda_status msda_fused_forward(int64_t B, int64_t S, int64_t M, int64_t D, int64
   a.lanes = pow2_at_least(nvec);
   a.chunks = static_cast<int>((nvec + a.lanes - 1) / a.lanes);
   a.groups = B * Lq * M * a.chunks;
-  return msda::launch_fused_forward(a, static_cast<cudaStream_t>(stream)) == cudaSuccess
-             ? MSDA_OK
-             : MSDA_ERR_CUDA;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (msda::arm_bounds(value, c.value_elems * (a.bf16 ? 2 : 4), nullptr, 0, nullptr, 0, nullptr,
+                       0, s) != cudaSuccess)
+    return MSDA_ERR_CUDA;
+  return msda::launch_fused_forward(a, s) == cudaSuccess ? MSDA_OK : MSDA_ERR_CUDA;
 }
 
 msda_status msda_fused_backward(int64_t B, int64_t S, int64_t M, int64_t D, int64_t Lq,
@@ -447,9 +463,12 @@ msda_status msda_fused_backward(int64_t B, int64_t S, int64_t M, int64_t D, int6
   a.groups = work ? B * Lq * M : 0;
   a.value_elements = c.value_elems;
   a.reference_elements = ref_elems;
-  return msda::launch_fused_backward(a, static_cast<cudaStream_t>(stream)) == cudaSuccess
-             ? MSDA_OK
-             : MSDA_ERR_CUDA;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const long long in_bytes = a.bf16 ? 2 : 4;
+  if (msda::arm_bounds(value, c.value_elems * in_bytes, grad_output, c.out_elems * in_bytes,
+                       grad_value, c.value_elems * 4, nullptr, 0, s) != cudaSuccess)
+    return MSDA_ERR_CUDA;
+  return msda::launch_fused_backward(a, s) == cudaSuccess ? MSDA_OK : MSDA_ERR_CUDA;
 }
 
 msda_status msda_backward_workspace_size(int64_t B, int64_t S, int64_t M, int64_t D,

@@ -172,8 +172,9 @@ backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial
         if (use_fixed) {
 #pragma unroll
           for (int c = 0; c < E; ++c)
-            atomicAdd(abase + o + c * dq, static_cast<unsigned long long>(
-                                              __float2ll_rn(__fmul_rn(w * g[c], scale))));
+            if (in_bounds(abase + o + c * dq, 8, true))
+              atomicAdd(abase + o + c * dq, static_cast<unsigned long long>(
+                                                __float2ll_rn(__fmul_rn(w * g[c], scale))));
           return;
         }
       }

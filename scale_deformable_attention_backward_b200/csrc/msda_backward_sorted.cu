@@ -492,7 +492,7 @@ __device__ __forceinline__ Row<CPL> load_row(const float* p, const bool (&on)[CP
   Row<CPL> r = zero_row<CPL>();
 #pragma unroll
   for (int h = 0; h < CPL / 4; ++h)
-    if (on[h]) {
+    if (on[h] && in_bounds(p + 4 * h, 16, false)) {
       const float4 x = __ldg(reinterpret_cast<const float4*>(p + 4 * h));
       r.v[4 * h + 0] = x.x;
       r.v[4 * h + 1] = x.y;
@@ -506,7 +506,7 @@ template <int CPL>
 __device__ __forceinline__ void red_row(float* p, const Row<CPL>& r, const bool (&on)[CPL / 4]) {
 #pragma unroll
   for (int h = 0; h < CPL / 4; ++h)
-    if (on[h])
+    if (on[h] && in_bounds(p + 4 * h, 16, true))
       atomicAdd(reinterpret_cast<float4*>(p + 4 * h),
                 make_float4(r.v[4 * h], r.v[4 * h + 1], r.v[4 * h + 2], r.v[4 * h + 3]));
 }
@@ -694,6 +694,10 @@ cell_kernel(const float* __restrict__ value, const int64_t* __restrict__ spatial
 #pragma unroll
         for (int h = 0; h < CPL / 4; ++h)
           if (on[h]) {
+            if (!in_bounds(src + 4 * h, 16, false)) {  // debug build only: a zero slice
+              ring[stage][j][h][threadIdx.x] = make_float4(0.f, 0.f, 0.f, 0.f);
+              continue;
+            }
             const unsigned dst =
                 static_cast<unsigned>(__cvta_generic_to_shared(&ring[stage][j][h][threadIdx.x]));
             asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src + 4 * h)

@@ -17,6 +17,44 @@ namespace msda {
 
 constexpr unsigned kFullMask = 0xffffffffu;
 
+// ---------------------------------------------------------------------------
+// Bounds checks of the debug build (libmsda_debug.so, compiled with
+// MSDA_DEBUG_BOUNDS).  Every gather of a value or grad_output row and every
+// reduction into grad_value (or the deterministic path's integer accumulators)
+// first checks that its bytes lie inside a buffer of the current call, which the
+// C ABI registers before it launches (bounds_ranges: two readable, two writable).
+// An access outside them is skipped -- a read gives zeros -- and the first one
+// is recorded in bounds_error as kind << 60 | address (kind 1: read, 2: write),
+// for msda_debug_bounds_check to report.  In the release build in_bounds() is a
+// constant true and the checks compile away.
+// ---------------------------------------------------------------------------
+struct BoundsRanges {
+  unsigned long long lo[4];  // [0, 2): readable; [2, 4): writable
+  unsigned long long hi[4];  // one past the end; lo == hi: no buffer
+};
+
+#ifdef MSDA_DEBUG_BOUNDS
+extern __device__ BoundsRanges bounds_ranges;
+extern __device__ unsigned long long bounds_error;
+#endif
+
+__device__ __forceinline__ bool in_bounds(const void* p, int bytes, bool write) {
+#ifdef MSDA_DEBUG_BOUNDS
+  const unsigned long long a = reinterpret_cast<unsigned long long>(p);
+  const int first = write ? 2 : 0;
+#pragma unroll
+  for (int i = first; i < first + 2; ++i)
+    if (a >= bounds_ranges.lo[i] && a + bytes <= bounds_ranges.hi[i]) return true;
+  atomicCAS(&bounds_error, 0ull, ((write ? 2ull : 1ull) << 60) | (a & ((1ull << 60) - 1)));
+  return false;
+#else
+  (void)p;
+  (void)bytes;
+  (void)write;
+  return true;
+#endif
+}
+
 // Per-level metadata staged in shared memory.  A level whose metadata would
 // reach outside `value` is staged as 0 x 0, so none of its corners is valid and
 // it is never read.
@@ -289,6 +327,7 @@ __device__ __forceinline__ void point_sums3(const float (&dot)[4], float fx, flo
 
 // grad_value[p .. p + 3] += w * g[0 .. 3], one 16-byte vector reduction.
 __device__ __forceinline__ void scatter_row4(float* p, float w, const float (&g)[4]) {
+  if (!in_bounds(p, 16, true)) return;
   const float2 ww = make_float2(w, w);
   const float2 lo = mul2(ww, make_float2(g[0], g[1]));
   const float2 hi = mul2(ww, make_float2(g[2], g[3]));
@@ -305,7 +344,8 @@ template <>
 struct Vec<float> {
   static constexpr int N = 4;
   __device__ __forceinline__ static void load(const float* p, float (&v)[N]) {
-    const float4 r = __ldg(reinterpret_cast<const float4*>(p));
+    const float4 r = in_bounds(p, 16, false) ? __ldg(reinterpret_cast<const float4*>(p))
+                                             : make_float4(0.f, 0.f, 0.f, 0.f);
     v[0] = r.x; v[1] = r.y; v[2] = r.z; v[3] = r.w;
   }
   __device__ __forceinline__ static void store(float* p, const float (&v)[N]) {
@@ -317,7 +357,8 @@ template <>
 struct Vec<__nv_bfloat16> {
   static constexpr int N = 8;
   __device__ __forceinline__ static void load(const __nv_bfloat16* p, float (&v)[N]) {
-    const uint4 r = __ldg(reinterpret_cast<const uint4*>(p));
+    const uint4 r = in_bounds(p, 16, false) ? __ldg(reinterpret_cast<const uint4*>(p))
+                                            : make_uint4(0u, 0u, 0u, 0u);
     const unsigned w[4] = {r.x, r.y, r.z, r.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -344,7 +385,8 @@ struct Vec4;
 template <>
 struct Vec4<float> {
   __device__ __forceinline__ static void load(const float* p, float (&v)[4]) {
-    const float4 r = __ldg(reinterpret_cast<const float4*>(p));
+    const float4 r = in_bounds(p, 16, false) ? __ldg(reinterpret_cast<const float4*>(p))
+                                             : make_float4(0.f, 0.f, 0.f, 0.f);
     v[0] = r.x; v[1] = r.y; v[2] = r.z; v[3] = r.w;
   }
 };
@@ -352,7 +394,8 @@ struct Vec4<float> {
 template <>
 struct Vec4<__nv_bfloat16> {
   __device__ __forceinline__ static void load(const __nv_bfloat16* p, float (&v)[4]) {
-    const uint2 r = __ldg(reinterpret_cast<const uint2*>(p));
+    const uint2 r = in_bounds(p, 8, false) ? __ldg(reinterpret_cast<const uint2*>(p))
+                                           : make_uint2(0u, 0u);
     v[0] = __uint_as_float(r.x << 16);
     v[1] = __uint_as_float(r.x & 0xffff0000u);
     v[2] = __uint_as_float(r.y << 16);

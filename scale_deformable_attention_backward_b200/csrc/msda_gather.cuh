@@ -52,6 +52,7 @@ struct Corner<float> {
   static constexpr int N = 4;
   // acc += w * value[0..3] for one corner inside the map.
   __device__ __forceinline__ static void accumulate(const float* p, float w, float2 (&acc)[2]) {
+    if (!in_bounds(p, 16, false)) return;
     const float4 v = __ldg(reinterpret_cast<const float4*>(p));
     const float2 ww = make_float2(w, w);
     acc[0] = fma2(ww, make_float2(v.x, v.y), acc[0]);
@@ -67,10 +68,14 @@ struct Corner<float> {
                                                      const float4& w, float2 (&acc)[2]) {
     const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
     float4 v0 = z, v1 = z, v2 = z, v3 = z;
-    if (o.x >= 0) v0 = __ldg(reinterpret_cast<const float4*>(vbase + o.x));
-    if (o.y >= 0) v1 = __ldg(reinterpret_cast<const float4*>(vbase + o.y));
-    if (o.z >= 0) v2 = __ldg(reinterpret_cast<const float4*>(vbase + o.z));
-    if (o.w >= 0) v3 = __ldg(reinterpret_cast<const float4*>(vbase + o.w));
+    if (o.x >= 0 && in_bounds(vbase + o.x, 16, false))
+      v0 = __ldg(reinterpret_cast<const float4*>(vbase + o.x));
+    if (o.y >= 0 && in_bounds(vbase + o.y, 16, false))
+      v1 = __ldg(reinterpret_cast<const float4*>(vbase + o.y));
+    if (o.z >= 0 && in_bounds(vbase + o.z, 16, false))
+      v2 = __ldg(reinterpret_cast<const float4*>(vbase + o.z));
+    if (o.w >= 0 && in_bounds(vbase + o.w, 16, false))
+      v3 = __ldg(reinterpret_cast<const float4*>(vbase + o.w));
     const float4 vs[4] = {v0, v1, v2, v3};
     const float ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
@@ -90,6 +95,7 @@ struct Corner<__nv_bfloat16> {
   static constexpr int N = 8;
   __device__ __forceinline__ static void accumulate(const __nv_bfloat16* p, float w,
                                                     float2 (&acc)[4]) {
+    if (!in_bounds(p, 16, false)) return;
     const uint4 r = __ldg(reinterpret_cast<const uint4*>(p));
     const unsigned u[4] = {r.x, r.y, r.z, r.w};
     const float2 ww = make_float2(w, w);

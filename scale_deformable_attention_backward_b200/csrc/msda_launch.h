@@ -107,6 +107,15 @@ cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t stream);
 cudaError_t launch_backward_sorted(const BackwardArgs& a, void* workspace, cudaStream_t stream);
 cudaError_t launch_zero(float* p, long long n, cudaStream_t stream);
 
+// Debug build (MSDA_DEBUG_BOUNDS): registers the call's buffers, in bytes, for
+// the kernels' bounds checks, stream-ordered (msda_bounds.cu).  A null pointer
+// or a size of 0 registers nothing in that slot.  The release build does
+// nothing and returns cudaSuccess.
+cudaError_t arm_bounds(const void* value, long long value_bytes, const void* grad_output,
+                       long long grad_output_bytes, const void* grad_value,
+                       long long grad_value_bytes, const void* workspace,
+                       long long workspace_bytes, cudaStream_t stream);
+
 // Output projection Y = X Wt^T + bias on the tensor cores (msda_proj.cu):
 // rows x c_in float32 X, c_out x c_in Wt; c_in % 8 == 0, c_out % 16 == 0,
 // 16 <= c_out <= 256, all pointers 16-byte aligned (bias 4-byte, may be null).

@@ -34,6 +34,28 @@ def test_library_exports_every_declared_symbol(lib):
         assert name in binding.SIGNATURES, f"binding has no signature for {name}"
 
 
+def test_debug_library_exports_every_declared_symbol():
+    from scale_deformable_attention_backward_b200.csrc import build
+    path = build.DEBUG_LIBRARY
+    assert os.path.exists(path), "libmsda_debug.so is missing: build.py --debug builds it"
+    dbg = ctypes.CDLL(path)
+    for name in declared_functions():
+        assert hasattr(dbg, name), f"libmsda_debug.so does not export {name}"
+    # The clip is host state only: no device is touched.
+    dbg.msda_debug_bounds_clip.argtypes = [ctypes.c_uint64, ctypes.c_uint64]
+    assert dbg.msda_debug_bounds_clip(0, 0) == OK
+
+
+def test_release_library_has_no_bounds_checks(lib):
+    kind, address = ctypes.c_int(7), ctypes.c_uint64(7)
+    assert lib.msda_debug_bounds_check(ctypes.byref(kind), ctypes.byref(address)) == UNSUP
+    assert (kind.value, address.value) == (0, 0)
+    assert lib.msda_debug_bounds_check(None, None) == NULLP
+    assert lib.msda_debug_bounds_clip(16, 16) == UNSUP
+    with pytest.raises(binding.MSDAError):
+        binding.debug_bounds_check()
+
+
 def test_status_strings_and_version(lib):
     for code in range(7):
         assert lib.msda_status_string(code)
