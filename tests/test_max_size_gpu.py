@@ -160,3 +160,5 @@ def test_largest_value_block_against_closed_forms():
         assert abs(total - touched) <= 1e-9 * touched, (tag, total, touched)
         del gv, gl, ga
         torch.cuda.empty_cache()
+    del value, out
+    torch.cuda.empty_cache()                 # hand the 16 GiB back to the tests that follow
