@@ -250,6 +250,48 @@ def test_far_and_nonfinite_locations():
     G.check_backward_paths(d, inp)
 
 
+
+def test_nonfinite_value_pixels():
+    """NaN and +-Inf in value, on the first pixel of every level (the pixel a
+    point with no corner in the map would stand nearest to) and inside the maps,
+    with locations spread over [-0.3, 1.3] so that many points sit partly or
+    wholly outside.  Zero padding means a corner outside the map adds nothing,
+    so the non-finite pixels reach exactly the outputs whose points touch them:
+    the forward matches the oracle element by element, NaN and Inf pattern
+    included.  grad_value does not depend on value and matches exactly as in
+    the finite case.  grad_attn and grad_loc combine corner differences
+    (P + fx Ex + ..., Ex = gO . (V10 - V00)), so an infinite corner may give
+    NaN where the oracle's direct sum gives +-Inf; everywhere else they agree."""
+    shapes = [(6, 7), (3, 5), (2, 3)]
+    inp = random_inputs(77, B=2, M=2, D=8, K=3, shapes=shapes, Lq=61)
+    value = inp.value.copy()
+    starts = inp.level_start_index
+    value[0, starts[0]] = np.nan
+    value[0, starts[1], 0] = np.inf
+    value[0, starts[2], 1, :4] = -np.inf
+    value[1, starts[0] + 17, 1, 2:5] = np.inf
+    value[1, starts[0] + 18, 1, 3] = -np.inf
+    value[1, starts[1] + 6, 0, :] = np.nan
+    inp = dataclasses.replace(inp, value=value)
+    d = G.device_inputs(inp)
+    ref = G.oracle_forward(inp)
+    assert 0 < (~np.isfinite(ref)).mean() < 0.5      # the pixels are reached, not everywhere
+    got = G.gpu_forward(d)
+    inf = np.isinf(ref)
+    assert np.array_equal(got[inf], ref[inf])
+    G.assert_forward_f32(np.where(inf, 0.0, got), np.where(inf, 0.0, ref))  # NaN pattern, finite values
+    rv, rl, ra = G.oracle_backward(inp)
+    assert np.all(np.isfinite(rv))
+    for path in G.backward_paths(d):
+        gv, gl, ga = G.gpu_backward(d, path)
+        G.assert_backward_f32(gv, rv, f"grad_value, non-finite value ({path})")
+        for got_t, ref_t, name in ((gl, rl, "grad_sampling_locations"),
+                                   (ga, ra, "grad_attention_weights")):
+            inf = np.isinf(ref_t)
+            what = f"{name}, non-finite value ({path})"
+            assert np.all((got_t[inf] == ref_t[inf]) | np.isnan(got_t[inf])), what
+            G.assert_backward_f32(got_t[~inf], ref_t[~inf], what)
+
 def test_empty_calls():
     inp = random_inputs(9, B=2, M=2, D=8, K=2, shapes=SHAPES[0], Lq=0)
     d = G.device_inputs(inp)
