@@ -120,6 +120,7 @@ backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial
   const int lane = threadIdx.x % LANES;
   const int gi = threadIdx.x / LANES;
   const int LK = L * K;
+  const unsigned kmagic = level_magic(K);
   const int MD = M * D;  // < 2^31: one image's value block is (checked by the C ABI)
   // Point split (SPLIT > 1): SPLIT consecutive sub-warps share one group,
   // subset s taking its points s, s + SPLIT, ...  Every result of the backward is
@@ -210,7 +211,7 @@ backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ spatial
           const long long pidx = g * LK + jr;
           const float2 xy = __ldg(reinterpret_cast<const float2*>(sampling_locations) + pidx);
           const float a = __ldg(attention_weights + pidx);
-          const int l = jr / K;
+          const int l = level_of(jr, kmagic);
           const int H = lv.H[l], W = lv.W[l];
           const Cell c = locate(xy.x, xy.y, H, W);
           const float hx = 1.0f - c.fx, hy = 1.0f - c.fy;

@@ -85,6 +85,7 @@ forward_body(const T* __restrict__ value, const int64_t* __restrict__ spatial_sh
   const int gi = threadIdx.x / LANES;
   const int LK = L * K;
   const int MD = M * D;
+  const unsigned kmagic = level_magic(K);
   // Point split (SPLIT > 1, non-fused, chunks == 1): SPLIT consecutive
   // sub-warps share one group, subset s taking its points s, s + SPLIT, ...;
   // their partial sums are added with shuffles before the store.  Work units
@@ -151,14 +152,14 @@ forward_body(const T* __restrict__ value, const int64_t* __restrict__ spatial_sh
         for (int o = PC / 2; o > 0; o >>= 1) sum += __shfl_xor_sync(kFullMask, sum, o, PC);
         pa[r] = e * (1.0f / sum);
         if (live) {
-          const int l = jr / K;
+          const int l = level_of(jr, kmagic);
           const long long bq = decompose(g, chunks, M, Lq).bq;
           pxy[r] = fused_location(reference_points + (bq * L + l) * R, pxy[r], R, lv.W[l],
                                   lv.H[l], K);
         }
       }
       if (live) {
-        const int l = jr / K;
+        const int l = level_of(jr, kmagic);
         const PointSetup su = setup_point(pxy[r].x, pxy[r].y, pa[r], lv.H[l], lv.W[l], lv.start[l], MD);
         const int slot = tj * G + (tg ^ (tj & 7));
         s_off[buf][slot] = su.off;

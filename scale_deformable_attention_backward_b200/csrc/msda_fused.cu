@@ -80,6 +80,7 @@ fused_forward_kernel(const T* __restrict__ value, const int64_t* __restrict__ sp
   const int lane = threadIdx.x % LANES;
   const int gi = threadIdx.x / LANES;
   const int LK = L * K;
+  const unsigned kmagic = level_magic(K);
   const int MD = M * D;
   const long long tiles = (groups + G - 1) / G;
 
@@ -109,7 +110,7 @@ fused_forward_kernel(const T* __restrict__ value, const int64_t* __restrict__ sp
           const long long bqm = chunks == 1 ? g : g / chunks;
           const long long bq = bqm / M;
           const int i = p0 + tj;
-          const int l = i / K;
+          const int l = level_of(i, kmagic);
           const long long p = bqm * LK + i;
           const float2 off = __ldg(reinterpret_cast<const float2*>(sampling_offsets) + p);
           const float2 loc = fused_location(reference_points + (bq * L + l) * R, off, R,
@@ -182,6 +183,7 @@ fused_backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ s
   const int lane = threadIdx.x % LANES;
   const int gi = threadIdx.x / LANES;
   const int LK = L * K;
+  const unsigned kmagic = level_magic(K);
   const int MD = M * D;  // < 2^31: one image's value block is (checked by the C ABI)
   const float half_over_k = 0.5f / static_cast<float>(K);
   const long long tiles = (groups + G - 1) / G;
@@ -224,7 +226,7 @@ fused_backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ s
         int cx0 = 0, cy0 = 0;
         if (live) {
           const long long pidx = g * LK + q0 + tj;
-          const int l = (q0 + tj) / K;
+          const int l = level_of(q0 + tj, kmagic);
           const int H = lv.H[l], W = lv.W[l];
           const float2 offj = __ldg(reinterpret_cast<const float2*>(sampling_offsets) + pidx);
           const long long bq = g / M;
@@ -308,7 +310,7 @@ fused_backward_kernel(const T* __restrict__ value, const int64_t* __restrict__ s
         if (active && jl < nb) {
           const int pj = q0 + j0 + jl;
           const long long p = grp.bqm * LK + pj;
-          const int lj = pj / K;
+          const int lj = level_of(pj, kmagic);
           const float a = s_g[(j0 + jl) * G + (gi ^ ((j0 + jl) & 7))].z;
           const float dA = keep[0], s_x = keep[1], s_y = keep[2];
           sum_adA = fmaf(a, dA, sum_adA);
