@@ -9,6 +9,9 @@ against brute force (the GPU parity tests check the kernels themselves):
   sub-warp of LANES lanes, the first exchange a reduce-scatter; which lane ends
   with which point's totals.
 
+- level_of: a point's level floor(j / K) by one multiply-high with
+  m = ceil(2^32 / K), in every kernel that maps points to levels.
+
 These restate the kernels' arithmetic in Python; they are not the oracle."""
 import random
 
@@ -125,3 +128,17 @@ def test_pair_reduction_places_each_point_total_once(lanes):
                 kept[lane] = 2 * u + (1 if lane & half else 0)
     assert kept == {lane: pair_lane_point(lanes, lane) for lane in range(lanes)}
     assert sorted(kept.values()) == list(range(lanes))
+
+
+def test_level_of_is_exact_integer_division():
+    """floor(j m / 2^32) with m = floor((2^32 - 1) / K) + 1 equals j // K for every
+    j < 2^16 and every K the op accepts (1 <= K <= 64; m = 0 stands for K = 1),
+    exhaustively."""
+    import numpy as np
+
+    j = np.arange(1 << 16, dtype=np.uint64)
+    for K in range(1, 65):
+        m = 0 if K == 1 else (0xFFFFFFFF // K) + 1
+        assert m < (1 << 32)
+        got = j if m == 0 else (j * np.uint64(m)) >> np.uint64(32)
+        assert np.array_equal(got, j // np.uint64(K)), K
