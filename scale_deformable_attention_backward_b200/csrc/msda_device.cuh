@@ -114,9 +114,10 @@ __device__ __forceinline__ void pixel_coordinate(float loc, float n, float& c, f
 // The sampling geometry of one point on its level.
 // The level of point j of a group, floor(j / K), without an integer division
 // per point: with m = ceil(2^32 / K) (K >= 2), floor(j m / 2^32) = floor(j / K)
-// for 0 <= j < 2^16 and K <= 2^16, because j m / 2^32 exceeds j / K by less
-// than j / 2^32 < 2^-16, too little to reach the next multiple of 1 / K.
-// Here j < L K <= 1024.  m = 0 stands for K = 1.
+// for 0 <= j < 2^16 and K <= 2^16.  j m / 2^32 exceeds j / K by less than
+// j / 2^32 < 2^-16 <= 1 / K, while the fraction of j / K is at most 1 - 1 / K,
+// so the sum stays below the next integer.  Here j < L K <= 1024.  m = 0
+// stands for K = 1.
 __device__ __forceinline__ unsigned level_magic(int K) {
   return K > 1 ? 0xFFFFFFFFu / static_cast<unsigned>(K) + 1u : 0u;
 }
