@@ -923,6 +923,21 @@ def run_b200(args, world, rank, local):
     return result
 
 
+CASES = ("step", "forward", "forward_encoder", "backward", "backward_sorted", "fused_forward",
+         "fused_backward", "projection", "projection_f32", "decoder_forward", "decoder_backward")
+
+
+def case_workload(case: str) -> str:
+    """The workload a single-launch case (--case) runs on."""
+    if case == "forward_encoder":
+        return FORWARD_WORKLOAD
+    if case == "decoder_forward":
+        return "decoder_fp32"
+    if case == "decoder_backward":
+        return "decoder_box_train_fp32"
+    return STEP_WORKLOAD
+
+
 def run_case(args, local):
     """One launch type alone (for profiler captures): W + K launches with an L2
     flush before each, and a one-line JSON with the mean event time."""
@@ -931,15 +946,7 @@ def run_case(args, local):
 
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
-    if args.case == "forward_encoder":
-        name = FORWARD_WORKLOAD
-    elif args.case == "decoder_forward":
-        name = "decoder_fp32"
-    elif args.case == "decoder_backward":
-        name = "decoder_box_train_fp32"
-    else:
-        name = STEP_WORKLOAD
-    cfg = W.CONFIGS[name]
+    cfg = W.CONFIGS[case_workload(args.case)]
     if args.case.startswith("fused"):
         fz = W.make_fused_inputs(cfg, seed=0)
         d = {k: torch.from_numpy(getattr(fz, k)).to(device) for k in
@@ -1046,10 +1053,7 @@ def parse_args(argv=None):
     p.add_argument("--impl", choices=["b200", "reference"], default="b200")
     p.add_argument("--no-cpu-baseline", action="store_true",
                    help="skip the CPU oracle timing (it takes ~10-20 s)")
-    p.add_argument("--case", choices=["step", "forward", "forward_encoder", "backward",
-                                      "backward_sorted", "fused_forward", "fused_backward",
-                                      "projection", "projection_f32", "decoder_forward",
-                                      "decoder_backward"],
+    p.add_argument("--case", choices=list(CASES),
                    default="step",
                    help="time one launch type alone (for profiler captures) instead of "
                         "the full benchmark")

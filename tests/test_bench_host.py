@@ -90,3 +90,14 @@ def test_committed_traffic_records_name_existing_sources():
         assert rec["dram_bytes_per_launch"] > 0, key
         for name in rec["files"]:
             assert os.path.exists(os.path.join(bench.KERNEL_SOURCES, name)), (key, name)
+
+
+def test_single_launch_cases_run_on_their_workloads():
+    assert bench.case_workload("forward_encoder") == "encoder_fp32"
+    assert bench.case_workload("decoder_forward") == "decoder_fp32"
+    assert bench.case_workload("decoder_backward") == "decoder_box_train_fp32"
+    for case in ("forward", "backward", "backward_sorted", "fused_forward", "fused_backward",
+                 "projection", "projection_f32"):
+        assert bench.case_workload(case) == "encoder_train_fp32", case
+    for case in bench.CASES:
+        assert bench.case_workload(case) in W.CONFIGS
